@@ -1,0 +1,363 @@
+#!/usr/bin/env python
+"""Benchmark of the W4.4A8 linear layer (MixLLM) on B200.
+
+One step = one pass of the hot path over one batch: activation quantization
+(fp16 X -> int8 A_q + fp32 s_a) followed by the fused W4.4A8 GEMM (both
+channel sets in one launch, fp16 Y scattered by channel index).  The weights
+are quantized and packed once before timing (an offline step).
+
+Default workload: Llama-3.1-8B q_proj shape, M=512 tokens, N=K=4096, 410 of
+4096 output channels 8-bit (p10), group 128 -- synthetic seeded inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Under torchrun (N > 1) every rank runs its own
+batch with replicated weights (data parallel, no collective on the data path);
+the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from mixed_precision_quantized_act_b200 import workloads as wl  # noqa: E402
+
+METRIC = "W4.4A8 GEMM effective TOPS at M=512,N=K=4096; % of B200 int8 TC peak"
+UNIT = "TOPS"
+NOMINAL_INT8_OVER_BF16 = 4.5 / 2.25  # dense tensor peaks, ops per bf16 flop
+GEMM_SRC = os.path.join(ROOT, "mixed_precision_quantized_act_b200", "csrc", "gemm_w4w8a8.cuh")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemm_w4w8a8_traffic.json")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=wl.Q_PROJ_P10.name)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def layer_for(name):
+    for l in wl.ALL:
+        if l.name == name:
+            return l
+    raise SystemExit(f"unknown workload {name}")
+
+
+def config_of(layer, n_gpus):
+    return {"workload": layer.name, "M": layer.M, "N": layer.N, "K": layer.K, "N8": layer.N8,
+            "N4": layer.N4, "group": 128,
+            "l2": "flushed by a 256 MiB device write before every timed step",
+            "parallelism": f"dp{n_gpus} (weights replicated, M tokens per GPU)"}
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(os.path.dirname(GEMM_SRC))):
+        with open(os.path.join(os.path.dirname(GEMM_SRC), f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index, period_s=0.002):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        except Exception:
+            self.ok = False
+        return self
+
+    def _run(self):
+        nv, h = self._nv, self._h
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                for name, bit in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples), "source": "nvml unavailable"}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml, 2 ms period"}
+
+
+# ------------------------------------------------------------------ oracle leg
+
+def oracle_rate(layer, X, W, is8, target_s, max_rows=None):
+    """Time the CPU oracle (quantize + two-step GEMM) on a row sample of the
+    workload; returns (TOPS-equivalent, seconds, rows)."""
+    import oracle
+    Wq = oracle.Quantized(W, is8)  # offline weight quantization, not timed
+    rows = 1
+    t0 = time.perf_counter()
+    A, s = oracle.quantize_act(X[:rows])
+    oracle.gemm_w4w8a8(A, s, Wq)
+    t1 = time.perf_counter() - t0
+    total_rows = max_rows or layer.M
+    rows = int(max(1, min(total_rows, target_s / max(t1, 1e-6))))
+    t0 = time.perf_counter()
+    A, s = oracle.quantize_act(X[:rows])
+    oracle.gemm_w4w8a8(A, s, Wq)
+    dt = time.perf_counter() - t0
+    return 2.0 * rows * layer.N * layer.K / dt / 1e12, dt, rows
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args, layer, rank, world):
+    """The oracle as it stands, on the machine's host cores, rank 0 only."""
+    if rank != 0:
+        return
+    import oracle
+    X, W, is8 = wl.make_x(layer, args.seed), wl.make_w(layer, args.seed), wl.make_bitmap(layer, args.seed)
+    Wq = oracle.Quantized(W, is8)
+    # one step = one token row of the workload through quantize + GEMM
+    # restricted to the first 512 output channels of each set (bounded sample)
+    sub_cols = np.arange(min(layer.N, 512))
+    Wq_s = oracle.Quantized(W[sub_cols], is8[sub_cols])
+    ops_per_step = 2.0 * 1 * len(sub_cols) * layer.K
+    for i in range(args.warmup):
+        A, s = oracle.quantize_act(X[i % layer.M: i % layer.M + 1])
+        oracle.gemm_w4w8a8(A, s, Wq_s)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        A, s = oracle.quantize_act(X[i % layer.M: i % layer.M + 1])
+        oracle.gemm_w4w8a8(A, s, Wq_s)
+    dt = time.perf_counter() - t0
+    del Wq
+    value = ops_per_step * args.steps / dt / 1e12
+    sample = f"per step: 1 token row x {len(sub_cols)} output channels x K={layer.K} (quantize + two-step GEMM)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic", "config": config_of(layer, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, layer, rank, world, local_rank):
+    import torch
+    import mixed_precision_quantized_act_b200 as mx
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    mx.load()
+    stream = torch.cuda.current_stream()
+
+    X = wl.make_x(layer, args.seed + rank)
+    W, is8 = wl.make_w(layer, args.seed), wl.make_bitmap(layer, args.seed)
+    Xd = torch.from_numpy(X).to(dev)
+    p = mx.pack_weights(torch.from_numpy(W).to(dev), torch.from_numpy(is8).to(dev))
+    A_q = torch.empty((layer.M, layer.K), dtype=torch.int8, device=dev)
+    s_a = torch.empty((layer.M, layer.K // 128), dtype=torch.float32, device=dev)
+    Y = torch.empty((layer.M, layer.N), dtype=torch.float16, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def step():
+        mx.quantize_act_into(Xd, A_q, s_a, stream)
+        mx.gemm_w4w8a8_into(A_q, s_a, p, Y, stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1)
+        step()
+    mx.sync_status(stream)
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            mx.quantize_act_into(Xd, A_q, s_a, stream)
+            ev[i][1].record(stream)
+            mx.gemm_w4w8a8_into(A_q, s_a, p, Y, stream)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    mx.sync_status(stream)
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    gemm_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    quant_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    t_step = max_over_ranks(sum(step_ms) / K, world)
+    t_gemm = max_over_ranks(sum(gemm_ms) / K, world)
+    t_quant = max_over_ranks(sum(quant_ms) / K, world)
+
+    # end to end through the public API: pinned host X in, host Y out
+    Xh = torch.from_numpy(X).pin_memory()
+    Yh = torch.empty((layer.M, layer.N), dtype=torch.float16).pin_memory()
+    Ke = min(K, 200)
+    ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Ke)]
+    for _ in range(3):
+        Xd.copy_(Xh, non_blocking=True)
+        step()
+        Yh.copy_(Y, non_blocking=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(Ke):
+        flush.fill_(i & 0xFF)
+        ee[i][0].record(stream)
+        Xd.copy_(Xh, non_blocking=True)
+        step()
+        Yh.copy_(Y, non_blocking=True)
+        ee[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    t_e2e = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ee) / Ke, world)
+
+    ops = layer.ops()
+    value = ops * world / (t_step * 1e-3) / 1e12
+    gemm_tops = ops / (t_gemm * 1e-3) / 1e12
+    peaks, peak_src = measured_peaks()
+    int8_peak = peaks["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
+    traffic = None
+    try:
+        with open(TRAFFIC_FILE) as f:
+            tr = json.load(f)
+        if tr.get("source_hash") == source_hash() and tr.get("workload") == layer.name:
+            traffic = tr["dram_bytes_per_launch"]
+    except (OSError, ValueError, KeyError):
+        pass
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1:
+            rate, secs, rows = oracle_rate(layer, X, W, is8, args.cpu_seconds)
+            cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
+                   "sample": f"{rows} of {layer.M} token rows x all {layer.N} channels x K={layer.K} "
+                             f"(quantize + two-step GEMM), {secs:.1f} s single-threaded"}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded N(0,1) X with x20 outlier "
+            "columns, N(0,0.02) W, random 8-bit channel set)", "config": config_of(layer, world),
+            "gemm_kernel": {"ms": t_gemm, "tops": gemm_tops, "frac_of_int8_peak": gemm_tops / int8_peak,
+                            "frac_of_nominal_4500": gemm_tops / 4500.0},
+            "quantize_act_kernel": {"ms": t_quant,
+                                    "gbs": (layer.M * layer.K * 3 + layer.M * layer.G * 4) / (t_quant * 1e-3) / 1e9},
+            "roofline": {"bound": "tensor", "achieved": gemm_tops, "peak": int8_peak, "unit": "TOPS",
+                         "frac": gemm_tops / int8_peak, "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x 2 (nominal int8/bf16)",
+                         "algorithmic_bytes": layer.algorithmic_bytes()},
+            "cpu_baseline": cpu,
+            "e2e": {"value": ops * world / (t_e2e * 1e-3) / 1e12, "unit": UNIT,
+                    "h2d_bytes_per_step": layer.M * layer.K * 2, "d2h_bytes_per_step": layer.M * layer.N * 2},
+            "gpu_launches": 2 * K,
+            "clocks": clocks.summary(),
+        }
+    return line
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    args = parse()
+    layer = layer_for(args.workload)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, layer, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, layer, rank, world, local_rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,200 @@
+/*
+ * mixllm.h -- C ABI of the B200 (sm_100a) W4.4A8 linear layer of MixLLM.
+ *
+ * The layer computes Y[M, N] = X[M, K] . W[N, K]^T with
+ *   - activations quantized per token to int8, symmetric, in groups of 128
+ *     along K (MLSys 2026 talk notes on MixLLM, notes.yuuk.io,
+ *     §設計判断の概要; awesome-system-papers page "MixLLM (MLSys 2026)",
+ *     核心方法),
+ *   - output channels split into a 4-bit asymmetric set (uint4 codes, uint4
+ *     zero point and fp16 scale per group of 128) and an 8-bit symmetric set
+ *     (int8 codes, fp16 scale per group) by a global channel bit map
+ *     (talk notes §設計判断の概要, §グローバル混合精度探索),
+ *   - both sets multiplied on int8 tensor cores with two-step dequantization:
+ *     P = sum over a group of (W_q - z) * A_q in int32, then
+ *     acc += float(P) * s_w * s_a in fp32, with the int32-to-float step done
+ *     by the 0x4b400000 bias trick (talk notes §二段階逆量子化による int8
+ *     Tensor Core 活用, §高速 I2F 変換),
+ *   - each channel's fp16 result written to its own column of one Y
+ *     (talk notes §並列実行, fused scatter epilogue).
+ *
+ * Conventions for every entry point:
+ *   - The caller owns every buffer and every stream; the library allocates
+ *     nothing on the call path.  Device pointers are plain CUDA device
+ *     addresses on the current device.  `stream` is a cudaStream_t (NULL =
+ *     the legacy default stream).
+ *   - Calls are asynchronous on `stream` unless stated otherwise.  Argument
+ *     errors are found on the host and returned at once, with nothing
+ *     launched.  A device-side wait that gives up (a hang guard, which never
+ *     fires in correct operation) is recorded in a device status word and
+ *     reported by mixllm_sync_status().
+ *   - No call aborts the process or throws; the message of the last error
+ *     of the calling thread is available from mixllm_last_error().
+ *   - The group size is fixed at 128 (talk notes §設計判断の概要); any other
+ *     value returns MIXLLM_ERR_UNSUPPORTED.  K must be a positive multiple
+ *     of 128.
+ */
+#ifndef MIXLLM_H_
+#define MIXLLM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MIXLLM_API __attribute__((visibility("default")))
+#else
+#define MIXLLM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MIXLLM_OK = 0,
+    MIXLLM_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad size      */
+    MIXLLM_ERR_UNSUPPORTED = 2, /* group != 128, K % 128 != 0, no sm_100a  */
+    MIXLLM_ERR_CUDA = 3,        /* a CUDA runtime call failed              */
+    MIXLLM_ERR_TIMEOUT = 4      /* a device-side wait gave up              */
+} mixllm_status;
+
+#define MIXLLM_GROUP 128
+
+/* Library version (major*10000 + minor*100 + patch). */
+MIXLLM_API int mixllm_version(void);
+
+/* Message of the last error returned to the calling thread ("" if none). */
+MIXLLM_API const char *mixllm_last_error(void);
+
+/*
+ * Byte sizes of the seven packed-weight buffers for N output channels, of
+ * which N8 are 8-bit, and inner size K:
+ *   out_bytes[0] W4    uint8 [N4, K/2]   4-bit codes, two per byte
+ *   out_bytes[1] z4    uint8 [G, N4p/2]  4-bit zero points, two per byte
+ *   out_bytes[2] s_w4  fp16  [G, N4p]    4-bit set scales
+ *   out_bytes[3] idx4  int32 [N4]        output column of each 4-bit row
+ *   out_bytes[4] W8    int8  [N8, K]     8-bit codes
+ *   out_bytes[5] s_w8  fp16  [G, N8p]    8-bit set scales
+ *   out_bytes[6] idx8  int32 [N8]        output column of each 8-bit row
+ * with N4 = N - N8, G = K/128 and Np = N rounded up to a multiple of 256.
+ * The 4-bit set's footprint is 0.5 + 2.5/G bytes per weight and the 8-bit
+ * set's 1 + 2/G (talk notes §ルーフラインモデルによる性能分析), plus the
+ * padding of the scale/zero arrays to 256 channels.
+ * Host-only; touches no device.
+ */
+MIXLLM_API mixllm_status mixllm_packed_sizes(int64_t N, int64_t K, int64_t N8, int32_t group,
+                                  size_t out_bytes[7]);
+
+/*
+ * Activation quantization (one kernel): for every token m and group g of
+ * 128 columns, amax = max |x|, s_a = amax / 127 (fp32, IEEE division),
+ * A_q = clamp(round_half_even(x / s_a), -127, 127); a group whose amax is 0
+ * gets s_a = 0 and A_q = 0.  (Talk notes §設計判断の概要: activations 8-bit
+ * symmetric, group-wise RTN; the rounding and scale precision are this
+ * library's reading of "RTN".)
+ *   X_f16  device, fp16 [M, K] row-major, 16-byte aligned, read only
+ *   A_q    device, int8 [M, K] row-major, 16-byte aligned, written
+ *   s_a    device, fp32 [M, K/128] row-major, 4-byte aligned, written
+ * M = 0 is a no-op.  Asynchronous on `stream`.
+ */
+MIXLLM_API mixllm_status mixllm_quantize_act(const void *X_f16, int64_t M, int64_t K, int32_t group,
+                                  int8_t *A_q, float *s_a, void *stream);
+
+/*
+ * Offline weight quantization and pre-pack (device kernels).  The channels
+ * with is8[n] != 0 form the 8-bit symmetric set, the rest the 4-bit
+ * asymmetric set; each set is listed in ascending channel order (the pages
+ * leave the order open; it does not change Y).
+ *   4-bit, per (channel, group): lo = min(0, min w), hi = max(0, max w),
+ *     s = fp16(min((hi - lo)/15, 65504)), z = clamp(rne(-lo/s), 0, 15),
+ *     q = clamp(rne(w/s) + z, 0, 15); s == 0 gives z = q = 0.
+ *   8-bit, per (channel, group): s = fp16(min(amax/127, 65504)),
+ *     q = clamp(rne(w/s), -127, 127); s == 0 gives q = 0.
+ * Packed layout (the buffers of mixllm_packed_sizes):
+ *   W4: row r holds channel idx4[r]; in each run of 32 consecutive k, byte
+ *       i (0..15) holds code k = 32c+i in its low nibble and k = 32c+16+i
+ *       in its high nibble.
+ *   z4: zero point of row r, group g in byte g*N4p/2 + r/2, low nibble for
+ *       even r, high for odd r; padding rows are 0.
+ *   s_w4 / s_w8: scale of row r, group g at g*Np + r; padding rows are 0.
+ *   W8: row r holds channel idx8[r], int8 codes in k order.
+ * Arguments:
+ *   W     device, fp32 [N, K] row-major, 16-byte aligned, read only
+ *   is8   device, uint8 [N], the global channel bit map, read only
+ *   N8    number of nonzero is8 entries (checked on the device)
+ *   outputs: device buffers of the sizes given by mixllm_packed_sizes, each
+ *     16-byte aligned (a buffer of size 0 may be NULL).
+ * SYNCHRONOUS: waits for `stream` and returns MIXLLM_ERR_INVALID_ARG if the
+ * bit map holds a number of 8-bit channels other than N8 (then the outputs
+ * are unspecified).
+ */
+MIXLLM_API mixllm_status mixllm_pack_weights(const float *W, int64_t N, int64_t K, const uint8_t *is8,
+                                  int64_t N8, int32_t group,
+                                  uint8_t *W4, uint8_t *z4, void *s_w4_f16, int32_t *idx4,
+                                  int8_t *W8, void *s_w8_f16, int32_t *idx8, void *stream);
+
+/*
+ * The fused W4.4A8 GEMM: one launch covers both channel sets.  For each
+ * output channel n of a set and token m,
+ *   P_g = sum_{k in group g} (W_q[n,k] - z[n,g]) * A_q[m,k]   (int32 exact,
+ *         z = 0 for the 8-bit set; int8 tensor cores, tcgen05 kind::i8),
+ *   acc = sum_g float(P_g) * s_w[n,g] * s_a[m,g]  (fp32; float(P_g) by the
+ *         0x4b400000 bias trick, exact for |P_g| <= 2^22),
+ *   Y[m, idx[n]] = fp16_rn(acc).
+ * Arguments:
+ *   A_q, s_a   device, as written by mixllm_quantize_act (A_q 16-byte
+ *              aligned, K a multiple of 128)
+ *   W4, z4, s_w4, idx4, N4   the 4-bit set as written by mixllm_pack_weights
+ *   W8, s_w8, idx8, N8       the 8-bit set as written by mixllm_pack_weights
+ *              (N4 = 0 or N8 = 0 is allowed; that set's pointers may be NULL)
+ *   Y          device, fp16 [M, N4 + N8] row-major, 2-byte aligned, written;
+ *              column idx[n] receives channel n.  idx4 and idx8 together must
+ *              list every column exactly once (not checked here).
+ * The weights' packed rows are padded by the caller-provided layout only in
+ * the scale and zero arrays; nothing is read outside the buffers sized by
+ * mixllm_packed_sizes.  Asynchronous on `stream`.
+ */
+MIXLLM_API mixllm_status mixllm_gemm_w4w8a8(const int8_t *A_q, const float *s_a, int64_t M, int64_t K,
+                                 const uint8_t *W4, const uint8_t *z4, const void *s_w4_f16,
+                                 const int32_t *idx4, int64_t N4,
+                                 const int8_t *W8, const void *s_w8_f16,
+                                 const int32_t *idx8, int64_t N8,
+                                 void *Y_f16, void *stream);
+
+/*
+ * Debug path of the same kernel: writes the per-group int32 partials
+ *   P[m, idx[n], g] = sum_{k in g} (W_q[n,k] - z[n,g]) * A_q[m,k]
+ * (step 2 of the two-step dequantization, without the bias) into
+ *   P   device, int32 [M, N4 + N8, K/128], 4-byte aligned,
+ * instead of Y.  Same arguments and rules otherwise.  Slow (uncoalesced
+ * stores); for parity tests only.
+ */
+MIXLLM_API mixllm_status mixllm_gemm_debug_partials(const int8_t *A_q, const float *s_a, int64_t M, int64_t K,
+                                         const uint8_t *W4, const uint8_t *z4, const void *s_w4_f16,
+                                         const int32_t *idx4, int64_t N4,
+                                         const int8_t *W8, const void *s_w8_f16,
+                                         const int32_t *idx8, int64_t N8,
+                                         int32_t *P, void *stream);
+
+/*
+ * Waits for `stream`, then reads and clears the device status word of the
+ * current device.  Returns MIXLLM_ERR_TIMEOUT if a kernel of this library
+ * gave up a wait since the last call, MIXLLM_ERR_CUDA if the stream reports
+ * a CUDA error, MIXLLM_OK otherwise.  SYNCHRONOUS.
+ */
+MIXLLM_API mixllm_status mixllm_sync_status(void *stream);
+
+/*
+ * Self-test of the hang guard: launches one small kernel whose wait on a
+ * shared-memory barrier that nothing signals gives up after `limit_us`
+ * microseconds (1..1000000) and records MIXLLM_ERR_TIMEOUT in the device
+ * status word, leaving the context usable.  Asynchronous; read the result
+ * with mixllm_sync_status().
+ */
+MIXLLM_API mixllm_status mixllm_selftest_wait_timeout(uint32_t limit_us, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MIXLLM_H_ */

@@ -1,0 +1,24 @@
+"""MixLLM W4.4A8 linear layer for NVIDIA B200 (sm_100a).
+
+The compute path is the CUDA library ``libmixllm_b200.so`` (C ABI in
+``include/mixllm.h``); this package is its thin Python binding plus the seeded
+synthetic workloads used by the tests and the benchmark.
+"""
+from ._lib import (  # noqa: F401
+    GROUP,
+    MixLLMError,
+    PackedLinear,
+    empty_packed,
+    gemm_debug_partials,
+    gemm_w4w8a8,
+    gemm_w4w8a8_into,
+    linear,
+    load,
+    pack_weights,
+    packed_sizes,
+    quantize_act,
+    quantize_act_into,
+    selftest_wait_timeout,
+    sync_status,
+    version,
+)

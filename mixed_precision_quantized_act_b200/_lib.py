@@ -1,0 +1,217 @@
+"""Python binding of the C ABI in ``include/mixllm.h`` (ctypes).
+
+Argument marshalling only: torch provides device memory and streams; every
+step of the layer runs in the CUDA library ``libmixllm_b200.so``.  There is no
+fallback: if the library or a CUDA device is missing, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmixllm_b200.so")
+GROUP = 128
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
+_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIMEOUT"}
+
+# Every entry point declared in include/mixllm.h, with (restype, argtypes).
+_i64, _i32, _u32, _vp = ctypes.c_int64, ctypes.c_int32, ctypes.c_uint32, ctypes.c_void_p
+SIGNATURES = {
+    "mixllm_version": (ctypes.c_int, []),
+    "mixllm_last_error": (ctypes.c_char_p, []),
+    "mixllm_packed_sizes": (ctypes.c_int, [_i64, _i64, _i64, _i32, ctypes.POINTER(ctypes.c_size_t)]),
+    "mixllm_quantize_act": (ctypes.c_int, [_vp, _i64, _i64, _i32, _vp, _vp, _vp]),
+    "mixllm_pack_weights": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i64, _i32,
+                                           _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "mixllm_gemm_w4w8a8": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64,
+                                          _vp, _vp, _vp, _i64, _vp, _vp]),
+    "mixllm_gemm_debug_partials": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64,
+                                                  _vp, _vp, _vp, _i64, _vp, _vp]),
+    "mixllm_sync_status": (ctypes.c_int, [_vp]),
+    "mixllm_selftest_wait_timeout": (ctypes.c_int, [_u32, _vp]),
+}
+
+
+class MixLLMError(RuntimeError):
+    def __init__(self, status: int, where: str, msg: str):
+        super().__init__(f"{where}: {_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load the CUDA library (raises if it was not built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise RuntimeError(
+                    f"{path} is missing: build it with `python -m mixed_precision_quantized_act_b200.build`")
+            L = ctypes.CDLL(path)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(L, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = L
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        msg = load().mixllm_last_error().decode(errors="replace")
+        raise MixLLMError(status, where, msg)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return t.data_ptr() if t.numel() > 0 else None
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and t.numel() > 0 and not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+
+
+# ---------------------------------------------------------------- entry points
+
+def version() -> int:
+    return load().mixllm_version()
+
+
+def packed_sizes(N: int, K: int, N8: int, group: int = GROUP):
+    out = (ctypes.c_size_t * 7)()
+    _check(load().mixllm_packed_sizes(N, K, N8, group, out), "mixllm_packed_sizes")
+    return list(out)
+
+
+def quantize_act_into(X: torch.Tensor, A_q: torch.Tensor, s_a: torch.Tensor, stream=None):
+    _need_cuda(X, A_q, s_a)
+    assert X.dtype == torch.float16 and A_q.dtype == torch.int8 and s_a.dtype == torch.float32
+    assert X.is_contiguous() and A_q.is_contiguous() and s_a.is_contiguous()
+    M, K = X.shape
+    _check(load().mixllm_quantize_act(_ptr(X), M, K, GROUP, _ptr(A_q), _ptr(s_a), _stream(stream)),
+           "mixllm_quantize_act")
+
+
+def quantize_act(X: torch.Tensor, stream=None):
+    """X fp16 [M, K] (CUDA) -> (A_q int8 [M, K], s_a fp32 [M, K/128])."""
+    M, K = X.shape
+    A_q = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    s_a = torch.empty((M, K // GROUP), dtype=torch.float32, device=X.device)
+    quantize_act_into(X, A_q, s_a, stream)
+    return A_q, s_a
+
+
+@dataclass
+class PackedLinear:
+    """Packed weights of one W4.4A8 linear layer (device tensors)."""
+    N: int
+    K: int
+    N4: int
+    N8: int
+    W4: torch.Tensor    # uint8 [N4, K/2]
+    z4: torch.Tensor    # uint8 [G, N4p/2]
+    s_w4: torch.Tensor  # fp16 [G, N4p]
+    idx4: torch.Tensor  # int32 [N4]
+    W8: torch.Tensor    # int8 [N8, K]
+    s_w8: torch.Tensor  # fp16 [G, N8p]
+    idx8: torch.Tensor  # int32 [N8]
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in
+                   (self.W4, self.z4, self.s_w4, self.idx4, self.W8, self.s_w8, self.idx8))
+
+
+def padded(n: int) -> int:
+    return (n + 255) // 256 * 256
+
+
+def empty_packed(N: int, K: int, N8: int, device) -> PackedLinear:
+    N4, G = N - N8, K // GROUP
+    u8, i8, f16, i32 = torch.uint8, torch.int8, torch.float16, torch.int32
+    return PackedLinear(
+        N, K, N4, N8,
+        torch.empty((N4, K // 2), dtype=u8, device=device),
+        torch.empty((G, padded(N4) // 2), dtype=u8, device=device),
+        torch.empty((G, padded(N4)), dtype=f16, device=device),
+        torch.empty((N4,), dtype=i32, device=device),
+        torch.empty((N8, K), dtype=i8, device=device),
+        torch.empty((G, padded(N8)), dtype=f16, device=device),
+        torch.empty((N8,), dtype=i32, device=device),
+    )
+
+
+def pack_weights(W: torch.Tensor, is8: torch.Tensor, stream=None) -> PackedLinear:
+    """W fp32 [N, K] and the channel bit map uint8 [N] (CUDA) -> PackedLinear.
+    Synchronous (offline step)."""
+    _need_cuda(W, is8)
+    assert W.dtype == torch.float32 and W.is_contiguous()
+    assert is8.dtype == torch.uint8 and is8.is_contiguous()
+    N, K = W.shape
+    N8 = int((is8 != 0).sum().item())
+    p = empty_packed(N, K, N8, W.device)
+    sizes = packed_sizes(N, K, N8)
+    got = [t.numel() * t.element_size() for t in (p.W4, p.z4, p.s_w4, p.idx4, p.W8, p.s_w8, p.idx8)]
+    assert got == sizes, (got, sizes)
+    _check(load().mixllm_pack_weights(_ptr(W), N, K, _ptr(is8), N8, GROUP, _ptr(p.W4), _ptr(p.z4),
+                                      _ptr(p.s_w4), _ptr(p.idx4), _ptr(p.W8), _ptr(p.s_w8),
+                                      _ptr(p.idx8), _stream(stream)), "mixllm_pack_weights")
+    return p
+
+
+def gemm_w4w8a8_into(A_q, s_a, p: PackedLinear, Y, stream=None):
+    _need_cuda(A_q, s_a, Y)
+    M, K = A_q.shape
+    assert K == p.K and Y.shape == (M, p.N) and Y.dtype == torch.float16 and Y.is_contiguous()
+    _check(load().mixllm_gemm_w4w8a8(_ptr(A_q), _ptr(s_a), M, K, _ptr(p.W4), _ptr(p.z4), _ptr(p.s_w4),
+                                     _ptr(p.idx4), p.N4, _ptr(p.W8), _ptr(p.s_w8), _ptr(p.idx8), p.N8,
+                                     _ptr(Y), _stream(stream)), "mixllm_gemm_w4w8a8")
+
+
+def gemm_w4w8a8(A_q, s_a, p: PackedLinear, stream=None) -> torch.Tensor:
+    Y = torch.empty((A_q.shape[0], p.N), dtype=torch.float16, device=A_q.device)
+    gemm_w4w8a8_into(A_q, s_a, p, Y, stream)
+    return Y
+
+
+def gemm_debug_partials(A_q, s_a, p: PackedLinear, stream=None) -> torch.Tensor:
+    """Per-group int32 partials P [M, N, K/128] (debug path of the fused kernel)."""
+    _need_cuda(A_q, s_a)
+    M, K = A_q.shape
+    P = torch.zeros((M, p.N, K // GROUP), dtype=torch.int32, device=A_q.device)
+    _check(load().mixllm_gemm_debug_partials(_ptr(A_q), _ptr(s_a), M, K, _ptr(p.W4), _ptr(p.z4),
+                                             _ptr(p.s_w4), _ptr(p.idx4), p.N4, _ptr(p.W8), _ptr(p.s_w8),
+                                             _ptr(p.idx8), p.N8, _ptr(P), _stream(stream)),
+           "mixllm_gemm_debug_partials")
+    return P
+
+
+def linear(X: torch.Tensor, p: PackedLinear, stream=None) -> torch.Tensor:
+    """The whole layer: quantize X then run the fused GEMM."""
+    A_q, s_a = quantize_act(X, stream)
+    return gemm_w4w8a8(A_q, s_a, p, stream)
+
+
+def sync_status(stream=None):
+    _check(load().mixllm_sync_status(_stream(stream)), "mixllm_sync_status")
+
+
+def selftest_wait_timeout(limit_us: int, stream=None):
+    _check(load().mixllm_selftest_wait_timeout(limit_us, _stream(stream)), "mixllm_selftest_wait_timeout")

@@ -1,0 +1,46 @@
+// launch.h -- host-side launchers of the library's kernels (internal).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace mixllm {
+
+cudaError_t launch_quantize_act(const void *X, int64_t M, int64_t K, int8_t *A_q, float *s_a,
+                                cudaStream_t stream);
+
+cudaError_t launch_split_channels(const uint8_t *is8, int64_t N, int64_t N8, int32_t *idx4, int32_t *idx8,
+                                  cudaStream_t stream);
+
+cudaError_t launch_pack_w4(const float *W, int64_t N, int64_t K, const int32_t *idx4, int64_t N4, int64_t N4p,
+                           uint8_t *W4, uint8_t *z4, void *s_w4, cudaStream_t stream);
+
+cudaError_t launch_pack_w8(const float *W, int64_t N, int64_t K, const int32_t *idx8, int64_t N8, int64_t N8p,
+                           int8_t *W8, void *s_w8, cudaStream_t stream);
+
+struct GemmArgs {
+  const int8_t *A_q;
+  const float *s_a;
+  int64_t M, K;
+  const uint8_t *W4;
+  const uint8_t *z4;
+  const void *s_w4;
+  const int32_t *idx4;
+  int64_t N4;
+  const int8_t *W8;
+  const void *s_w8;
+  const int32_t *idx8;
+  int64_t N8;
+  void *Y;     // fp16 [M, N4 + N8]
+  int32_t *P;  // debug partials [M, N, G] or null
+};
+
+// Returns a CUDA error, or cudaErrorNotSupported when the tensor-map encoder
+// is unavailable.  *msg receives a static description on failure.
+cudaError_t launch_gemm_w4w8a8(const GemmArgs &a, cudaStream_t stream, const char **msg);
+
+cudaError_t launch_selftest_wait_timeout(uint32_t limit_us, cudaStream_t stream);
+
+int64_t padded_channels(int64_t n);  // n rounded up to a multiple of 256
+
+}  // namespace mixllm

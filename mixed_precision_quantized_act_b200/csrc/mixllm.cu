@@ -1,0 +1,227 @@
+// mixllm.cu -- the C ABI declared in include/mixllm.h.  One translation unit:
+// it includes the kernels so that they share the device status word.
+//
+// Host code here only validates arguments, encodes TMA descriptors and
+// launches kernels; every step of the layer's arithmetic runs on the GPU.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/mixllm.h"
+#include "gemm_w4w8a8.cuh"
+#include "launch.h"
+#include "quant.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+mixllm_status fail(mixllm_status st, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+mixllm_status ok() {
+  g_last_error[0] = '\0';
+  return MIXLLM_OK;
+}
+
+mixllm_status cuda_fail(cudaError_t e, const char *what) {
+  return fail(MIXLLM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shape checks shared by the entry points.
+mixllm_status check_k(int64_t K, int32_t group) {
+  if (group != MIXLLM_GROUP) return fail(MIXLLM_ERR_UNSUPPORTED, "group size %d is not supported (only 128)", group);
+  if (K <= 0 || K % MIXLLM_GROUP != 0)
+    return fail(MIXLLM_ERR_UNSUPPORTED, "K = %lld must be a positive multiple of 128", static_cast<long long>(K));
+  if (K > (1ll << 30)) return fail(MIXLLM_ERR_INVALID_ARG, "K = %lld is too large", static_cast<long long>(K));
+  return MIXLLM_OK;
+}
+
+mixllm_status check_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0)
+    return fail(MIXLLM_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a only", dev, major,
+                minor);
+  return MIXLLM_OK;
+}
+
+mixllm_status gemm_common(const int8_t *A_q, const float *s_a, int64_t M, int64_t K, const uint8_t *W4,
+                          const uint8_t *z4, const void *s_w4, const int32_t *idx4, int64_t N4, const int8_t *W8,
+                          const void *s_w8, const int32_t *idx8, int64_t N8, void *Y, int32_t *P, void *stream) {
+  mixllm_status st = check_k(K, MIXLLM_GROUP);
+  if (st != MIXLLM_OK) return st;
+  if (M < 0 || N4 < 0 || N8 < 0) return fail(MIXLLM_ERR_INVALID_ARG, "negative size");
+  if (M > 0x7FFFFFFF || N4 + N8 > 0x7FFFFFF0)
+    return fail(MIXLLM_ERR_INVALID_ARG, "M or N beyond the supported 2^31 range");
+  if (M == 0 || N4 + N8 == 0) return ok();
+  if (!A_q || !s_a || !(Y || P)) return fail(MIXLLM_ERR_INVALID_ARG, "null A_q, s_a or output");
+  if (!aligned(A_q, 16)) return fail(MIXLLM_ERR_INVALID_ARG, "A_q must be 16-byte aligned");
+  if (!aligned(s_a, 4)) return fail(MIXLLM_ERR_INVALID_ARG, "s_a must be 4-byte aligned");
+  if (Y && !aligned(Y, 2)) return fail(MIXLLM_ERR_INVALID_ARG, "Y must be 2-byte aligned");
+  if (P && !aligned(P, 4)) return fail(MIXLLM_ERR_INVALID_ARG, "P must be 4-byte aligned");
+  if (N4 > 0) {
+    if (!W4 || !z4 || !s_w4 || !idx4) return fail(MIXLLM_ERR_INVALID_ARG, "null 4-bit set buffer");
+    if (!aligned(W4, 16) || !aligned(z4, 16) || !aligned(s_w4, 16) || !aligned(idx4, 4))
+      return fail(MIXLLM_ERR_INVALID_ARG, "4-bit set buffers must be 16-byte aligned (idx4: 4)");
+  }
+  if (N8 > 0) {
+    if (!W8 || !s_w8 || !idx8) return fail(MIXLLM_ERR_INVALID_ARG, "null 8-bit set buffer");
+    if (!aligned(W8, 16) || !aligned(s_w8, 16) || !aligned(idx8, 4))
+      return fail(MIXLLM_ERR_INVALID_ARG, "8-bit set buffers must be 16-byte aligned (idx8: 4)");
+  }
+  st = check_device();
+  if (st != MIXLLM_OK) return st;
+  mixllm::GemmArgs a{A_q, s_a, M, K, W4, z4, s_w4, idx4, N4, W8, s_w8, idx8, N8, Y, P};
+  const char *msg = "";
+  cudaError_t e = mixllm::launch_gemm_w4w8a8(a, static_cast<cudaStream_t>(stream), &msg);
+  if (e == cudaErrorNotSupported) return fail(MIXLLM_ERR_UNSUPPORTED, "%s", msg);
+  if (e != cudaSuccess) return fail(MIXLLM_ERR_CUDA, "%s: %s", msg, cudaGetErrorString(e));
+  return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+int mixllm_version(void) { return 100; }
+
+const char *mixllm_last_error(void) { return g_last_error; }
+
+mixllm_status mixllm_packed_sizes(int64_t N, int64_t K, int64_t N8, int32_t group, size_t out_bytes[7]) {
+  mixllm_status st = check_k(K, group);
+  if (st != MIXLLM_OK) return st;
+  if (!out_bytes) return fail(MIXLLM_ERR_INVALID_ARG, "null out_bytes");
+  if (N < 0 || N8 < 0 || N8 > N) return fail(MIXLLM_ERR_INVALID_ARG, "need 0 <= N8 <= N");
+  const int64_t N4 = N - N8, G = K / MIXLLM_GROUP;
+  const int64_t N4p = mixllm::padded_channels(N4), N8p = mixllm::padded_channels(N8);
+  out_bytes[0] = static_cast<size_t>(N4 * (K / 2));
+  out_bytes[1] = static_cast<size_t>(G * (N4p / 2));
+  out_bytes[2] = static_cast<size_t>(G * N4p * 2);
+  out_bytes[3] = static_cast<size_t>(N4 * 4);
+  out_bytes[4] = static_cast<size_t>(N8 * K);
+  out_bytes[5] = static_cast<size_t>(G * N8p * 2);
+  out_bytes[6] = static_cast<size_t>(N8 * 4);
+  return ok();
+}
+
+mixllm_status mixllm_quantize_act(const void *X_f16, int64_t M, int64_t K, int32_t group, int8_t *A_q, float *s_a,
+                                  void *stream) {
+  mixllm_status st = check_k(K, group);
+  if (st != MIXLLM_OK) return st;
+  if (M < 0) return fail(MIXLLM_ERR_INVALID_ARG, "M < 0");
+  if (M == 0) return ok();
+  if (!X_f16 || !A_q || !s_a) return fail(MIXLLM_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(X_f16, 16) || !aligned(A_q, 16) || !aligned(s_a, 4))
+    return fail(MIXLLM_ERR_INVALID_ARG, "X and A_q must be 16-byte aligned, s_a 4-byte aligned");
+  st = check_device();
+  if (st != MIXLLM_OK) return st;
+  cudaError_t e = mixllm::launch_quantize_act(X_f16, M, K, A_q, s_a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "quantize_act launch");
+  return ok();
+}
+
+mixllm_status mixllm_pack_weights(const float *W, int64_t N, int64_t K, const uint8_t *is8, int64_t N8,
+                                  int32_t group, uint8_t *W4, uint8_t *z4, void *s_w4_f16, int32_t *idx4,
+                                  int8_t *W8, void *s_w8_f16, int32_t *idx8, void *stream) {
+  mixllm_status st = check_k(K, group);
+  if (st != MIXLLM_OK) return st;
+  if (N < 0 || N8 < 0 || N8 > N) return fail(MIXLLM_ERR_INVALID_ARG, "need 0 <= N8 <= N");
+  if (N > 0x7FFFFFF0) return fail(MIXLLM_ERR_INVALID_ARG, "N beyond the supported range");
+  if (N == 0) return ok();
+  const int64_t N4 = N - N8;
+  if (!W || !is8) return fail(MIXLLM_ERR_INVALID_ARG, "null W or is8");
+  if (!aligned(W, 16)) return fail(MIXLLM_ERR_INVALID_ARG, "W must be 16-byte aligned");
+  if (N4 > 0 && (!W4 || !z4 || !s_w4_f16 || !idx4)) return fail(MIXLLM_ERR_INVALID_ARG, "null 4-bit output");
+  if (N8 > 0 && (!W8 || !s_w8_f16 || !idx8)) return fail(MIXLLM_ERR_INVALID_ARG, "null 8-bit output");
+  if ((W4 && !aligned(W4, 16)) || (z4 && !aligned(z4, 16)) || (s_w4_f16 && !aligned(s_w4_f16, 16)) ||
+      (W8 && !aligned(W8, 16)) || (s_w8_f16 && !aligned(s_w8_f16, 16)) || (idx4 && !aligned(idx4, 4)) ||
+      (idx8 && !aligned(idx8, 4)))
+    return fail(MIXLLM_ERR_INVALID_ARG, "packed outputs must be 16-byte aligned (idx: 4)");
+  st = check_device();
+  if (st != MIXLLM_OK) return st;
+  // clear any stale status first so a bad bit map is attributed to this call
+  st = mixllm_sync_status(stream);
+  if (st != MIXLLM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = mixllm::launch_split_channels(is8, N, N8, idx4, idx8, s);
+  if (e != cudaSuccess) return cuda_fail(e, "split_channels launch");
+  if (N4 > 0) {
+    e = mixllm::launch_pack_w4(W, N, K, idx4, N4, mixllm::padded_channels(N4), W4, z4, s_w4_f16, s);
+    if (e != cudaSuccess) return cuda_fail(e, "pack_w4 launch");
+  }
+  if (N8 > 0) {
+    e = mixllm::launch_pack_w8(W, N, K, idx8, N8, mixllm::padded_channels(N8), W8, s_w8_f16, s);
+    if (e != cudaSuccess) return cuda_fail(e, "pack_w8 launch");
+  }
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "pack synchronize");
+  int status = 0;
+  e = cudaMemcpyFromSymbol(&status, mixllm::g_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (status != 0) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(mixllm::g_status, &zero, sizeof(int));
+    if (status == mixllm::kStatusBadBitmap)
+      return fail(MIXLLM_ERR_INVALID_ARG, "the bit map does not flag exactly N8 = %lld channels",
+                  static_cast<long long>(N8));
+    return fail(MIXLLM_ERR_TIMEOUT, "a device wait gave up during the pack");
+  }
+  return ok();
+}
+
+mixllm_status mixllm_gemm_w4w8a8(const int8_t *A_q, const float *s_a, int64_t M, int64_t K, const uint8_t *W4,
+                                 const uint8_t *z4, const void *s_w4_f16, const int32_t *idx4, int64_t N4,
+                                 const int8_t *W8, const void *s_w8_f16, const int32_t *idx8, int64_t N8,
+                                 void *Y_f16, void *stream) {
+  if (!Y_f16 && M > 0 && N4 + N8 > 0) return fail(MIXLLM_ERR_INVALID_ARG, "null Y");
+  return gemm_common(A_q, s_a, M, K, W4, z4, s_w4_f16, idx4, N4, W8, s_w8_f16, idx8, N8, Y_f16, nullptr, stream);
+}
+
+mixllm_status mixllm_gemm_debug_partials(const int8_t *A_q, const float *s_a, int64_t M, int64_t K,
+                                         const uint8_t *W4, const uint8_t *z4, const void *s_w4_f16,
+                                         const int32_t *idx4, int64_t N4, const int8_t *W8, const void *s_w8_f16,
+                                         const int32_t *idx8, int64_t N8, int32_t *P, void *stream) {
+  if (!P && M > 0 && N4 + N8 > 0) return fail(MIXLLM_ERR_INVALID_ARG, "null P");
+  return gemm_common(A_q, s_a, M, K, W4, z4, s_w4_f16, idx4, N4, W8, s_w8_f16, idx8, N8, nullptr, P, stream);
+}
+
+mixllm_status mixllm_sync_status(void *stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  int status = 0;
+  e = cudaMemcpyFromSymbol(&status, mixllm::g_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (status != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(mixllm::g_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "status clear");
+    if (status == mixllm::kStatusTimeout) return fail(MIXLLM_ERR_TIMEOUT, "a device-side wait gave up");
+    return fail(MIXLLM_ERR_INVALID_ARG, "device reported status %d", status);
+  }
+  return ok();
+}
+
+mixllm_status mixllm_selftest_wait_timeout(uint32_t limit_us, void *stream) {
+  if (limit_us < 1 || limit_us > 1000000) return fail(MIXLLM_ERR_INVALID_ARG, "limit_us must be in 1..1000000");
+  mixllm_status st = check_device();
+  if (st != MIXLLM_OK) return st;
+  cudaError_t e = mixllm::launch_selftest_wait_timeout(limit_us, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+  return ok();
+}
+
+}  // extern "C"

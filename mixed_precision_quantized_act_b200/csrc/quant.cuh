@@ -1,0 +1,279 @@
+// quant.cuh -- activation quantization, offline weight pack, and the
+// hang-guard self-test kernel.
+//
+// Sources: MLSys 2026 talk notes on MixLLM (notes.yuuk.io), §設計判断の概要
+// (activations 8-bit symmetric group-wise RTN; weights 4-bit asymmetric with
+// group 128, salient channels 8-bit symmetric) and §ソフトウェアパイプライン
+// (weights packed and interleaved offline so no permutation runs at run time).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "launch.h"
+#include "ptx_sm100.cuh"
+
+namespace mixllm {
+
+// ---------------------------------------------------------------------------
+// Activation quantization.  One half-warp per (token m, group g): 16 lanes x
+// 8 fp16 = the 128 values of the group, loaded as one 16-byte vector per lane.
+// amax over the group, s_a = amax / 127 (IEEE division, fp32),
+// q = clamp(round_half_even(x / s_a), -127, 127); amax == 0 gives s_a = q = 0.
+// The division is the correctly rounded one (not a reciprocal multiply) so
+// that the codes are the same as a plain CPU evaluation of the definition.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) quantize_act_kernel(const __half *__restrict__ X, int64_t M, int64_t K,
+                                                           int8_t *__restrict__ A_q, float *__restrict__ s_a) {
+  const int64_t G = K >> 7;
+  const int64_t total = M * G;
+  const int lane16 = threadIdx.x & 15;
+  const unsigned mask = 0xFFFFu << (threadIdx.x & 16);
+  const int64_t stride = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 4;
+  for (int64_t hw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4; hw < total; hw += stride) {
+    const int64_t m = hw / G, g = hw - m * G;
+    const int64_t off = m * K + (g << 7) + lane16 * 8;
+    const uint4 raw = *reinterpret_cast<const uint4 *>(X + off);
+    const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw);
+    float x[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(h2[i]);
+      x[2 * i] = f.x;
+      x[2 * i + 1] = f.y;
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(mask, amax, o));
+    const float s = __fdiv_rn(amax, 127.0f);
+    uint32_t packed[2] = {0u, 0u};
+    if (s != 0.0f) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        int q = __float2int_rn(__fdiv_rn(x[i], s));
+        q = max(-127, min(127, q));
+        packed[i >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << ((i & 3) * 8);
+      }
+    }
+    *reinterpret_cast<uint2 *>(A_q + off) = make_uint2(packed[0], packed[1]);
+    if (lane16 == 0) s_a[m * G + g] = s;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Channel split: one block scans the bit map and lists the 8-bit channels and
+// the 4-bit channels, each in ascending order.  Writes stay inside idx8[N8]
+// and idx4[N - N8] even if the map holds a different count, which is then
+// recorded in the status word.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) split_channels_kernel(const uint8_t *__restrict__ is8, int64_t N, int64_t N8,
+                                                              int32_t *__restrict__ idx4, int32_t *__restrict__ idx8) {
+  __shared__ int warp_cnt[32];
+  __shared__ int warp_off[32];
+  __shared__ int64_t seen8;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) seen8 = 0;
+  __syncthreads();
+  for (int64_t start = 0; start < N; start += 1024) {
+    const int64_t n = start + tid;
+    const int f = (n < N && is8[n] != 0) ? 1 : 0;
+    const unsigned b = __ballot_sync(0xFFFFFFFFu, f);
+    const int before_in_warp = __popc(b & ((1u << lane) - 1u));
+    if (lane == 0) warp_cnt[warp] = __popc(b);
+    __syncthreads();
+    if (warp == 0) {
+      const int c = warp_cnt[lane];
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      warp_off[lane] = incl - c;
+    }
+    __syncthreads();
+    const int64_t pre8 = seen8 + warp_off[warp] + before_in_warp;  // 8-bit channels before n
+    if (n < N) {
+      if (f) {
+        if (pre8 < N8) idx8[pre8] = static_cast<int32_t>(n);
+      } else {
+        const int64_t pre4 = n - pre8;
+        if (pre4 < N - N8) idx4[pre4] = static_cast<int32_t>(n);
+      }
+    }
+    __syncthreads();
+    if (tid == 0) seen8 += warp_off[31] + warp_cnt[31];
+    __syncthreads();
+  }
+  if (tid == 0 && seen8 != N8) record_status(kStatusBadBitmap);
+}
+
+__device__ __forceinline__ float warp_min(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+// ---------------------------------------------------------------------------
+// 4-bit asymmetric pack.  One warp per (pair of packed rows, group): the two
+// rows share the zero-point byte.  Lane l writes packed bytes 2l and 2l+1 of
+// the row's 64-byte group slice; byte b = 16c + i of a 32-k run c holds codes
+// k = 32c + i (low nibble) and k = 32c + 16 + i (high nibble).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) pack_w4_kernel(const float *__restrict__ W, int64_t N, int64_t K,
+                                                      const int32_t *__restrict__ idx4, int64_t N4, int64_t N4p,
+                                                      uint8_t *__restrict__ W4, uint8_t *__restrict__ z4,
+                                                      __half *__restrict__ s_w4) {
+  const int64_t G = K >> 7;
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= (N4p >> 1) * G) return;
+  const int64_t p = wid / G, g = wid - p * G;
+  uint32_t zpair = 0;
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int64_t r = 2 * p + e;
+    // a channel index outside [0, N) (a bit map that disagrees with N8) packs as zeros
+    const int64_t n = r < N4 ? static_cast<int64_t>(idx4[r]) : -1;
+    if (r < N4) {
+      const float *w = W + (n >= 0 && n < N ? n : 0) * K + (g << 7);
+      const float keep = (n >= 0 && n < N) ? 1.0f : 0.0f;
+      const int c = lane >> 3, i0 = (2 * lane) & 15;
+      const float v[4] = {keep * w[32 * c + i0], keep * w[32 * c + 16 + i0], keep * w[32 * c + i0 + 1],
+                          keep * w[32 * c + 16 + i0 + 1]};
+      float lo = 0.0f, hi = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        lo = fminf(lo, v[i]);
+        hi = fmaxf(hi, v[i]);
+      }
+      lo = warp_min(lo);
+      hi = warp_max(hi);
+      const float sc = fminf(__fdiv_rn(__fsub_rn(hi, lo), 15.0f), 65504.0f);
+      const __half sh = __float2half_rn(sc);
+      const float sf = __half2float(sh);
+      int z = 0;
+      uint32_t q[4] = {0u, 0u, 0u, 0u};
+      if (sf != 0.0f) {
+        z = max(0, min(15, __float2int_rn(__fdiv_rn(-lo, sf))));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) q[i] = static_cast<uint32_t>(max(0, min(15, __float2int_rn(__fdiv_rn(v[i], sf)) + z)));
+      }
+      const uint32_t two = (q[0] | (q[1] << 4)) | ((q[2] | (q[3] << 4)) << 8);
+      *reinterpret_cast<uint16_t *>(W4 + r * (K >> 1) + (g << 6) + 2 * lane) = static_cast<uint16_t>(two);
+      if (lane == 0) s_w4[g * N4p + r] = sh;
+      zpair |= static_cast<uint32_t>(z) << (4 * e);
+    } else if (lane == 0) {
+      s_w4[g * N4p + r] = __float2half_rn(0.0f);
+    }
+  }
+  if (lane == 0) z4[g * (N4p >> 1) + p] = static_cast<uint8_t>(zpair);
+}
+
+// ---------------------------------------------------------------------------
+// 8-bit symmetric pack.  One warp per (row, group); lane l quantizes k = 4l..4l+3.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) pack_w8_kernel(const float *__restrict__ W, int64_t N, int64_t K,
+                                                      const int32_t *__restrict__ idx8, int64_t N8, int64_t N8p,
+                                                      int8_t *__restrict__ W8, __half *__restrict__ s_w8) {
+  const int64_t G = K >> 7;
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= N8p * G) return;
+  const int64_t r = wid / G, g = wid - r * G;
+  if (r >= N8) {
+    if (lane == 0) s_w8[g * N8p + r] = __float2half_rn(0.0f);
+    return;
+  }
+  const int64_t n = idx8[r];
+  const bool n_ok = n >= 0 && n < N;  // an index outside [0, N) packs as zeros
+  const float4 v4 = n_ok ? *reinterpret_cast<const float4 *>(W + n * K + (g << 7) + 4 * lane)
+                         : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  amax = warp_max(amax);
+  const float sc = fminf(__fdiv_rn(amax, 127.0f), 65504.0f);
+  const __half sh = __float2half_rn(sc);
+  const float sf = __half2float(sh);
+  uint32_t packed = 0;
+  if (sf != 0.0f) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int q = max(-127, min(127, __float2int_rn(__fdiv_rn(v[i], sf))));
+      packed |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * i);
+    }
+  }
+  *reinterpret_cast<uint32_t *>(W8 + r * K + (g << 7) + 4 * lane) = packed;
+  if (lane == 0) s_w8[g * N8p + r] = sh;
+}
+
+// ---------------------------------------------------------------------------
+// Hang-guard self-test: thread 0 waits on a barrier that nothing signals; the
+// bounded wait gives up and records a timeout.  No copy or MMA is in flight.
+// ---------------------------------------------------------------------------
+__global__ void selftest_wait_kernel(long long limit_cycles) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, &abort_flag, limit_cycles);
+  __syncthreads();
+}
+
+int64_t padded_channels(int64_t n) { return (n + 255) / 256 * 256; }
+
+static int grid_for(int64_t threads_needed, int block) {
+  const int64_t b = (threads_needed + block - 1) / block;
+  return static_cast<int>(b < 1 ? 1 : (b > (1ll << 30) ? (1ll << 30) : b));
+}
+
+cudaError_t launch_quantize_act(const void *X, int64_t M, int64_t K, int8_t *A_q, float *s_a, cudaStream_t stream) {
+  const int64_t groups = M * (K >> 7);
+  const int64_t blocks = (groups + 15) / 16;
+  const int grid = static_cast<int>(blocks < 148 * 64 ? blocks : 148 * 64);
+  quantize_act_kernel<<<grid, 256, 0, stream>>>(static_cast<const __half *>(X), M, K, A_q, s_a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_split_channels(const uint8_t *is8, int64_t N, int64_t N8, int32_t *idx4, int32_t *idx8,
+                                  cudaStream_t stream) {
+  split_channels_kernel<<<1, 1024, 0, stream>>>(is8, N, N8, idx4, idx8);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_w4(const float *W, int64_t N, int64_t K, const int32_t *idx4, int64_t N4, int64_t N4p,
+                           uint8_t *W4, uint8_t *z4, void *s_w4, cudaStream_t stream) {
+  const int64_t warps = (N4p / 2) * (K >> 7);
+  pack_w4_kernel<<<grid_for(warps * 32, 256), 256, 0, stream>>>(W, N, K, idx4, N4, N4p, W4, z4,
+                                                                 static_cast<__half *>(s_w4));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_w8(const float *W, int64_t N, int64_t K, const int32_t *idx8, int64_t N8, int64_t N8p,
+                           int8_t *W8, void *s_w8, cudaStream_t stream) {
+  const int64_t warps = N8p * (K >> 7);
+  pack_w8_kernel<<<grid_for(warps * 32, 256), 256, 0, stream>>>(W, N, K, idx8, N8, N8p, W8,
+                                                                 static_cast<__half *>(s_w8));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_wait_timeout(uint32_t limit_us, cudaStream_t stream) {
+  // SM clocks stay below 2.1 GHz, so 2100 cycles per microsecond is an upper bound.
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(static_cast<long long>(limit_us) * 2100ll);
+  return cudaGetLastError();
+}
+
+}  // namespace mixllm

@@ -1,0 +1,117 @@
+"""The C-ABI library loads, exports every declared entry point, and rejects bad
+arguments on the host before touching a device (CPU only, no compute calls).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mixed_precision_quantized_act_b200 import _lib
+from mixed_precision_quantized_act_b200 import build as libbuild
+from mixed_precision_quantized_act_b200 import workloads as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mixllm.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    libbuild.build()
+    return _lib.load()
+
+
+def declared_entry_points():
+    with open(HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"MIXLLM_API\s+[\w\s\*]*?\b(mixllm_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_entry_points()
+    for required in ("mixllm_quantize_act", "mixllm_pack_weights", "mixllm_gemm_w4w8a8",
+                     "mixllm_gemm_debug_partials", "mixllm_packed_sizes", "mixllm_last_error",
+                     "mixllm_sync_status"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_entry_points()
+    assert names
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(_lib.SIGNATURES), "binding and header disagree"
+
+
+def test_library_has_no_runtime_dependency_on_a_gpu_driver():
+    # static CUDA runtime; the driver is looked up lazily
+    import subprocess
+    out = subprocess.run(["ldd", _lib.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out and "libcudart.so" not in out
+
+
+def test_packed_sizes_footprint(L):
+    N, K, N8 = 4096, 4096, 410
+    s = _lib.packed_sizes(N, K, N8)
+    N4, G = N - N8, K // 128
+    N4p, N8p = 3840, 512
+    assert s == [N4 * K // 2, G * N4p // 2, G * N4p * 2, N4 * 4, N8 * K, G * N8p * 2, N8 * 4]
+    # without padding the per-weight footprints are the pages' 0.5 + 2.5/G and 1 + 2/G
+    s2 = _lib.packed_sizes(512, 1024, 256)
+    assert (s2[0] + s2[1] + s2[2]) / (256 * 1024) == 0.5 + 2.5 / 128
+    assert (s2[4] + s2[5]) / (256 * 1024) == 1 + 2 / 128
+
+
+@pytest.mark.parametrize("layer", [wl.TINY, wl.Q_PROJ_P10, wl.LLAMA70B[2]])
+def test_packed_sizes_cover_the_binding_layout(L, layer):
+    s = _lib.packed_sizes(layer.N, layer.K, layer.N8)
+    N4p, N8p = _lib.padded(layer.N4), _lib.padded(layer.N8)
+    assert s[1] == layer.G * N4p // 2 and s[5] == layer.G * N8p * 2
+
+
+def _status(L, fn, *args):
+    return getattr(L, fn)(*args)
+
+
+def test_host_validation_rejects_before_any_device_call(L):
+    null = None
+    # unsupported group size / K
+    assert L.mixllm_quantize_act(null, 4, 256, 64, null, null, null) == _lib.ERR_UNSUPPORTED
+    assert L.mixllm_quantize_act(null, 4, 200, 128, null, null, null) == _lib.ERR_UNSUPPORTED
+    assert b"group" in L.mixllm_last_error() or b"K" in L.mixllm_last_error()
+    # null pointers
+    assert L.mixllm_quantize_act(null, 4, 256, 128, null, null, null) == _lib.ERR_INVALID_ARG
+    # misaligned pointer (never dereferenced: rejected on the host)
+    assert L.mixllm_quantize_act(ctypes.c_void_p(0x1001), 4, 256, 128, ctypes.c_void_p(0x2000),
+                                 ctypes.c_void_p(0x3000), null) == _lib.ERR_INVALID_ARG
+    # M = 0 is a no-op that succeeds without a device
+    assert L.mixllm_quantize_act(null, 0, 256, 128, null, null, null) == _lib.OK
+    # GEMM: bad K, negative sizes, null outputs, misaligned A
+    args = [null, null, 4, 256, null, null, null, null, 8, null, null, null, 0, null, null]
+    a = list(args); a[3] = 100; a[13] = ctypes.c_void_p(0x3000)
+    assert L.mixllm_gemm_w4w8a8(*a) == _lib.ERR_UNSUPPORTED
+    a = list(args); a[8] = -1
+    assert L.mixllm_gemm_w4w8a8(*a) == _lib.ERR_INVALID_ARG
+    assert L.mixllm_gemm_w4w8a8(*args) == _lib.ERR_INVALID_ARG  # null Y
+    a = list(args)
+    a[0], a[1], a[13] = ctypes.c_void_p(0x1008), ctypes.c_void_p(0x2000), ctypes.c_void_p(0x3000)
+    assert L.mixllm_gemm_w4w8a8(*a) == _lib.ERR_INVALID_ARG
+    assert b"16-byte" in L.mixllm_last_error()
+    # empty problems succeed without a device
+    a = list(args); a[2] = 0
+    assert L.mixllm_gemm_w4w8a8(*a) == _lib.OK
+    # pack: N8 > N
+    assert L.mixllm_pack_weights(null, 4, 256, null, 5, 128, *([null] * 8)) == _lib.ERR_INVALID_ARG
+    # self-test limit range
+    assert L.mixllm_selftest_wait_timeout(0, null) == _lib.ERR_INVALID_ARG
+    # packed sizes argument checks
+    out = (ctypes.c_size_t * 7)()
+    assert L.mixllm_packed_sizes(10, 256, 11, 128, out) == _lib.ERR_INVALID_ARG
+    assert L.mixllm_packed_sizes(10, 256, 1, 32, out) == _lib.ERR_UNSUPPORTED
+
+
+def test_binding_raises_without_cuda_tensors(L):
+    import torch
+    with pytest.raises(ValueError):
+        _lib.quantize_act_into(torch.zeros(2, 128, dtype=torch.float16), torch.zeros(2, 128, dtype=torch.int8),
+                               torch.zeros(2, 1), None)
