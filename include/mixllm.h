@@ -87,11 +87,13 @@ MIXLLM_API mixllm_status mixllm_packed_sizes(int64_t N, int64_t K, int64_t N8, i
 
 /*
  * Activation quantization (one kernel): for every token m and group g of
- * 128 columns, amax = max |x|, s_a = amax / 127 (fp32, IEEE division),
+ * 128 columns, amax = max |x|, s_a = amax / 127 (fp32, IEEE division)
+ * rounded to bfloat16 precision (8 significant bits, kept as an fp32 value),
  * A_q = clamp(round_half_even(x / s_a), -127, 127); a group whose amax is 0
  * gets s_a = 0 and A_q = 0.  (Talk notes §設計判断の概要: activations 8-bit
- * symmetric, group-wise RTN; the rounding and scale precision are this
- * library's reading of "RTN".)
+ * symmetric, group-wise RTN; the rounding mode and the scale precision are
+ * this library's reading -- the pages give neither.  With a bf16 scale the
+ * RTN error stays within s_a/2 and the GEMM's bias term 1.5*2^23*s_a is exact.)
  *   X_f16  device, fp16 [M, K] row-major, 16-byte aligned, read only
  *   A_q    device, int8 [M, K] row-major, 16-byte aligned, written
  *   s_a    device, fp32 [M, K/128] row-major, 4-byte aligned, written
@@ -138,8 +140,9 @@ MIXLLM_API mixllm_status mixllm_pack_weights(const float *W, int64_t N, int64_t 
  * output channel n of a set and token m,
  *   P_g = sum_{k in group g} (W_q[n,k] - z[n,g]) * A_q[m,k]   (int32 exact,
  *         z = 0 for the 8-bit set; int8 tensor cores, tcgen05 kind::i8),
- *   acc = sum_g float(P_g) * s_w[n,g] * s_a[m,g]  (fp32; float(P_g) by the
- *         0x4b400000 bias trick, exact for |P_g| <= 2^22),
+ *   acc = sum_g float(P_g) * s_a[m,g] * s_w[n,g]  (fp32; float(P_g) by the
+ *         0x4b400000 bias trick, exact for |P_g| <= 2^22; the product with
+ *         s_a is correctly rounded, then accumulated with an FMA by s_w),
  *   Y[m, idx[n]] = fp16_rn(acc).
  * Arguments:
  *   A_q, s_a   device, as written by mixllm_quantize_act (A_q 16-byte

@@ -8,27 +8,32 @@
 //     acc += float(P_g) * s_w[n,g] * s_a[m,g]      fp32
 //   then Y[m, idx[n]] = fp16(acc).
 //
-// How it runs on B200 (one CTA per 128 x BN output tile, both channel sets in
-// the same launch, warp-specialized):
+// How it runs on B200 (one CTA of 16 warps per 128 x BN output tile, both
+// channel sets in the same launch, warp-specialized, registers rebalanced
+// with setmaxnreg toward the epilogue):
 //   warp 0      TMA producer: A_q tile [128 x 128] (128-byte swizzle) and the
 //               weight tile of group g -- int8 [BN x 128] for the 8-bit set,
 //               packed uint4 [BN x 64 B] plus the group's zero points for the
 //               4-bit set -- into a ring of kStages shared-memory stages.
-//   warps 2-3   4-bit set only: unpack nibbles and subtract the zero point in
-//               SWAR form (four bytes per 32-bit op, no borrow between bytes)
-//               into an int8 tile in the 128-byte swizzled K-major layout the
-//               tensor core reads -- the B200 counterpart of the pages' vsub4
-//               pre-dequantization step (§ソフトウェアパイプライン).
 //   warp 1      one thread issues 4 x tcgen05.mma.kind::i8 (K = 32 each) per
 //               group into one of kAccBufs int32 accumulators in tensor memory
 //               (TMEM), so the MMA of later groups overlaps the SIMT work on
 //               earlier ones.
-//   warps 4-11  epilogue: tcgen05.ld a group's int32 partials, convert with the
-//               bias trick (bits of P + 0x4b400000 read as float equal
-//               1.5*2^23 + P exactly for |P| <= 2^22) and fold the bias into an
-//               exact FMA: u = fma(v, s_w, -1.5*2^23*s_w) = fl(P*s_w), since
-//               1.5*2^23*s_w is exact for an fp16 s_w; then acc = fma(u, s_a,
-//               acc), two f32x2 FMAs per pair of elements.  After the last
+//   warp 2      stages, per group, the column scales s_w (fp32) and the row
+//               scales s_a of the tile in a small ring the epilogue reads.
+//   warps 12-15 4-bit set only: unpack nibbles and subtract the zero point in
+//               SWAR form (four bytes per 32-bit op, no borrow between bytes)
+//               into an int8 tile in the 128-byte swizzled K-major layout the
+//               tensor core reads -- the B200 counterpart of the pages' vsub4
+//               pre-dequantization step (§ソフトウェアパイプライン).
+//   warps 4-11  epilogue: tcgen05.ld a group's int32 partials, which the
+//               accumulator already holds biased by 0x4b400000 (TMEM is preset
+//               to the bias), so their bits read as float are 1.5*2^23 + P
+//               exactly for |P| <= 2^22 -- the bias trick with no integer add.
+//               The bias is folded into an exact FMA with the row scale:
+//               u = fma(v, s_a, -1.5*2^23*s_a) = fl(P*s_a), exact because s_a
+//               is bf16-valued; then acc = fma(u, s_w, acc): two f32x2 FMAs
+//               per pair of elements, one shared-memory load per four.  After the last
 //               group, fp16 results are staged in shared memory and scattered
 //               row-wise to Y[:, idx] so each warp store covers a short run of
 //               one output row.
@@ -48,31 +53,43 @@ namespace mixllm {
 
 constexpr int kBM = 128;         // tile rows (tokens) = TMEM lanes
 constexpr int kKG = 128;         // K per group = K per pipeline stage
-constexpr int kThreads = 384;    // 12 warps
-constexpr int kEpiWarps = 8;
+constexpr int kThreads = 512;    // 16 warps = 4 warpgroups
+constexpr int kEpiWarps = 8;     // warps 4..11
 constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kXformWarps = 4;   // warps 12..15
 constexpr float kI2FBias = 12582912.0f;     // 1.5 * 2^23, the float with bits 0x4b400000
 constexpr uint32_t kI2FBiasBits = 0x4B400000u;
+// register split (all four warpgroups together must stay within 65536):
+// 128 * (kRegsCtl + kRegsXform) + 256 * kRegsEpi <= 512 * 128 (the launch's registers)
+constexpr int kRegsCtl = 112, kRegsXform = 48, kRegsEpi = 176;
+static_assert(128 * (kRegsCtl + kRegsXform) + 256 * kRegsEpi <= 65536, "register split");
 
 template <int BN>
 struct GemmCfg {
-  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "BN");
+  static_assert(BN == 128, "the warp roles below are laid out for BN = 128");
   static constexpr int kStages = 5;
-  static constexpr int kAccBufs = (4 * BN <= 512) ? 4 : 2;
-  static constexpr int kTmemCols = kAccBufs * BN;  // power of two for BN in {64, 128, 256}
+  static constexpr int kAccBufs = 4;
+  static constexpr int kTabSlots = 4;
+  static constexpr int kTmemCols = kAccBufs * BN;  // 512
   static constexpr int kABytes = kBM * kKG;        // 16 KB
   static constexpr int kWBytes = BN * kKG;         // int8 weight tile
   static constexpr int kStageBytes = kABytes + kWBytes;
   static constexpr int kTBufBytes = BN * kKG;      // unpacked 4-bit tile
   static constexpr int kZBytes = 128;              // zero points of one group (BN/2 used)
-  static constexpr int kColsPerThread = BN * kBM / kEpiThreads;  // BN / 2
+  static constexpr int kColsPerThread = BN * kBM / kEpiThreads;  // 64
+  static constexpr int kTabSwBytes = BN * 4;                   // s_w of the tile's columns (fp32)
+  static constexpr int kTabBytes = kTabSwBytes + kBM * 4;      // + s_a of the tile's rows
+  static constexpr int kStgSlots = 8;                          // raw scale staging ring
+  static constexpr int kStgDist = 6;                           // groups prefetched ahead
+  static constexpr int kStgBytes = BN * 2 + kBM * 4;           // raw fp16 s_w + fp32 s_a
   // shared-memory layout (offsets from a 1024-byte aligned base)
   static constexpr int kOffStages = 0;
   static constexpr int kOffTBuf = kStages * kStageBytes;
   static constexpr int kOffZ = kOffTBuf + 2 * kTBufBytes;
-  static constexpr int kOffTab = kOffZ + kStages * kZBytes;  // [2][BN/2] float4
-  static constexpr int kOffBar = kOffTab + 2 * (BN / 2) * 16;
-  static constexpr int kNumBars = 2 * kStages + 2 + 2 + 2 * kAccBufs + 1;
+  static constexpr int kOffTab = kOffZ + kStages * kZBytes;
+  static constexpr int kOffStg = kOffTab + kTabSlots * kTabBytes;
+  static constexpr int kOffBar = kOffStg + kStgSlots * kStgBytes;
+  static constexpr int kNumBars = kStages + 2 + 2 * kAccBufs + 2 * kTabSlots + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;
@@ -99,13 +116,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
-  uint64_t *full = bars;
-  uint64_t *empty = bars + C::kStages;
-  uint64_t *tfull = bars + 2 * C::kStages;
-  uint64_t *tempty = tfull + 2;
-  uint64_t *accfull = tempty + 2;
-  uint64_t *accempty = accfull + C::kAccBufs;
-  uint64_t *drain = accempty + C::kAccBufs;
+  uint64_t *full = bars;                          // TMA -> MMA / unpack      (per stage)
+  uint64_t *tfull = full + C::kStages;            // unpack -> MMA            (per unpacked buffer)
+  uint64_t *done = tfull + 2;                     // MMA of group g complete  (ring of kAccBufs): frees
+                                                  // its stage, its unpacked buffer, and fills its accumulator
+  uint64_t *accempty = done + C::kAccBufs;        // epilogue -> MMA          (per TMEM accumulator)
+  uint64_t *tabfull = accempty + C::kAccBufs;     // scale warp -> epilogue   (per table slot)
+  uint64_t *tabempty = tabfull + C::kTabSlots;    // epilogue -> scale warp
+  uint64_t *drain = tabempty + C::kTabSlots;      // [2]: one per MMA issuer
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kOffMisc + 4);
 
@@ -126,24 +144,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto stage_w = [&](int s) { return smem + C::kOffStages + s * C::kStageBytes + C::kABytes; };
   auto tbuf = [&](int b) { return smem + C::kOffTBuf + b * C::kTBufBytes; };
   auto zmeta = [&](int s) { return smem + C::kOffZ + s * C::kZBytes; };
-  float4 *table = reinterpret_cast<float4 *>(smem + C::kOffTab);  // [2][BN/2]
+  auto table = [&](int slot) { return reinterpret_cast<float4 *>(smem + C::kOffTab + slot * C::kTabBytes); };
+  auto table_sa = [&](int slot) {
+    return reinterpret_cast<float *>(smem + C::kOffTab + slot * C::kTabBytes + C::kTabSwBytes);
+  };
+  auto stg_sw = [&](int i) { return smem + C::kOffStg + i * C::kStgBytes; };
+  auto stg_sa = [&](int i) { return reinterpret_cast<float *>(smem + C::kOffStg + i * C::kStgBytes + BN * 2); };
 
   if (threadIdx.x == 0) {
     prefetch_tmap(&tmA);
     if (is4) prefetch_tmap(&tmW4); else prefetch_tmap(&tmW8);
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&tfull[b], 2);
-      mbar_init(&tempty[b], 1);
-    }
+    for (int s = 0; s < C::kStages; ++s) mbar_init(&full[s], 1);
+    for (int b = 0; b < 2; ++b) mbar_init(&tfull[b], kXformWarps);
     for (int a = 0; a < C::kAccBufs; ++a) {
-      mbar_init(&accfull[a], 1);
+      mbar_init(&done[a], 1);
       mbar_init(&accempty[a], kEpiWarps);
     }
-    mbar_init(drain, 1);
+    for (int i = 0; i < C::kTabSlots; ++i) {
+      mbar_init(&tabfull[i], 1);
+      mbar_init(&tabempty[i], kEpiWarps);
+    }
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -156,67 +178,131 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int issued = 0;
-      const uint32_t bytes = C::kABytes + (is4 ? BN * 64 + BN / 2 : BN * kKG);
-      for (int g = 0; g < G; ++g) {
-        const int s = g % C::kStages;
-        if (!mbar_wait(&empty[s], ((g / C::kStages) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&full[s], bytes);
-        tma_load_2d(stage_a(s), &tmA, &full[s], g * kKG, m0);
-        if (is4) {
-          tma_load_2d(stage_w(s), &tmW4, &full[s], g * (kKG / 2), n0);
-          bulk_load(zmeta(s), z4 + static_cast<int64_t>(g) * (N4p >> 1) + (n0 >> 1), BN / 2, &full[s]);
-        } else {
-          tma_load_2d(stage_w(s), &tmW8, &full[s], g * kKG, n0);
-        }
-        issued = g + 1;
-      }
-      // Let every copy this thread issued land before the CTA can exit.
-      for (int g = (issued > C::kStages ? issued - C::kStages : 0); g < issued; ++g) {
-        volatile int never = 0;
-        (void)mbar_wait(&full[g % C::kStages], (g / C::kStages) & 1, &never, 1ll << 26);
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(kBM, BN);
-      for (int g = 0; g < G; ++g) {
-        const int s = g % C::kStages, b = g & 1, a = g % C::kAccBufs;
-        if (!mbar_wait(&full[s], (g / C::kStages) & 1, abort_flag)) break;
-        if (is4 && !mbar_wait(&tfull[b], (g >> 1) & 1, abort_flag)) break;
-        if (!mbar_wait(&accempty[a], ((g / C::kAccBufs) & 1) ^ 1, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t a_addr = smem_u32(stage_a(s));
-        const uint32_t b_addr = smem_u32(is4 ? tbuf(b) : stage_w(s));
-        const uint32_t d = tmem_base + static_cast<uint32_t>(a * BN);
+  // Every accumulator starts at the bias 0x4b400000 (and is reset to it after
+  // each drain), so the int32 sum the MMAs leave there, read as a float, is
+  // 1.5*2^23 + P exactly: the bias trick with no per-element integer add.
+  if (warp >= 4 && warp < 12) {
+    const uint32_t base = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) +
+                          static_cast<uint32_t>(((warp - 4) >> 2) * C::kColsPerThread);
 #pragma unroll
-        for (int kk = 0; kk < kKG / 32; ++kk)
-          mma_i8(d, sw128_kmajor_desc(a_addr + 32 * kk), sw128_kmajor_desc(b_addr + 32 * kk), idesc, kk > 0);
-        mma_commit(&empty[s]);
-        if (is4) mma_commit(&tempty[b]);
-        mma_commit(&accfull[a]);
+    for (int a = 0; a < C::kAccBufs; ++a)
+#pragma unroll
+      for (int c = 0; c < C::kColsPerThread; c += 32) tmem_st_32x32b_x32_fill(base + a * BN + c, kI2FBiasBits);
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  if (warp < 4) {
+    regs_dec<kRegsCtl>();
+    if (warp == 0) {
+      // ---------------------------------------------------------- TMA producer
+      if (lane == 0) {
+        int issued = 0;
+        const uint32_t bytes = C::kABytes + (is4 ? BN * 64 + BN / 2 : BN * kKG);
+        for (int g = 0; g < G; ++g) {
+          const int s = g % C::kStages;
+          // stage s last held group g - kStages; it is free once that group's MMAs are done
+          if (g >= C::kStages) {
+            const int gp = g - C::kStages;
+            if (!mbar_wait(&done[gp % C::kAccBufs], (gp / C::kAccBufs) & 1, abort_flag)) break;
+          }
+          mbar_arrive_expect_tx(&full[s], bytes);
+          tma_load_2d(stage_a(s), &tmA, &full[s], g * kKG, m0);
+          if (is4) {
+            tma_load_2d(stage_w(s), &tmW4, &full[s], g * (kKG / 2), n0);
+            bulk_load(zmeta(s), z4 + static_cast<int64_t>(g) * (N4p >> 1) + (n0 >> 1), BN / 2, &full[s]);
+          } else {
+            tma_load_2d(stage_w(s), &tmW8, &full[s], g * kKG, n0);
+          }
+          issued = g + 1;
+        }
+        // let every copy this thread issued land before the CTA can exit
+        for (int g = (issued > C::kStages ? issued - C::kStages : 0); g < issued; ++g)
+          (void)mbar_wait_drain(&full[g % C::kStages], (g / C::kStages) & 1, 1ll << 26);
       }
-      mma_commit(drain);
-      volatile int never = 0;
-      (void)mbar_wait(drain, 0, &never, 1ll << 28);
+    } else if (warp == 1 || warp == 3) {
+      // ---------------------------------------------------------- MMA issuers
+      // Two threads issue alternate groups (warp 1 the even ones, warp 3 the
+      // odd ones): a single issuing thread leaves the tensor pipe idle between
+      // groups, two keep it busy.  Each commits its group to done[g % kAccBufs].
+      if (lane == 0) {
+        constexpr uint32_t idesc = idesc_i8(kBM, BN);
+        const int who = warp == 1 ? 0 : 1;
+        for (int g = who; g < G; g += 2) {
+          const int s = g % C::kStages, b = g & 1, a = g % C::kAccBufs;
+          if (!mbar_wait(&full[s], (g / C::kStages) & 1, abort_flag)) break;
+          if (is4 && !mbar_wait(&tfull[b], (g >> 1) & 1, abort_flag)) break;
+          if (!mbar_wait(&accempty[a], ((g / C::kAccBufs) & 1) ^ 1, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(stage_a(s));
+          const uint32_t b_addr = smem_u32(is4 ? tbuf(b) : stage_w(s));
+          const uint32_t d = tmem_base + static_cast<uint32_t>(a * BN);
+#pragma unroll
+          for (int kk = 0; kk < kKG / 32; ++kk)
+            mma_i8(d, sw128_kmajor_desc(a_addr + 32 * kk), sw128_kmajor_desc(b_addr + 32 * kk), idesc, 1u);
+          mma_commit(&done[a]);
+        }
+        mma_commit(&drain[who]);
+        (void)mbar_wait_drain(&drain[who], 0, 1ll << 28);
+      }
+    } else if (warp == 2) {
+      // ---------------------------------------------------------- scale table
+      // Slot `slot` of group g holds s_w of the tile's BN columns as fp32,
+      // followed by s_a of the tile's 128 rows.  Raw scales are prefetched
+      // kStgDist groups ahead with cp.async into a staging ring, so no load
+      // latency sits on the epilogue's path.
+      auto issue = [&](int g) {
+        if (g < G) {
+          const int i = g % C::kStgSlots;
+          cp_async_8(stg_sw(i) + 8 * lane, s_w + static_cast<int64_t>(g) * Np + n0 + 4 * lane);
+#pragma unroll
+          for (int j = 0; j < kBM / 32; ++j) {
+            const int row = lane + 32 * j;
+            const bool in = m0 + row < M;
+            cp_async_4(stg_sa(i) + row, s_a + (in ? static_cast<int64_t>(m0 + row) * G + g : 0), in ? 4u : 0u);
+          }
+        }
+        cp_async_commit();
+      };
+      for (int g = 0; g < C::kStgDist; ++g) issue(g);
+      for (int g = 0; g < G; ++g) {
+        const int slot = g % C::kTabSlots, i = g % C::kStgSlots;
+        cp_async_wait<C::kStgDist - 1>();
+        __syncwarp();
+        if (!warp_wait(&tabempty[slot], ((g / C::kTabSlots) & 1) ^ 1, abort_flag)) break;
+        const uint2 raw = *reinterpret_cast<const uint2 *>(stg_sw(i) + 8 * lane);
+        const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&raw.x));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&raw.y));
+        table(slot)[lane] = make_float4(a.x, a.y, b.x, b.y);
+        float *tsa = table_sa(slot);
+        const float *ssa = stg_sa(i);
+#pragma unroll
+        for (int j = 0; j < kBM / 32; ++j) tsa[lane + 32 * j] = ssa[lane + 32 * j];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tabfull[slot]);
+        issue(g + C::kStgDist);
+      }
+      cp_async_wait<0>();
     }
-  } else if (warp < 4) {
+  } else if (warp >= 12) {
+    regs_dec<kRegsXform>();
     // ------------------------------------------------------------ 4-bit unpack
     if (is4) {
-      const int tt = threadIdx.x - 64;
+      const int tt = threadIdx.x - 384;  // 0..127
       for (int g = 0; g < G; ++g) {
         const int s = g % C::kStages, b = g & 1;
-        if (!mbar_wait(&full[s], (g / C::kStages) & 1, abort_flag)) break;
-        if (!mbar_wait(&tempty[b], ((g >> 1) & 1) ^ 1, abort_flag)) break;
+        if (!warp_wait(&full[s], (g / C::kStages) & 1, abort_flag)) break;
+        if (g >= 2) {  // tbuf[b] last held group g - 2
+          const int gp = g - 2;
+          if (!warp_wait(&done[gp % C::kAccBufs], (gp / C::kAccBufs) & 1, abort_flag)) break;
+        }
         const uint8_t *raw = stage_w(s);
         const uint8_t *zb = zmeta(s);
         uint8_t *dst = tbuf(b);
-#pragma unroll 2
-        for (int it = tt; it < BN * 4; it += 64) {
+#pragma unroll
+        for (int it = tt; it < BN * 4; it += 32 * kXformWarps) {
           const int r = it >> 2, c = it & 3;
           const uint4 x = *reinterpret_cast<const uint4 *>(raw + r * 64 + c * 16);
           const uint32_t zz = ((zb[r >> 1] >> ((r & 1) * 4)) & 0xFu) * 0x01010101u;
@@ -239,82 +325,100 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
+    regs_inc<kRegsEpi>();
     // ------------------------------------------------------------ epilogue
-    constexpr int CPT = C::kColsPerThread;  // columns per thread
+    constexpr int CPT = C::kColsPerThread;  // 64 columns per thread
     const int e = warp - 4;                 // 0..7
     const int quad = warp & 3;              // TMEM lane quadrant of this warp
     const int half = e >> 2;                // column half
     const int row = quad * 32 + lane;
     const int m = m0 + row;
-    const int et = threadIdx.x - 128;       // 0..255
     const bool row_ok = m < M;
 
     float acc[CPT];
 #pragma unroll
     for (int j = 0; j < CPT; ++j) acc[j] = 0.0f;
 
-    float sa_q[4];
+    // Software pipeline over 16-column chunks: while one chunk is converted
+    // and accumulated, the tcgen05.ld of the next one (this group's next
+    // chunk, or the next group's first) is in flight.
+    constexpr int CW = 16, NCH = CPT / CW;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + half * CPT;
+    uint32_t rbuf[2][CW];
+    // v = bits of (1.5*2^23 + P) as float; u = fma(v, s_a, -1.5*2^23*s_a) is
+    // exactly fl(P * s_a) (the bias term is exact for a bf16-valued s_a); then
+    // acc += u * s_w.  tab holds the s_w of 4 consecutive columns per float4.
+    auto convert = [&](uint32_t(&r)[CW], const float4 *tab, float2 sa2, float2 cb2, int c0) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) sa_q[i] = (row_ok && i < G) ? __ldg(s_a + static_cast<int64_t>(m) * G + i) : 0.0f;
-    __half sw_q[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-      sw_q[i] = (et < BN && i < G) ? s_w[static_cast<int64_t>(i) * Np + n0 + et] : __float2half_rn(0.0f);
-
-    for (int g = 0; g < G; ++g) {
-      const int a = g % C::kAccBufs;
-      // column scales of group g, and the exact bias term -1.5*2^23*s_w
-      if (et < BN) {
-        const float sw = __half2float((g & 1) ? sw_q[1] : sw_q[0]);
-        float *tab = reinterpret_cast<float *>(table + (g & 1) * (BN / 2));
-        tab[(et >> 1) * 4 + (et & 1)] = sw;
-        tab[(et >> 1) * 4 + 2 + (et & 1)] = -kI2FBias * sw;
-        const __half nxt = (g + 2 < G) ? s_w[static_cast<int64_t>(g + 2) * Np + n0 + et] : __float2half_rn(0.0f);
-        if (g & 1) sw_q[1] = nxt; else sw_q[0] = nxt;
+      for (int j = 0; j < CW / 4; ++j) {
+        const float4 sw = tab[j];
+        const float2 v0 = make_float2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]));
+        const float2 v1 = make_float2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+        const float2 u0 = __ffma2_rn(v0, sa2, cb2);
+        const float2 u1 = __ffma2_rn(v1, sa2, cb2);
+        const float2 o0 = __ffma2_rn(u0, make_float2(sw.x, sw.y), make_float2(acc[c0 + 4 * j], acc[c0 + 4 * j + 1]));
+        const float2 o1 =
+            __ffma2_rn(u1, make_float2(sw.z, sw.w), make_float2(acc[c0 + 4 * j + 2], acc[c0 + 4 * j + 3]));
+        acc[c0 + 4 * j] = o0.x;
+        acc[c0 + 4 * j + 1] = o0.y;
+        acc[c0 + 4 * j + 2] = o1.x;
+        acc[c0 + 4 * j + 3] = o1.y;
       }
-      named_bar_sync(1, kEpiThreads);
-      const float sa = sa_q[0];
-      sa_q[0] = sa_q[1];
-      sa_q[1] = sa_q[2];
-      sa_q[2] = sa_q[3];
-      sa_q[3] = (row_ok && g + 4 < G) ? __ldg(s_a + static_cast<int64_t>(m) * G + g + 4) : 0.0f;
-
-      (void)mbar_wait(&accfull[a], (g / C::kAccBufs) & 1, abort_flag);
-      tc_fence_after();
-      const uint32_t tcol = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                            static_cast<uint32_t>(a * BN + half * CPT);
-      const float4 *tab = table + (g & 1) * (BN / 2) + half * (CPT / 2);
-#pragma unroll
-      for (int c = 0; c < CPT / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tcol + c * 32, r);
-        tmem_ld_wait();
-        if constexpr (kDebugP) {
-          if (row_ok) {
+    };
+    auto dump = [&](uint32_t(&r)[CW], int g, int c0) {
+      if (row_ok) {
 #pragma unroll 4
-            for (int j = 0; j < 32; ++j) {
-              const int col = half * CPT + c * 32 + j;
-              if (n0 + col < Nset)
-                P[(static_cast<int64_t>(m) * N + idx[n0 + col]) * G + g] = static_cast<int32_t>(r[j]);
-            }
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float4 tv = tab[c * 16 + j];
-            const float2 v = make_float2(__uint_as_float(r[2 * j] + kI2FBiasBits),
-                                         __uint_as_float(r[2 * j + 1] + kI2FBiasBits));
-            const float2 u = __ffma2_rn(v, make_float2(tv.x, tv.y), make_float2(tv.z, tv.w));
-            const float2 o = __ffma2_rn(u, make_float2(sa, sa), make_float2(acc[c * 32 + 2 * j], acc[c * 32 + 2 * j + 1]));
-            acc[c * 32 + 2 * j] = o.x;
-            acc[c * 32 + 2 * j + 1] = o.y;
-          }
+        for (int j = 0; j < CW; ++j) {
+          const int col = half * CPT + c0 + j;
+          if (n0 + col < Nset)
+            P[(static_cast<int64_t>(m) * N + idx[n0 + col]) * G + g] = static_cast<int32_t>(r[j] - kI2FBiasBits);
         }
       }
+    };
+
+    bool live = warp_wait(&done[0], 0, abort_flag);
+    if (live) {
+      tc_fence_after();
+      tmem_ld_32x32b_x16(lane_base, rbuf[0]);
+    }
+    for (int g = 0; live && g < G; ++g) {
+      const int a = g % C::kAccBufs, slot = g % C::kTabSlots;
+      const uint32_t col = lane_base + static_cast<uint32_t>(a * BN);
+      if (!warp_wait(&tabfull[slot], (g / C::kTabSlots) & 1, abort_flag)) break;
+      const float sa = table_sa(slot)[row];
+      const float2 sa2 = make_float2(sa, sa);
+      const float2 cb2 = make_float2(-kI2FBias * sa, -kI2FBias * sa);
+      const float4 *tab = table(slot) + half * (CPT / 4);
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) {
+        tmem_ld_wait();
+        reg_fence(rbuf[c & 1]);
+        if (c + 1 < NCH) {
+          tmem_ld_32x32b_x16(col + CW * (c + 1), rbuf[(c + 1) & 1]);
+        } else if (g + 1 < G) {
+          const int a1 = (g + 1) % C::kAccBufs;
+          live = warp_wait(&done[a1], ((g + 1) / C::kAccBufs) & 1, abort_flag);
+          if (live) {
+            tc_fence_after();
+            tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(a1 * BN), rbuf[(c + 1) & 1]);
+          }
+        }
+        tmem_st_32x32b_x16_fill(col + CW * c, kI2FBiasBits);  // hand the chunk back preset to the bias
+        if constexpr (kDebugP) {
+          dump(rbuf[c & 1], g, CW * c);
+        } else {
+          convert(rbuf[c & 1], tab + (CW / 4) * c, sa2, cb2, CW * c);
+        }
+      }
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&accempty[a]);
+      if (lane == 0) {
+        mbar_arrive(&accempty[a]);
+        mbar_arrive(&tabempty[slot]);
+      }
     }
+    tmem_ld_wait();
 
     if constexpr (!kDebugP) {
       // stage fp16 results: row `row`, columns half*CPT .. +CPT

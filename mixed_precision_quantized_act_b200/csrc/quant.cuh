@@ -7,6 +7,7 @@
 // (weights packed and interleaved offline so no permutation runs at run time).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cstdint>
 
@@ -18,8 +19,10 @@ namespace mixllm {
 // ---------------------------------------------------------------------------
 // Activation quantization.  One half-warp per (token m, group g): 16 lanes x
 // 8 fp16 = the 128 values of the group, loaded as one 16-byte vector per lane.
-// amax over the group, s_a = amax / 127 (IEEE division, fp32),
-// q = clamp(round_half_even(x / s_a), -127, 127); amax == 0 gives s_a = q = 0.
+// amax over the group, s_a = bf16(amax / 127) (IEEE division in fp32, then
+// rounded to bfloat16 precision and kept as fp32), q = clamp(round_half_even(
+// x / s_a), -127, 127); amax == 0 gives s_a = q = 0.  The bf16 scale keeps the
+// RTN error within s_a/2 and makes 1.5*2^23*s_a exact for the GEMM epilogue.
 // The division is the correctly rounded one (not a reciprocal multiply) so
 // that the codes are the same as a plain CPU evaluation of the definition.
 // ---------------------------------------------------------------------------
@@ -47,7 +50,7 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const __half *__restr
     for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(mask, amax, o));
-    const float s = __fdiv_rn(amax, 127.0f);
+    const float s = __bfloat162float(__float2bfloat16_rn(__fdiv_rn(amax, 127.0f)));
     uint32_t packed[2] = {0u, 0u};
     if (s != 0.0f) {
 #pragma unroll

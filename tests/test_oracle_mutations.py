@@ -21,7 +21,9 @@ MUTATIONS = {
         "float scale = oracle_f16_to_f32(s4[n * G + g]) * s_a[m * G];"),
     "truncate_instead_of_round": ("float r = nearbyintf(oracle_f16_to_f32(x[i]) / s);",
                                   "float r = truncf(oracle_f16_to_f32(x[i]) / s);"),
-    "scale_divisor_128": ("float s = amax / 127.0f;", "float s = amax / 128.0f;"),
+    "scale_divisor_128": ("oracle_round_bf16(amax / 127.0f)", "oracle_round_bf16(amax / 128.0f)"),
+    "scale_not_rounded_to_bf16": ("float s = oracle_round_bf16(amax / 127.0f);", "float s = amax / 127.0f;"),
+    "bf16_truncates": ("if (dropped > 0x8000u || (dropped == 0x8000u && (keep & 1u))) keep += 1u;", ""),
     "f16_ties_away": ("float r = nearbyintf(units); /* ties to even */",
                       "float r = floorf(units + 0.5f);"),
     "w8_operand_shift": ("p += (int32_t)q[i] * (int32_t)a[i];",
@@ -39,6 +41,7 @@ MUTATIONS = {
 
 def _pins():
     yield pins.test_f32_to_f16_matches_ieee_rne, ()
+    yield pins.test_round_bf16_matches_torch, ()
     yield pins.test_act_quant_invariants, ()
     yield pins.test_act_quant_ties_half_even_and_zero_group, ()
     yield pins.test_act_quant_lossless_grid, ()

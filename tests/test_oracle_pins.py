@@ -56,6 +56,25 @@ def test_f32_to_f16_matches_ieee_rne(oracle_mod):
     assert np.array_equal(got, ref)
 
 
+def test_round_bf16_matches_torch(oracle_mod):
+    """The bf16 rounding of the activation scale: RNE to 8 significant bits,
+    checked against torch's float32 -> bfloat16 conversion."""
+    import torch
+    rng = np.random.default_rng(11)
+    parts = [rng.standard_normal(200000).astype(np.float32) * np.float32(50.0),
+             (rng.standard_normal(50000) * 1e-30).astype(np.float32),
+             np.array([0.0, -0.0, 1.0, 3.4e38, -3.4e38, np.inf, -np.inf, 1e-45, 2.0 ** -126], np.float32)]
+    # exact ties between adjacent bf16 values
+    b = (np.arange(0x3F00, 0x4100, dtype=np.uint32) << 16)
+    lo = b.view(np.float32).astype(np.float64)
+    hi = ((b + 0x10000).view(np.float32)).astype(np.float64)
+    parts.append(((lo + hi) / 2).astype(np.float32))
+    x = np.concatenate(parts)
+    got = oracle_mod.round_bf16(x)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float32).numpy()
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
 # ------------------------------------------------------------ fast I2F
 
 def test_i2f_bias_exhaustive_window(oracle_mod, golden):
@@ -88,9 +107,11 @@ def test_act_quant_invariants(oracle_mod):
     assert np.all(np.abs(a).max(axis=2) == 127)  # amax maps to +-127
     err = np.abs(x - s[:, :, None].astype(np.float64) * a)
     assert np.all(err <= s[:, :, None] * 0.5 * (1 + 1e-5))  # + rounding of x/s
-    # the scale is amax/127 in fp32
+    # the scale is amax/127 (fp32 quotient) rounded to bfloat16 precision
+    import torch
     amax = np.abs(x).max(axis=2)
-    assert np.array_equal(s, (amax / np.float32(127.0)).astype(np.float32))
+    q = torch.from_numpy((amax / np.float32(127.0)).astype(np.float32))
+    assert np.array_equal(s, q.to(torch.bfloat16).to(torch.float32).numpy())
 
 
 def test_act_quant_ties_half_even_and_zero_group(oracle_mod):
@@ -98,7 +119,7 @@ def test_act_quant_ties_half_even_and_zero_group(oracle_mod):
     x[0, 0] = 127.0        # amax = 127 -> s_a = 1 exactly
     x[0, 1:9] = [2.5, 3.5, -2.5, 0.5, 1.5, -1.5, 126.5, -0.5]
     A, s = oracle_mod.quantize_act(x)
-    assert s[0, 0] == 1.0
+    assert s[0, 0] == 1.0  # 127/127, exact in bf16
     assert list(A[0, 1:9]) == [2, 4, -2, 0, 2, -2, 126, 0]
     assert s[0, 1] == 0.0 and np.all(A[0, 128:] == 0)   # all-zero group
     assert s[1, 0] == 0.0 and np.all(A[1] == 0)
