@@ -32,6 +32,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+from mixed_precision_quantized_act_b200 import dist as dp  # noqa: E402
 from mixed_precision_quantized_act_b200 import workloads as wl  # noqa: E402
 
 METRIC = "W4.4A8 GEMM effective TOPS at M=512,N=K=4096; % of B200 int8 TC peak"
@@ -145,22 +146,26 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ oracle leg
 
-def oracle_rate(layer, X, W, is8, target_s, max_rows=None):
-    """Time the CPU oracle (quantize + two-step GEMM) on a row sample of the
-    workload; returns (TOPS-equivalent, seconds, rows)."""
+def oracle_rate(layer, X, W, is8, target_s):
+    """Time the CPU oracle (quantize + two-step GEMM), single-threaded, on
+    token rows of the workload, cycling through the batch until about
+    `target_s` seconds of work; returns (TOPS-equivalent, seconds, rows)."""
     import oracle
     Wq = oracle.Quantized(W, is8)  # offline weight quantization, not timed
-    rows = 1
     t0 = time.perf_counter()
-    A, s = oracle.quantize_act(X[:rows])
+    A, s = oracle.quantize_act(X[:1])
     oracle.gemm_w4w8a8(A, s, Wq)
-    t1 = time.perf_counter() - t0
-    total_rows = max_rows or layer.M
-    rows = int(max(1, min(total_rows, target_s / max(t1, 1e-6))))
-    t0 = time.perf_counter()
-    A, s = oracle.quantize_act(X[:rows])
-    oracle.gemm_w4w8a8(A, s, Wq)
-    dt = time.perf_counter() - t0
+    t1 = max(time.perf_counter() - t0, 1e-6)
+    rows = int(max(1, target_s / t1))
+    done, dt = 0, 0.0
+    while done < rows:
+        r0 = done % layer.M
+        n = min(rows - done, layer.M - r0)
+        t0 = time.perf_counter()
+        A, s = oracle.quantize_act(X[r0:r0 + n])
+        oracle.gemm_w4w8a8(A, s, Wq)
+        dt += time.perf_counter() - t0
+        done += n
     return 2.0 * rows * layer.N * layer.K / dt / 1e12, dt, rows
 
 
@@ -172,9 +177,8 @@ def run_reference(args, layer, rank, world):
         return
     import oracle
     X, W, is8 = wl.make_x(layer, args.seed), wl.make_w(layer, args.seed), wl.make_bitmap(layer, args.seed)
-    Wq = oracle.Quantized(W, is8)
-    # one step = one token row of the workload through quantize + GEMM
-    # restricted to the first 512 output channels of each set (bounded sample)
+    # one step = one token row of the workload through quantize + two-step GEMM,
+    # restricted to the layer's first 512 output channels (a bounded sample)
     sub_cols = np.arange(min(layer.N, 512))
     Wq_s = oracle.Quantized(W[sub_cols], is8[sub_cols])
     ops_per_step = 2.0 * 1 * len(sub_cols) * layer.K
@@ -186,7 +190,6 @@ def run_reference(args, layer, rank, world):
         A, s = oracle.quantize_act(X[i % layer.M: i % layer.M + 1])
         oracle.gemm_w4w8a8(A, s, Wq_s)
     dt = time.perf_counter() - t0
-    del Wq
     value = ops_per_step * args.steps / dt / 1e12
     sample = f"per step: 1 token row x {len(sub_cols)} output channels x K={layer.K} (quantize + two-step GEMM)"
     line = {
@@ -211,7 +214,7 @@ def run_ours(args, layer, rank, world, local_rank):
     mx.load()
     stream = torch.cuda.current_stream()
 
-    X = wl.make_x(layer, args.seed + rank)
+    X = wl.make_x(layer, dp.batch_seed(args.seed, rank))
     W, is8 = wl.make_w(layer, args.seed), wl.make_bitmap(layer, args.seed)
     Xd = torch.from_numpy(X).to(dev)
     p = mx.pack_weights(torch.from_numpy(W).to(dev), torch.from_numpy(is8).to(dev))
@@ -293,8 +296,8 @@ def run_ours(args, layer, rank, world, local_rank):
         if world == 1:
             rate, secs, rows = oracle_rate(layer, X, W, is8, args.cpu_seconds)
             cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
-                   "sample": f"{rows} of {layer.M} token rows x all {layer.N} channels x K={layer.K} "
-                             f"(quantize + two-step GEMM), {secs:.1f} s single-threaded"}
+                   "sample": f"{rows} token rows (cycling over the {layer.M}-row batch) x all {layer.N} "
+                             f"channels x K={layer.K}, quantize + two-step GEMM, {secs:.1f} s single-threaded"}
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True, "scaling": "weak",
@@ -318,19 +321,11 @@ def run_ours(args, layer, rank, world, local_rank):
 
 
 def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    dp.barrier(world)
 
 
 def max_over_ranks(x, world):
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return dp.max_over_ranks(x, world, device="cuda")
 
 
 def main():
@@ -343,20 +338,15 @@ def main():
         run_reference(args, layer, rank, world)
         return
     if world > 1:
-        import datetime
         import torch
-        import torch.distributed as dist
         torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local_rank))
+        dp.init("nccl", timeout_s=120, device=torch.device("cuda", local_rank))
     try:
         line = run_ours(args, layer, rank, world, local_rank)
         if line is not None:
             print(json.dumps(line), flush=True)
     finally:
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
+        dp.shutdown(world)
 
 
 if __name__ == "__main__":
