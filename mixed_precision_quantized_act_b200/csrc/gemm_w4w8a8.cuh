@@ -67,8 +67,12 @@ static_assert(128 * (kRegsCtl + kRegsXform) + 256 * kRegsEpi <= 65536, "register
 template <int BN>
 struct GemmCfg {
   static_assert(BN == 128, "the warp roles below are laid out for BN = 128");
-  static constexpr int kStages = 5;
+  // An even stage count gives each stage to one of the two MMA issuers (group
+  // g uses stage g % kStages, and the issuers take alternate groups), so every
+  // waiter sees each phase of each barrier in order, which parity waits need.
+  static constexpr int kStages = 4;
   static constexpr int kAccBufs = 4;
+  static_assert(kStages % 2 == 0, "stages must alternate between the two MMA issuers");
   static constexpr int kTabSlots = 4;
   static constexpr int kTmemCols = kAccBufs * BN;  // 512
   static constexpr int kABytes = kBM * kKG;        // 16 KB
@@ -393,30 +397,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < NCH; ++c) {
         tmem_ld_wait();
         reg_fence(rbuf[c & 1]);
-        if (c + 1 < NCH) {
-          tmem_ld_32x32b_x16(col + CW * (c + 1), rbuf[(c + 1) & 1]);
-        } else if (g + 1 < G) {
-          const int a1 = (g + 1) % C::kAccBufs;
-          live = warp_wait(&done[a1], ((g + 1) / C::kAccBufs) & 1, abort_flag);
-          if (live) {
-            tc_fence_after();
-            tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(a1 * BN), rbuf[(c + 1) & 1]);
+        if (c + 1 < NCH) tmem_ld_32x32b_x16(col + CW * (c + 1), rbuf[(c + 1) & 1]);
+        tmem_st_32x32b_x16_fill(col + CW * c, kI2FBiasBits);  // hand the chunk back preset to the bias
+        if (c + 1 == NCH) {
+          // Every partial of group g is in registers and its accumulator is
+          // reset: release the accumulator before waiting for group g+1, so
+          // the MMAs can run kAccBufs groups ahead of this warp.
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&accempty[a]);
+          if (g + 1 < G) {
+            const int a1 = (g + 1) % C::kAccBufs;
+            live = warp_wait(&done[a1], ((g + 1) / C::kAccBufs) & 1, abort_flag);
+            if (live) {
+              tc_fence_after();
+              tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(a1 * BN), rbuf[(c + 1) & 1]);
+            }
           }
         }
-        tmem_st_32x32b_x16_fill(col + CW * c, kI2FBiasBits);  // hand the chunk back preset to the bias
         if constexpr (kDebugP) {
           dump(rbuf[c & 1], g, CW * c);
         } else {
           convert(rbuf[c & 1], tab + (CW / 4) * c, sa2, cb2, CW * c);
         }
       }
-      tmem_st_wait();
-      tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&accempty[a]);
-        mbar_arrive(&tabempty[slot]);
-      }
+      if (lane == 0) mbar_arrive(&tabempty[slot]);  // table slot read for the last time
     }
     tmem_ld_wait();
 
