@@ -11,14 +11,18 @@
 // How it runs on B200 (one CTA of 16 warps per 128 x BN output tile, both
 // channel sets in the same launch, warp-specialized, registers rebalanced
 // with setmaxnreg toward the epilogue):
-//   warp 0      TMA producer: A_q tile [128 x 128] (128-byte swizzle) and the
-//               weight tile of group g -- int8 [BN x 128] for the 8-bit set,
-//               packed uint4 [BN x 64 B] plus the group's zero points for the
-//               4-bit set -- into a ring of kStages shared-memory stages.
-//   warp 1      one thread issues 4 x tcgen05.mma.kind::i8 (K = 32 each) per
-//               group into one of kAccBufs int32 accumulators in tensor memory
-//               (TMEM), so the MMA of later groups overlaps the SIMT work on
-//               earlier ones.
+//   warp 0      TMA producer: the A_q tile [128 x 128] (128-byte swizzle) of
+//               every group -- together with the int8 weight tile [BN x 128]
+//               on 8-bit tiles -- into a ring of stages, and on 4-bit tiles
+//               the packed uint4 weight tile [BN x 64 B] and the group's zero
+//               points into a ring of their own; L2 prefetch of the boxes a few
+//               groups further on.
+//   warps 1, 3  one thread each issues the MMAs of alternate groups: 4 x
+//               tcgen05.mma.kind::i8 (K = 32 each) into one of kAccBufs int32
+//               accumulators in tensor memory (TMEM), then one commit to the
+//               group's `done` barrier, which frees the A stage and unpacked
+//               buffer it read and hands the accumulator to the epilogue.  The
+//               MMA of later groups overlaps the SIMT work on earlier ones.
 //   warp 2      stages, per group, the column scales s_w (fp32) and the row
 //               scales s_a of the tile in a small ring the epilogue reads.
 //   warps 12-15 4-bit set only: unpack nibbles and subtract the zero point in
@@ -37,8 +41,12 @@
 //               group, fp16 results are staged in shared memory and scattered
 //               row-wise to Y[:, idx] so each warp store covers a short run of
 //               one output row.
-// Every wait is bounded; on a timeout the CTA records an error in the status
-// word, drains its own copies and MMAs, frees TMEM and exits.
+// Every ring slot is refilled as soon as its own consumer is done with it (the
+// A stages and unpacked buffers through the group's `done` barrier, the packed
+// tiles through the unpack warps), and the rings are deep enough to cover the
+// load latency of HBM.  Every wait is bounded; on a timeout the CTA records
+// an error in the status word, drains its own copies and MMAs, frees TMEM and
+// exits.
 #pragma once
 
 #include <cuda.h>
@@ -61,44 +69,65 @@ constexpr float kI2FBias = 12582912.0f;     // 1.5 * 2^23, the float with bits 0
 constexpr uint32_t kI2FBiasBits = 0x4B400000u;
 // register split (all four warpgroups together must stay within 65536):
 // 128 * (kRegsCtl + kRegsXform) + 256 * kRegsEpi <= 512 * 128 (the launch's registers)
-constexpr int kRegsCtl = 112, kRegsXform = 48, kRegsEpi = 176;
+constexpr int kRegsCtl = 88, kRegsXform = 72, kRegsEpi = 176;
 static_assert(128 * (kRegsCtl + kRegsXform) + 256 * kRegsEpi <= 65536, "register split");
 
 template <int BN>
 struct GemmCfg {
   static_assert(BN == 128, "the warp roles below are laid out for BN = 128");
-  // An even stage count gives each stage to one of the two MMA issuers (group
-  // g uses stage g % kStages, and the issuers take alternate groups), so every
-  // waiter sees each phase of each barrier in order, which parity waits need.
-  static constexpr int kStages = 4;
+  static constexpr int kABytes = kBM * kKG;        // 16 KB A_q tile of one group
+  static constexpr int kW8Bytes = BN * kKG;        // 16 KB int8 weight tile
+  static constexpr int kW4Bytes = BN * kKG / 2;    //  8 KB packed uint4 weight tile
+  static constexpr int kTBufBytes = BN * kKG;      // 16 KB unpacked 4-bit tile
+  static constexpr int kZBytes = BN / 2;           // zero points of one group, two per byte
+  // The ring region is laid out one of two ways, chosen per CTA:
+  //   8-bit tile: kStages8 stages of [A | W8]                      (32 KB each)
+  //   4-bit tile: kStagesA4 A stages, kTBufs unpacked buffers and kRaw packed
+  //               tiles                                            (16/16/8 KB)
+  static constexpr int kStages8 = 6;
+  static constexpr int kStagesA4 = 6;
+  static constexpr int kTBufs = 4;
+  static constexpr int kRaw = 4;
+  static constexpr int kMaxStages = kStages8 > kStagesA4 ? kStages8 : kStagesA4;
+  // Two threads issue the MMAs of alternate groups.  Every barrier an issuer
+  // waits on must belong to one issuer only, or a parity wait could see a
+  // phase meant for the other one: the slot counts of those rings are even.
+  static_assert(kStages8 % 2 == 0 && kStagesA4 % 2 == 0 && kTBufs % 2 == 0, "rings the issuers wait on");
+  // One commit per group, to done[g % kDone]; a waiter never falls a full ring
+  // behind as long as kDone covers every ring that is released through it.
+  static constexpr int kDone = kMaxStages;
+  static constexpr int kRing8 = kStages8 * (kABytes + kW8Bytes);
+  static constexpr int kRing4 = kStagesA4 * kABytes + kTBufs * kTBufBytes + kRaw * kW4Bytes;
+  static constexpr int kRingBytes = kRing8 > kRing4 ? kRing8 : kRing4;
   static constexpr int kAccBufs = 4;
-  static_assert(kStages % 2 == 0, "stages must alternate between the two MMA issuers");
+  static_assert(kAccBufs % 2 == 0, "accumulators alternate between the issuers");
+  static_assert(kDone >= kStages8 && kDone >= kStagesA4 && kDone >= kTBufs && kDone >= kAccBufs, "done ring");
   static constexpr int kTabSlots = 4;
   static constexpr int kTmemCols = kAccBufs * BN;  // 512
-  static constexpr int kABytes = kBM * kKG;        // 16 KB
-  static constexpr int kWBytes = BN * kKG;         // int8 weight tile
-  static constexpr int kStageBytes = kABytes + kWBytes;
-  static constexpr int kTBufBytes = BN * kKG;      // unpacked 4-bit tile
-  static constexpr int kZBytes = 128;              // zero points of one group (BN/2 used)
   static constexpr int kColsPerThread = BN * kBM / kEpiThreads;  // 64
   static constexpr int kTabSwBytes = BN * 4;                   // s_w of the tile's columns (fp32)
   static constexpr int kTabBytes = kTabSwBytes + kBM * 4;      // + s_a of the tile's rows
   static constexpr int kStgSlots = 8;                          // raw scale staging ring
   static constexpr int kStgDist = 6;                           // groups prefetched ahead
   static constexpr int kStgBytes = BN * 2 + kBM * 4;           // raw fp16 s_w + fp32 s_a
+  // L2 prefetch distance in groups, past the loads the ring already holds
+  static constexpr int kPrefetchAhead = 4;
   // shared-memory layout (offsets from a 1024-byte aligned base)
-  static constexpr int kOffStages = 0;
-  static constexpr int kOffTBuf = kStages * kStageBytes;
-  static constexpr int kOffZ = kOffTBuf + 2 * kTBufBytes;
-  static constexpr int kOffTab = kOffZ + kStages * kZBytes;
+  static constexpr int kOffRing = 0;
+  static constexpr int kOffZ = kOffRing + kRingBytes;
+  static constexpr int kOffTab = kOffZ + kRaw * kZBytes;
   static constexpr int kOffStg = kOffTab + kTabSlots * kTabBytes;
-  static constexpr int kOffBar = kOffStg + kStgSlots * kStgBytes;
-  static constexpr int kNumBars = kStages + 2 + 2 * kAccBufs + 2 * kTabSlots + 2;
+  static constexpr int kOffIdx = kOffStg + kStgSlots * kStgBytes;  // output channel of each tile column
+  static constexpr int kOffBar = kOffIdx + BN * 4;
+  // full per stage, done per group ring, full/empty per packed tile, full per unpacked buffer,
+  // empty per accumulator, full/empty per table slot, one drain per issuer
+  static constexpr int kNumBars = kMaxStages + kDone + 2 * kRaw + kTBufs + kAccBufs + 2 * kTabSlots + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;
   static constexpr int kStagingStride = (BN + 2) * 2;  // bytes per staged fp16 row
-  static_assert(kBM * kStagingStride <= kOffTBuf, "staging must fit in the stage ring");
+  static_assert(kBM * kStagingStride <= kRingBytes, "staging must fit in the ring region");
+  static_assert(kABytes % 1024 == 0 && kTBufBytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
 };
 
@@ -120,14 +149,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
-  uint64_t *full = bars;                          // TMA -> MMA / unpack      (per stage)
-  uint64_t *tfull = full + C::kStages;            // unpack -> MMA            (per unpacked buffer)
-  uint64_t *done = tfull + 2;                     // MMA of group g complete  (ring of kAccBufs): frees
-                                                  // its stage, its unpacked buffer, and fills its accumulator
-  uint64_t *accempty = done + C::kAccBufs;        // epilogue -> MMA          (per TMEM accumulator)
-  uint64_t *tabfull = accempty + C::kAccBufs;     // scale warp -> epilogue   (per table slot)
+  uint64_t *full = bars;                          // TMA -> MMA              (per stage)
+  uint64_t *done = full + C::kMaxStages;          // MMA commit of group g   (ring of kDone): frees the
+                                                  // group's A stage and unpacked buffer, fills its accumulator
+  uint64_t *rfull = done + C::kDone;              // TMA -> unpack           (per packed tile)
+  uint64_t *rempty = rfull + C::kRaw;             // unpack -> TMA           (per packed tile)
+  uint64_t *tfull = rempty + C::kRaw;             // unpack -> MMA           (per unpacked buffer)
+  uint64_t *accempty = tfull + C::kTBufs;         // epilogue -> MMA         (per TMEM accumulator)
+  uint64_t *tabfull = accempty + C::kAccBufs;     // scale warp -> epilogue  (per table slot)
   uint64_t *tabempty = tabfull + C::kTabSlots;    // epilogue -> scale warp
-  uint64_t *drain = tabempty + C::kTabSlots;      // [2]: one per MMA issuer
+  uint64_t *drain = tabempty + C::kTabSlots;      // [2]: each MMA issuer's final commit
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kOffMisc + 4);
 
@@ -143,27 +174,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int N = N4 + N8;
   const __half *s_w = is4 ? s_w4 : s_w8;
   const int32_t *idx = is4 ? idx4 : idx8;
+  const int S = is4 ? C::kStagesA4 : C::kStages8;  // A stages of this tile
 
-  auto stage_a = [&](int s) { return smem + C::kOffStages + s * C::kStageBytes; };
-  auto stage_w = [&](int s) { return smem + C::kOffStages + s * C::kStageBytes + C::kABytes; };
-  auto tbuf = [&](int b) { return smem + C::kOffTBuf + b * C::kTBufBytes; };
-  auto zmeta = [&](int s) { return smem + C::kOffZ + s * C::kZBytes; };
+  // ring region: 8-bit tiles [A | W8] x kStages8; 4-bit tiles A x kStagesA4, then unpacked, then packed
+  const int stage_bytes = is4 ? C::kABytes : C::kABytes + C::kW8Bytes;
+  auto stage_a = [&](int s) { return smem + C::kOffRing + s * stage_bytes; };
+  auto stage_w8 = [&](int s) { return smem + C::kOffRing + s * stage_bytes + C::kABytes; };
+  auto tbuf = [&](int b) { return smem + C::kOffRing + C::kStagesA4 * C::kABytes + b * C::kTBufBytes; };
+  auto raw_w4 = [&](int r) {
+    return smem + C::kOffRing + C::kStagesA4 * C::kABytes + C::kTBufs * C::kTBufBytes + r * C::kW4Bytes;
+  };
+  auto zmeta = [&](int r) { return smem + C::kOffZ + r * C::kZBytes; };
   auto table = [&](int slot) { return reinterpret_cast<float4 *>(smem + C::kOffTab + slot * C::kTabBytes); };
   auto table_sa = [&](int slot) {
     return reinterpret_cast<float *>(smem + C::kOffTab + slot * C::kTabBytes + C::kTabSwBytes);
   };
   auto stg_sw = [&](int i) { return smem + C::kOffStg + i * C::kStgBytes; };
   auto stg_sa = [&](int i) { return reinterpret_cast<float *>(smem + C::kOffStg + i * C::kStgBytes + BN * 2); };
+  int32_t *col_idx = reinterpret_cast<int32_t *>(smem + C::kOffIdx);
+
+  // Loads of the A ring (and of W8 on 8-bit tiles) for group g into stage g % S.
+  const uint32_t a_bytes = static_cast<uint32_t>(is4 ? C::kABytes : C::kABytes + C::kW8Bytes);
+  auto load_a = [&](int g) {
+    const int s = g % S;
+    mbar_arrive_expect_tx(&full[s], a_bytes);
+    tma_load_2d(stage_a(s), &tmA, &full[s], g * kKG, m0);
+    if (!is4) tma_load_2d(stage_w8(s), &tmW8, &full[s], g * kKG, n0);
+  };
 
   if (threadIdx.x == 0) {
     prefetch_tmap(&tmA);
     if (is4) prefetch_tmap(&tmW4); else prefetch_tmap(&tmW8);
-    for (int s = 0; s < C::kStages; ++s) mbar_init(&full[s], 1);
-    for (int b = 0; b < 2; ++b) mbar_init(&tfull[b], kXformWarps);
-    for (int a = 0; a < C::kAccBufs; ++a) {
-      mbar_init(&done[a], 1);
-      mbar_init(&accempty[a], kEpiWarps);
+    for (int s = 0; s < C::kMaxStages; ++s) mbar_init(&full[s], 1);
+    for (int i = 0; i < C::kDone; ++i) mbar_init(&done[i], 1);
+    for (int r = 0; r < C::kRaw; ++r) {
+      mbar_init(&rfull[r], 1);
+      mbar_init(&rempty[r], kXformWarps);
     }
+    for (int b = 0; b < C::kTBufs; ++b) mbar_init(&tfull[b], kXformWarps);
+    for (int a = 0; a < C::kAccBufs; ++a) mbar_init(&accempty[a], kEpiWarps);
     for (int i = 0; i < C::kTabSlots; ++i) {
       mbar_init(&tabfull[i], 1);
       mbar_init(&tabempty[i], kEpiWarps);
@@ -172,6 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // the first stages need nothing but their barriers: start them before the CTA-wide sync
+    for (int g = 0; g < S && g < G; ++g) load_a(g);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
@@ -182,76 +233,102 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  // Every accumulator starts at the bias 0x4b400000 (and is reset to it after
-  // each drain), so the int32 sum the MMAs leave there, read as a float, is
-  // 1.5*2^23 + P exactly: the bias trick with no per-element integer add.
-  if (warp >= 4 && warp < 12) {
-    const uint32_t base = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) +
-                          static_cast<uint32_t>(((warp - 4) >> 2) * C::kColsPerThread);
-#pragma unroll
-    for (int a = 0; a < C::kAccBufs; ++a)
-#pragma unroll
-      for (int c = 0; c < C::kColsPerThread; c += 32) tmem_st_32x32b_x32_fill(base + a * BN + c, kI2FBiasBits);
-    tmem_st_wait();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-
   if (warp < 4) {
     regs_dec<kRegsCtl>();
     if (warp == 0) {
       // ---------------------------------------------------------- TMA producer
+      // One thread feeds both rings: the A stages (with W8 on 8-bit tiles),
+      // each refilled once the MMAs of the group that held it are done, and on
+      // 4-bit tiles the packed W4 tiles, each refilled once unpacked.  It
+      // polls both, so neither ring waits on the other, and keeps L2
+      // prefetches kPrefetchAhead groups ahead of each.
       if (lane == 0) {
-        int issued = 0;
-        const uint32_t bytes = C::kABytes + (is4 ? BN * 64 + BN / 2 : BN * kKG);
-        for (int g = 0; g < G; ++g) {
-          const int s = g % C::kStages;
-          // stage s last held group g - kStages; it is free once that group's MMAs are done
-          if (g >= C::kStages) {
-            const int gp = g - C::kStages;
-            if (!mbar_wait(&done[gp % C::kAccBufs], (gp / C::kAccBufs) & 1, abort_flag)) break;
+        auto prefetch_a = [&](int g) {
+          if (g < G) {
+            tma_prefetch_l2_2d(&tmA, g * kKG, m0);
+            if (!is4) tma_prefetch_l2_2d(&tmW8, g * kKG, n0);
           }
-          mbar_arrive_expect_tx(&full[s], bytes);
-          tma_load_2d(stage_a(s), &tmA, &full[s], g * kKG, m0);
-          if (is4) {
-            tma_load_2d(stage_w(s), &tmW4, &full[s], g * (kKG / 2), n0);
-            bulk_load(zmeta(s), z4 + static_cast<int64_t>(g) * (N4p >> 1) + (n0 >> 1), BN / 2, &full[s]);
-          } else {
-            tma_load_2d(stage_w(s), &tmW8, &full[s], g * kKG, n0);
+        };
+        auto prefetch_w4 = [&](int g) {
+          if (g < G) {
+            tma_prefetch_l2_2d(&tmW4, g * (kKG / 2), n0);
+            bulk_prefetch_l2(z4 + static_cast<int64_t>(g) * (N4p >> 1) + (n0 >> 1), C::kZBytes);
           }
-          issued = g + 1;
+        };
+        int ga = S < G ? S : G;  // next A group; the prologue issued groups 0 .. S-1
+        int gw = is4 ? 0 : G;    // next packed W4 group
+        for (int g = ga; g < ga + C::kPrefetchAhead; ++g) prefetch_a(g);
+        if (is4)
+          for (int g = 0; g < C::kRaw + C::kPrefetchAhead; ++g) prefetch_w4(g);
+        long long idle_since = -1;
+        while (ga < G || gw < G) {
+          bool progressed = false;
+          // packed slot gw % kRaw last held group gw - kRaw; the unpack warps released it
+          if (gw < G &&
+              (gw < C::kRaw || mbar_try_wait(smem_u32(&rempty[gw % C::kRaw]), ((gw / C::kRaw) - 1) & 1))) {
+            const int r = gw % C::kRaw;
+            mbar_arrive_expect_tx(&rfull[r], static_cast<uint32_t>(C::kW4Bytes + C::kZBytes));
+            tma_load_2d(raw_w4(r), &tmW4, &rfull[r], gw * (kKG / 2), n0);
+            bulk_load(zmeta(r), z4 + static_cast<int64_t>(gw) * (N4p >> 1) + (n0 >> 1), C::kZBytes, &rfull[r]);
+            prefetch_w4(gw + C::kRaw + C::kPrefetchAhead);
+            ++gw;
+            progressed = true;
+          }
+          // A stage ga % S last held group ga - S; it is free once that group is done
+          if (ga < G && mbar_try_wait(smem_u32(&done[(ga - S) % C::kDone]), ((ga - S) / C::kDone) & 1)) {
+            load_a(ga);
+            prefetch_a(ga + C::kPrefetchAhead);
+            ++ga;
+            progressed = true;
+          }
+          if (progressed) {
+            idle_since = -1;
+            continue;
+          }
+          if (*abort_flag) break;
+          const long long now = clock64();
+          if (idle_since < 0) {
+            idle_since = now;
+          } else if (now - idle_since > (1ll << 32)) {
+            *abort_flag = 1;
+            record_status(kStatusTimeout);
+            break;
+          }
+          __nanosleep(64);
         }
         // let every copy this thread issued land before the CTA can exit
-        for (int g = (issued > C::kStages ? issued - C::kStages : 0); g < issued; ++g)
-          (void)mbar_wait_drain(&full[g % C::kStages], (g / C::kStages) & 1, 1ll << 26);
+        for (int g = (ga > S ? ga - S : 0); g < ga; ++g) (void)mbar_wait_drain(&full[g % S], (g / S) & 1, 1ll << 26);
+        if (is4)
+          for (int g = (gw > C::kRaw ? gw - C::kRaw : 0); g < gw; ++g)
+            (void)mbar_wait_drain(&rfull[g % C::kRaw], (g / C::kRaw) & 1, 1ll << 26);
       }
     } else if (warp == 1 || warp == 3) {
       // ---------------------------------------------------------- MMA issuers
       // Two threads issue alternate groups (warp 1 the even ones, warp 3 the
-      // odd ones): a single issuing thread leaves the tensor pipe idle between
-      // groups, two keep it busy.  Each commits its group to done[g % kAccBufs].
+      // odd ones): one thread pays for every tcgen05.mma and commit it issues
+      // and leaves the tensor pipe idle between groups, two keep it busy.
       if (lane == 0) {
         constexpr uint32_t idesc = idesc_i8(kBM, BN);
         const int who = warp == 1 ? 0 : 1;
         for (int g = who; g < G; g += 2) {
-          const int s = g % C::kStages, b = g & 1, a = g % C::kAccBufs;
-          if (!mbar_wait(&full[s], (g / C::kStages) & 1, abort_flag)) break;
-          if (is4 && !mbar_wait(&tfull[b], (g >> 1) & 1, abort_flag)) break;
-          if (!mbar_wait(&accempty[a], ((g / C::kAccBufs) & 1) ^ 1, abort_flag)) break;
+          const int s = g % S, b = g % C::kTBufs, a = g % C::kAccBufs;
+          if (!mbar_wait(&full[s], (g / S) & 1, abort_flag)) break;
+          if (is4 && !mbar_wait(&tfull[b], (g / C::kTBufs) & 1, abort_flag)) break;
+          // phase 0 of accempty[a] is the epilogue's bias fill; phase u+1 its drain of use u
+          if (!mbar_wait(&accempty[a], (g / C::kAccBufs) & 1, abort_flag)) break;
           tc_fence_after();
           const uint32_t a_addr = smem_u32(stage_a(s));
-          const uint32_t b_addr = smem_u32(is4 ? tbuf(b) : stage_w(s));
+          const uint32_t b_addr = smem_u32(is4 ? tbuf(b) : stage_w8(s));
           const uint32_t d = tmem_base + static_cast<uint32_t>(a * BN);
 #pragma unroll
           for (int kk = 0; kk < kKG / 32; ++kk)
             mma_i8(d, sw128_kmajor_desc(a_addr + 32 * kk), sw128_kmajor_desc(b_addr + 32 * kk), idesc, 1u);
-          mma_commit(&done[a]);
+          mma_commit(&done[g % C::kDone]);
         }
         mma_commit(&drain[who]);
         (void)mbar_wait_drain(&drain[who], 0, 1ll << 28);
       }
-    } else if (warp == 2) {
+    } else {
       // ---------------------------------------------------------- scale table
       // Slot `slot` of group g holds s_w of the tile's BN columns as fp32,
       // followed by s_a of the tile's 128 rows.  Raw scales are prefetched
@@ -271,6 +348,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         cp_async_commit();
       };
       for (int g = 0; g < C::kStgDist; ++g) issue(g);
+      // output channel of every tile column (-1 past the set), published to
+      // the epilogue by the first tabfull arrival
+#pragma unroll
+      for (int i = 0; i < BN / 32; ++i) {
+        const int col = lane + 32 * i;
+        col_idx[col] = n0 + col < Nset ? __ldg(idx + n0 + col) : -1;
+      }
       for (int g = 0; g < G; ++g) {
         const int slot = g % C::kTabSlots, i = g % C::kStgSlots;
         cp_async_wait<C::kStgDist - 1>();
@@ -294,38 +378,55 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_dec<kRegsXform>();
     // ------------------------------------------------------------ 4-bit unpack
     if (is4) {
+      // Thread tt owns the 16-byte column chunk c = tt % 4 (32 nibbles = 32
+      // weights) of rows r0, r0+32, r0+64, r0+96 (r0 = tt / 4): all four loads
+      // are issued before any arithmetic, so one warp per SM sub-partition
+      // keeps several shared-memory loads in flight.
       const int tt = threadIdx.x - 384;  // 0..127
+      const int c = tt & 3, r0 = tt >> 2;
+      const int zshift = (r0 & 1) * 4;   // rows r0 + 32k share r0's parity and swizzle phase
+      const int sw = r0 & 7;
+      constexpr int kRowsPerThread = BN / 32;
       for (int g = 0; g < G; ++g) {
-        const int s = g % C::kStages, b = g & 1;
-        if (!warp_wait(&full[s], (g / C::kStages) & 1, abort_flag)) break;
-        if (g >= 2) {  // tbuf[b] last held group g - 2
-          const int gp = g - 2;
-          if (!warp_wait(&done[gp % C::kAccBufs], (gp / C::kAccBufs) & 1, abort_flag)) break;
+        const int r = g % C::kRaw, b = g % C::kTBufs;
+        if (!warp_wait(&rfull[r], (g / C::kRaw) & 1, abort_flag)) break;
+        // unpacked buffer b last held group g - kTBufs: free once that group is done
+        if (g >= C::kTBufs) {
+          const int gp = g - C::kTBufs;
+          if (!warp_wait(&done[gp % C::kDone], (gp / C::kDone) & 1, abort_flag)) break;
         }
-        const uint8_t *raw = stage_w(s);
-        const uint8_t *zb = zmeta(s);
+        const uint8_t *raw = raw_w4(r);
+        const uint8_t *zb = zmeta(r);
         uint8_t *dst = tbuf(b);
+        uint4 x[kRowsPerThread];
+        uint32_t zz[kRowsPerThread];
 #pragma unroll
-        for (int it = tt; it < BN * 4; it += 32 * kXformWarps) {
-          const int r = it >> 2, c = it & 3;
-          const uint4 x = *reinterpret_cast<const uint4 *>(raw + r * 64 + c * 16);
-          const uint32_t zz = ((zb[r >> 1] >> ((r & 1) * 4)) & 0xFu) * 0x01010101u;
+        for (int k = 0; k < kRowsPerThread; ++k) {
+          const int rr = r0 + 32 * k;
+          x[k] = *reinterpret_cast<const uint4 *>(raw + rr * 64 + c * 16);
+          zz[k] = ((static_cast<uint32_t>(zb[rr >> 1]) >> zshift) & 0xFu) * 0x01010101u;
+        }
+#pragma unroll
+        for (int k = 0; k < kRowsPerThread; ++k) {
+          const int rr = r0 + 32 * k;
           uint4 lo, hi;
-          lo.x = sub_zero_bytes(x.x & 0x0F0F0F0Fu, zz);
-          lo.y = sub_zero_bytes(x.y & 0x0F0F0F0Fu, zz);
-          lo.z = sub_zero_bytes(x.z & 0x0F0F0F0Fu, zz);
-          lo.w = sub_zero_bytes(x.w & 0x0F0F0F0Fu, zz);
-          hi.x = sub_zero_bytes((x.x >> 4) & 0x0F0F0F0Fu, zz);
-          hi.y = sub_zero_bytes((x.y >> 4) & 0x0F0F0F0Fu, zz);
-          hi.z = sub_zero_bytes((x.z >> 4) & 0x0F0F0F0Fu, zz);
-          hi.w = sub_zero_bytes((x.w >> 4) & 0x0F0F0F0Fu, zz);
-          const int sw = r & 7;
-          *reinterpret_cast<uint4 *>(dst + r * 128 + (((2 * c) ^ sw) << 4)) = lo;
-          *reinterpret_cast<uint4 *>(dst + r * 128 + (((2 * c + 1) ^ sw) << 4)) = hi;
+          lo.x = sub_zero_bytes(x[k].x & 0x0F0F0F0Fu, zz[k]);
+          lo.y = sub_zero_bytes(x[k].y & 0x0F0F0F0Fu, zz[k]);
+          lo.z = sub_zero_bytes(x[k].z & 0x0F0F0F0Fu, zz[k]);
+          lo.w = sub_zero_bytes(x[k].w & 0x0F0F0F0Fu, zz[k]);
+          hi.x = sub_zero_bytes((x[k].x >> 4) & 0x0F0F0F0Fu, zz[k]);
+          hi.y = sub_zero_bytes((x[k].y >> 4) & 0x0F0F0F0Fu, zz[k]);
+          hi.z = sub_zero_bytes((x[k].z >> 4) & 0x0F0F0F0Fu, zz[k]);
+          hi.w = sub_zero_bytes((x[k].w >> 4) & 0x0F0F0F0Fu, zz[k]);
+          *reinterpret_cast<uint4 *>(dst + rr * 128 + (((2 * c) ^ sw) << 4)) = lo;
+          *reinterpret_cast<uint4 *>(dst + rr * 128 + (((2 * c + 1) ^ sw) << 4)) = hi;
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tfull[b]);
+        if (lane == 0) {
+          mbar_arrive(&rempty[r]);
+          mbar_arrive(&tfull[b]);
+        }
       }
     }
   } else {
@@ -339,6 +440,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int m = m0 + row;
     const bool row_ok = m < M;
 
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + half * CPT;
+    // Every accumulator starts at the bias 0x4b400000 (and is reset to it after
+    // each drain), so the int32 sum the MMAs leave there, read as a float, is
+    // 1.5*2^23 + P exactly: the bias trick with no per-element integer add.
+#pragma unroll
+    for (int a = 0; a < C::kAccBufs; ++a)
+#pragma unroll
+      for (int c = 0; c < CPT; c += 32) tmem_st_32x32b_x32_fill(lane_base + a * BN + c, kI2FBiasBits);
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0)
+      for (int a = 0; a < C::kAccBufs; ++a) mbar_arrive(&accempty[a]);
+
     float acc[CPT];
 #pragma unroll
     for (int j = 0; j < CPT; ++j) acc[j] = 0.0f;
@@ -347,7 +462,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // and accumulated, the tcgen05.ld of the next one (this group's next
     // chunk, or the next group's first) is in flight.
     constexpr int CW = 16, NCH = CPT / CW;
-    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + half * CPT;
     uint32_t rbuf[2][CW];
     // v = bits of (1.5*2^23 + P) as float; u = fma(v, s_a, -1.5*2^23*s_a) is
     // exactly fl(P * s_a) (the bias term is exact for a bf16-valued s_a); then
@@ -409,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) mbar_arrive(&accempty[a]);
           if (g + 1 < G) {
             const int a1 = (g + 1) % C::kAccBufs;
-            live = warp_wait(&done[a1], ((g + 1) / C::kAccBufs) & 1, abort_flag);
+            live = warp_wait(&done[(g + 1) % C::kDone], ((g + 1) / C::kDone) & 1, abort_flag);
             if (live) {
               tc_fence_after();
               tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(a1 * BN), rbuf[(c + 1) & 1]);
@@ -429,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if constexpr (!kDebugP) {
       // stage fp16 results: row `row`, columns half*CPT .. +CPT
-      uint8_t *st = smem + C::kOffStages;
+      uint8_t *st = smem + C::kOffRing;
       __half2 *dst = reinterpret_cast<__half2 *>(st + row * C::kStagingStride + half * CPT * 2);
 #pragma unroll
       for (int j = 0; j < CPT / 2; ++j) dst[j] = __floats2half2_rn(acc[2 * j], acc[2 * j + 1]);
@@ -437,13 +551,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!*abort_flag) {
         constexpr int CPL = BN / 32;  // columns per lane
         int col_out[CPL];
-        bool col_ok[CPL];
 #pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-          const int col = lane + 32 * i;
-          col_ok[i] = n0 + col < Nset;
-          col_out[i] = col_ok[i] ? __ldg(idx + n0 + col) : 0;
-        }
+        for (int i = 0; i < CPL; ++i) col_out[i] = col_idx[lane + 32 * i];
         for (int rr = e; rr < kBM; rr += kEpiWarps) {
           const int mm = m0 + rr;
           if (mm >= M) break;
@@ -451,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           __half *yrow = Y + static_cast<int64_t>(mm) * N;
 #pragma unroll
           for (int i = 0; i < CPL; ++i)
-            if (col_ok[i]) yrow[col_out[i]] = srow[lane + 32 * i];
+            if (col_out[i] >= 0) yrow[col_out[i]] = srow[lane + 32 * i];
         }
       }
     }
