@@ -232,27 +232,41 @@ def run_ours(args, layer, rank, world, local_rank):
         step()
     mx.sync_status(stream)
 
+    # Timed region: whole steps.  The GEMM is launched as a programmatic
+    # dependent of the quantizer, so nothing is recorded between the two.
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clocks:
         for i in range(K):
             flush.fill_(i & 0xFF)
             ev[i][0].record(stream)
-            mx.quantize_act_into(Xd, A_q, s_a, stream)
+            step()
             ev[i][1].record(stream)
-            mx.gemm_w4w8a8_into(A_q, s_a, p, Y, stream)
-            ev[i][2].record(stream)
         torch.cuda.synchronize()
     barrier(world)
     mx.sync_status(stream)
-    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
-    gemm_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    quant_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    t_step = max_over_ranks(sum(step_ms) / K, world)
-    t_gemm = max_over_ranks(sum(gemm_ms) / K, world)
-    t_quant = max_over_ranks(sum(quant_ms) / K, world)
+    t_step = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / K, world)
+
+    # Per-kernel durations for the roofline: the same steps with an event
+    # between the two kernels (which also keeps the GEMM from starting early,
+    # so this is its stand-alone duration).
+    Kk = min(K, 500)
+    ek = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(Kk)]
+    torch.cuda.synchronize()
+    for i in range(Kk):
+        flush.fill_(i & 0xFF)
+        ek[i][0].record(stream)
+        mx.quantize_act_into(Xd, A_q, s_a, stream)
+        ek[i][1].record(stream)
+        mx.gemm_w4w8a8_into(A_q, s_a, p, Y, stream)
+        ek[i][2].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    mx.sync_status(stream)
+    t_gemm = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ek) / Kk, world)
+    t_quant = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ek) / Kk, world)
 
     # end to end through the public API: pinned host X in, host Y out
     Xh = torch.from_numpy(X).pin_memory()
@@ -304,7 +318,8 @@ def run_ours(args, layer, rank, world, local_rank):
             "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded N(0,1) X with x20 outlier "
             "columns, N(0,0.02) W, random 8-bit channel set)", "config": config_of(layer, world),
             "gemm_kernel": {"ms": t_gemm, "tops": gemm_tops, "frac_of_int8_peak": gemm_tops / int8_peak,
-                            "frac_of_nominal_4500": gemm_tops / 4500.0},
+                            "frac_of_nominal_4500": gemm_tops / 4500.0,
+                            "timed": f"{Kk} launches with an event before and after each, L2 flushed before each"},
             "quantize_act_kernel": {"ms": t_quant,
                                     "gbs": (layer.M * layer.K * 3 + layer.M * layer.G * 4) / (t_quant * 1e-3) / 1e9},
             "roofline": {"bound": "tensor", "achieved": gemm_tops, "peak": int8_peak, "unit": "TOPS",
@@ -315,6 +330,8 @@ def run_ours(args, layer, rank, world, local_rank):
             "e2e": {"value": ops * world / (t_e2e * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": layer.M * layer.K * 2, "d2h_bytes_per_step": layer.M * layer.N * 2},
             "gpu_launches": 2 * K,
+            "step": "quantize_act then the fused GEMM, launched as its programmatic dependent (its "
+                    "prologue overlaps the quantizer's tail; it reads A_q and s_a only after the quantizer ends)",
             "clocks": clocks.summary(),
         }
     return line

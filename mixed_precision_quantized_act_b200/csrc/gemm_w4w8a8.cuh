@@ -107,8 +107,8 @@ struct GemmCfg {
   static constexpr int kColsPerThread = BN * kBM / kEpiThreads;  // 64
   static constexpr int kTabSwBytes = BN * 4;                   // s_w of the tile's columns (fp32)
   static constexpr int kTabBytes = kTabSwBytes + kBM * 4;      // + s_a of the tile's rows
-  static constexpr int kStgSlots = 8;                          // raw scale staging ring
-  static constexpr int kStgDist = 6;                           // groups prefetched ahead
+  static constexpr int kStgSlots = 12;                         // raw scale staging ring
+  static constexpr int kStgDist = 10;                          // groups prefetched ahead
   static constexpr int kStgBytes = BN * 2 + kBM * 4;           // raw fp16 s_w + fp32 s_a
   // L2 prefetch distance in groups, past the loads the ring already holds
   static constexpr int kPrefetchAhead = 4;
@@ -221,6 +221,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // Weights do not depend on the kernel before this one: hint the first
+    // tiles into L2 while it may still be running (launched as a programmatic
+    // dependent, this CTA can start before the activation quantizer ends).
+    for (int g = 0; g < S && g < G; ++g) {
+      if (is4) tma_prefetch_l2_2d(&tmW4, g * (kKG / 2), n0); else tma_prefetch_l2_2d(&tmW8, g * kKG, n0);
+    }
+    // Every global read of this grid comes after this wait: here, in the
+    // table warp, and in the roles ordered after these loads by barriers.
+    pdl_wait();
     // the first stages need nothing but their barriers: start them before the CTA-wide sync
     for (int g = 0; g < S && g < G; ++g) load_a(g);
   }
@@ -347,6 +356,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         cp_async_commit();
       };
+      pdl_wait();
+      // The row scales of this tile are whole rows of s_a [M, G] (one
+      // contiguous range) and its column scales one 2*BN-byte piece per group:
+      // bring both into L2 first, so the scattered 4-byte reads below hit there.
+      if (lane == 0) {
+        const int rows = M - m0 < kBM ? M - m0 : kBM;
+        const uint32_t sa_bytes = static_cast<uint32_t>(rows) * static_cast<uint32_t>(G) * 4u;
+        const float *sa_rows = s_a + static_cast<int64_t>(m0) * G;  // s_a is only 4-byte aligned
+        if (sa_bytes >= 16 && (reinterpret_cast<uintptr_t>(sa_rows) & 15u) == 0) bulk_prefetch_l2(sa_rows, sa_bytes & ~15u);
+      }
+      for (int g = lane; g < G; g += 32) bulk_prefetch_l2(s_w + static_cast<int64_t>(g) * Np + n0, BN * 2);
       for (int g = 0; g < C::kStgDist; ++g) issue(g);
       // output channel of every tile column (-1 past the set), published to
       // the epilogue by the first tabfull arrival
@@ -649,12 +669,25 @@ static cudaError_t launch_gemm_bn(const GemmArgs &a, cudaStream_t stream, const 
     }
     configured |= 1ull << dev;
   }
-  kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemAlloc, stream>>>(
-      tmA, tmW4, tmW8, a.s_a, a.z4, static_cast<const __half *>(a.s_w4), a.idx4,
+  // Launched as a programmatic dependent of the previous kernel in the stream:
+  // the CTAs set up barriers and TMEM while that kernel finishes, and wait for
+  // it (griddepcontrol.wait) before their first global read.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmemAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(
+      &cfg, kern, tmA, tmW4, tmW8, a.s_a, a.z4, static_cast<const __half *>(a.s_w4), a.idx4,
       static_cast<const __half *>(a.s_w8), a.idx8, static_cast<int>(a.M), static_cast<int>(a.K),
       static_cast<int>(a.N4), static_cast<int>(a.N8), static_cast<int>(padded_channels(a.N4)),
       static_cast<int>(padded_channels(a.N8)), mt, nt4, static_cast<__half *>(a.Y), a.P);
-  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) *msg = "launch of the fused GEMM failed";
   return e;
 }

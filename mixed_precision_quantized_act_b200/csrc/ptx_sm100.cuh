@@ -109,6 +109,17 @@ __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
 }
 
+// ----------------------------------------------------------------- programmatic dependent launch
+
+// Lets the next kernel in the stream, if it was launched as a programmatic
+// dependent, start its CTAs (their prologue overlaps this grid's tail).
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Blocks until the grids this one depends on have completed and their writes
+// are visible; returns at once when there are none.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ----------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *m) {

@@ -23,11 +23,27 @@ namespace mixllm {
 // rounded to bfloat16 precision and kept as fp32), q = clamp(round_half_even(
 // x / s_a), -127, 127); amax == 0 gives s_a = q = 0.  The bf16 scale keeps the
 // RTN error within s_a/2 and makes 1.5*2^23*s_a exact for the GEMM epilogue.
-// The division is the correctly rounded one (not a reciprocal multiply) so
-// that the codes are the same as a plain CPU evaluation of the definition.
+//
+// The codes are those of rint(fl(x / s_a)), the plain CPU evaluation of the
+// definition, without a division per element:
+//   * fl(x/s) never crosses or lands on a half-integer k + 1/2 unless x/s is
+//     exactly k + 1/2: with x = mx 2^a (fp16, |mx| < 2^11) and s = ms 2^b
+//     (bf16, 2^7 <= ms < 2^8), x/s - (k + 1/2) = (mx 2^(a+1) - (2k+1) ms 2^b)
+//     / (2 ms 2^b) is, when non-zero, at least 2^-12 in magnitude for every
+//     |x/s| >= 1/2 (smaller quotients round to 0 either way), far above the
+//     2^-17 that fl() can move a quotient below 128.  So rint(fl(x/s)) is
+//     round_half_even of the exact quotient.
+//   * That is computed from q0 = rint(x * (1/s)), which is off by at most one,
+//     and the remainder e = x - q0*s, which one FMA gives exactly (q0*s has at
+//     most 15 significant bits and e is a multiple of the smaller of the two
+//     operands' last places, below 2^13 of them): |e| < s/2 keeps q0, |e| >
+//     s/2 moves q0 one step toward e, |e| = s/2 is a tie and picks the even one.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) quantize_act_kernel(const __half *__restrict__ X, int64_t M, int64_t K,
                                                            int8_t *__restrict__ A_q, float *__restrict__ s_a) {
+  // the GEMM that consumes A_q and s_a may start its prologue now; it reads
+  // them only after this grid has completed
+  pdl_launch_dependents();
   const int64_t G = K >> 7;
   const int64_t total = M * G;
   const int lane16 = threadIdx.x & 15;
@@ -53,11 +69,17 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const __half *__restr
     const float s = __bfloat162float(__float2bfloat16_rn(__fdiv_rn(amax, 127.0f)));
     uint32_t packed[2] = {0u, 0u};
     if (s != 0.0f) {
+      const float r = __frcp_rn(s);
+      const float half_s = 0.5f * s;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        int q = __float2int_rn(__fdiv_rn(x[i], s));
-        q = max(-127, min(127, q));
-        packed[i >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << ((i & 3) * 8);
+        const int q0 = __float2int_rn(x[i] * r);
+        const float e = __fmaf_rn(-static_cast<float>(q0), s, x[i]);  // exact remainder x - q0*s
+        const float ae = fabsf(e);
+        int qi = q0;
+        if (ae > half_s || (ae == half_s && (q0 & 1))) qi += e > 0.0f ? 1 : -1;
+        qi = max(-127, min(127, qi));
+        packed[i >> 2] |= (static_cast<uint32_t>(qi) & 0xFFu) << ((i & 3) * 8);
       }
     }
     *reinterpret_cast<uint2 *>(A_q + off) = make_uint2(packed[0], packed[1]);

@@ -91,6 +91,56 @@ def test_quantize_act_special_values(dev):
     assert np.array_equal(s_a.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
 
 
+def _tie_groups():
+    """Groups whose scale is known exactly (amax = 127 * s0, s0 bf16-valued and
+    127 * s0 fp16-valued), filled with the exact half-integer multiples
+    (k + 1/2) * s0 that fp16 holds and with their fp16 neighbours on both sides:
+    rounding ties and the values that must not be taken for ties."""
+    rows = []
+    for s0 in (2.0 ** -4, 3.0 / 256, 5.0 * 2 ** -10, 0.75, 1.5, 192.0, 2.0 ** -20):
+        top = np.float16(127 * s0)
+        assert float(top) == 127 * s0
+        ties = []
+        for k in range(-127, 127):
+            v = np.float16((k + 0.5) * s0)
+            if float(v) == (k + 0.5) * s0 and abs(float(v)) < 127 * s0:
+                ties.append(v)
+        ties = np.array(ties, np.float16)
+        up = np.nextafter(ties, np.float16(np.inf))
+        dn = np.nextafter(ties, np.float16(-np.inf))
+        pool = np.concatenate([ties, up, dn])
+        pool = pool[np.abs(pool.astype(np.float64)) < 127 * s0]
+        for start in range(0, len(pool), 127):
+            g = np.zeros(128, np.float16)
+            g[0] = top if start % 2 == 0 else -top
+            chunk = pool[start:start + 127]
+            g[1:1 + len(chunk)] = chunk
+            rows.append(g)
+    G = 4
+    rows += [np.zeros(128, np.float16)] * ((-len(rows)) % G)
+    return np.stack(rows).reshape(-1, 128 * G)
+
+
+def test_quantize_act_ties_and_near_ties(dev):
+    X = _tie_groups()
+    A_q, s_a = mx.quantize_act(torch.from_numpy(X).to(dev))
+    A_ref, s_ref = oracle.quantize_act(X)
+    assert np.array_equal(s_a.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(A_q.cpu().numpy(), A_ref)
+
+
+def test_quantize_act_wide_magnitudes(dev):
+    # every group at its own scale, from fp16 subnormals to near the fp16 maximum
+    rng = np.random.default_rng(17)
+    M, K = 256, 2048
+    scale = np.exp2(rng.uniform(-24, 15, size=(M, K // 128, 1)))
+    X = (rng.standard_normal((M, K // 128, 128)) * scale).clip(-65504, 65504).astype(np.float16).reshape(M, K)
+    A_q, s_a = mx.quantize_act(torch.from_numpy(X).to(dev))
+    A_ref, s_ref = oracle.quantize_act(X)
+    assert np.array_equal(s_a.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(A_q.cpu().numpy(), A_ref)
+
+
 def test_quantize_act_empty(dev):
     A_q, s_a = mx.quantize_act(torch.zeros((0, 256), dtype=torch.float16, device=dev))
     mx.sync_status()
