@@ -180,6 +180,47 @@ MIXLLM_API mixllm_status mixllm_gemm_debug_partials(const int8_t *A_q, const flo
                                          int32_t *P, void *stream);
 
 /*
+ * Bytes of workspace mixllm_gemm_w4w8a8_small_m needs for this shape (0 when
+ * the shape is not split along K), in *bytes.  Pure host function.
+ * Requires 1 <= M <= 64 and K a positive multiple of 128.
+ */
+MIXLLM_API mixllm_status mixllm_small_m_workspace_bytes(int64_t M, int64_t K, int64_t N4, int64_t N8,
+                                             size_t *bytes);
+
+/*
+ * The same layer and the same result rule as mixllm_gemm_w4w8a8, laid out
+ * for few tokens (1 <= M <= 64, the decode regime, where the packed weights
+ * are nearly all the bytes and HBM bandwidth bounds the layer): the weight
+ * tile is the tensor core's 128-row side and the tokens its 16/32/64-column
+ * side, and the groups of every 128-channel tile are split among several
+ * CTAs so the grid fills the GPU.  Each split writes fp32 partial sums to the
+ * workspace; the last split of a tile to finish adds them in split order (the
+ * result does not depend on timing) and writes Y.  The rounding differs from
+ * mixllm_gemm_w4w8a8 only in the order of the fp32 operations (Y is within
+ * the same tolerance of the reference definition).
+ * Arguments: as mixllm_gemm_w4w8a8, plus
+ *   workspace        device, at least mixllm_small_m_workspace_bytes() bytes,
+ *                    16-byte aligned, owned by the caller: fp32 partial sums
+ *                    followed by one int32 counter per 128-channel tile.  It
+ *                    must be zero-filled before its first use; every call
+ *                    returns the counters to zero (the partial sums are
+ *                    scratch), so it stays ready for the next call.  Two calls
+ *                    that run at the same time must not share one.  After a
+ *                    MIXLLM_ERR_TIMEOUT zero it again.  May be NULL when the
+ *                    size is 0.
+ *   workspace_bytes  its size.
+ * Asynchronous on `stream`.  Returns MIXLLM_ERR_INVALID_ARG for M > 64 or a
+ * workspace that is too small.
+ */
+MIXLLM_API mixllm_status mixllm_gemm_w4w8a8_small_m(const int8_t *A_q, const float *s_a, int64_t M, int64_t K,
+                                         const uint8_t *W4, const uint8_t *z4, const void *s_w4_f16,
+                                         const int32_t *idx4, int64_t N4,
+                                         const int8_t *W8, const void *s_w8_f16,
+                                         const int32_t *idx8, int64_t N8,
+                                         void *Y_f16, void *workspace, size_t workspace_bytes,
+                                         void *stream);
+
+/*
  * Waits for `stream`, then reads and clears the device status word of the
  * current device.  Returns MIXLLM_ERR_TIMEOUT if a kernel of this library
  * gave up a wait since the last call, MIXLLM_ERR_CUDA if the stream reports

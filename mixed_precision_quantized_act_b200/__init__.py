@@ -7,11 +7,14 @@ synthetic workloads used by the tests and the benchmark.
 from ._lib import (  # noqa: F401
     GROUP,
     MixLLMError,
+    SMALL_M_MAX,
     PackedLinear,
     empty_packed,
     gemm_debug_partials,
     gemm_w4w8a8,
     gemm_w4w8a8_into,
+    gemm_w4w8a8_small_m,
+    gemm_w4w8a8_small_m_into,
     linear,
     load,
     pack_weights,
@@ -19,6 +22,8 @@ from ._lib import (  # noqa: F401
     quantize_act,
     quantize_act_into,
     selftest_wait_timeout,
+    small_m_workspace,
+    small_m_workspace_bytes,
     sync_status,
     version,
 )

@@ -33,6 +33,9 @@ SIGNATURES = {
                                           _vp, _vp, _vp, _i64, _vp, _vp]),
     "mixllm_gemm_debug_partials": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64,
                                                   _vp, _vp, _vp, _i64, _vp, _vp]),
+    "mixllm_small_m_workspace_bytes": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(ctypes.c_size_t)]),
+    "mixllm_gemm_w4w8a8_small_m": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64,
+                                                  _vp, _vp, _vp, _i64, _vp, _vp, ctypes.c_size_t, _vp]),
     "mixllm_sync_status": (ctypes.c_int, [_vp]),
     "mixllm_selftest_wait_timeout": (ctypes.c_int, [_u32, _vp]),
 }
@@ -203,9 +206,48 @@ def gemm_debug_partials(A_q, s_a, p: PackedLinear, stream=None) -> torch.Tensor:
     return P
 
 
-def linear(X: torch.Tensor, p: PackedLinear, stream=None) -> torch.Tensor:
-    """The whole layer: quantize X then run the fused GEMM."""
+SMALL_M_MAX = 64
+
+
+def small_m_workspace_bytes(M: int, K: int, N4: int, N8: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(load().mixllm_small_m_workspace_bytes(M, K, N4, N8, ctypes.byref(out)), "mixllm_small_m_workspace_bytes")
+    return out.value
+
+
+def small_m_workspace(M: int, p: PackedLinear, device) -> torch.Tensor:
+    """A zero-filled workspace for mixllm_gemm_w4w8a8_small_m (every call
+    returns its tile counters, the last 4 bytes per 128-channel tile, to zero)."""
+    n = small_m_workspace_bytes(M, p.K, p.N4, p.N8)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def gemm_w4w8a8_small_m_into(A_q, s_a, p: PackedLinear, Y, workspace: torch.Tensor, stream=None):
+    _need_cuda(A_q, s_a, Y, workspace)
+    M, K = A_q.shape
+    assert K == p.K and Y.shape == (M, p.N) and Y.dtype == torch.float16 and Y.is_contiguous()
+    assert workspace.is_contiguous()
+    _check(load().mixllm_gemm_w4w8a8_small_m(_ptr(A_q), _ptr(s_a), M, K, _ptr(p.W4), _ptr(p.z4), _ptr(p.s_w4),
+                                             _ptr(p.idx4), p.N4, _ptr(p.W8), _ptr(p.s_w8), _ptr(p.idx8), p.N8,
+                                             _ptr(Y), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                             _stream(stream)), "mixllm_gemm_w4w8a8_small_m")
+
+
+def gemm_w4w8a8_small_m(A_q, s_a, p: PackedLinear, workspace: torch.Tensor = None, stream=None) -> torch.Tensor:
+    M = A_q.shape[0]
+    if workspace is None:
+        workspace = small_m_workspace(M, p, A_q.device)
+    Y = torch.empty((M, p.N), dtype=torch.float16, device=A_q.device)
+    gemm_w4w8a8_small_m_into(A_q, s_a, p, Y, workspace, stream)
+    return Y
+
+
+def linear(X: torch.Tensor, p: PackedLinear, stream=None, workspace: torch.Tensor = None) -> torch.Tensor:
+    """The whole layer: quantize X then run the fused GEMM (the few-token
+    variant for M <= 64, with `workspace` or a fresh zero-filled one)."""
     A_q, s_a = quantize_act(X, stream)
+    if 0 < A_q.shape[0] <= SMALL_M_MAX:
+        return gemm_w4w8a8_small_m(A_q, s_a, p, workspace, stream)
     return gemm_w4w8a8(A_q, s_a, p, stream)
 
 

@@ -1,0 +1,548 @@
+// gemm_small_m.cuh -- the W4.4A8 layer for few tokens (M <= 64) on sm_100a.
+//
+// Same arithmetic as the tiled kernel (MLSys 2026 talk notes on MixLLM,
+// notes.yuuk.io, §二段階逆量子化による int8 Tensor Core 活用, §高速 I2F 変換,
+// §並列実行): per quantization group g of 128 along K,
+//     P_g  = sum_{k in g} (W_q - z) * A_q          int8 MMA, int32 exact
+//     acc += float(P_g) * s_w[n,g] * s_a[m,g]      fp32
+// and Y[m, idx[n]] = fp16(acc).  With a handful of tokens the layer is bound
+// by HBM (the packed weights are nearly all the bytes), so the work is laid
+// out for bandwidth rather than for the tensor pipe:
+//   * operands swapped: the weight tile is the MMA's M = 128 side (TMEM lane =
+//     output channel) and the tokens its N side (Mp = 16, 32 or 64 columns), so
+//     the per-group drain is 128 x Mp values instead of 128 x 128, and the
+//     channel scale is a per-thread constant (the bias fold uses s_w:
+//     u = fma(v, s_w, -1.5*2^23*s_w) = fl(P*s_w), exact because s_w is fp16);
+//   * split-K: the groups of every 128-channel tile are divided among S CTAs
+//     so that the grid fills the SMs; each CTA writes its fp32 partial sums to
+//     a workspace and the last CTA of a tile to finish (an atomic counter, no
+//     waiting) adds the S partials in split order -- the result does not
+//     depend on which CTA finishes last -- and writes the fp16 outputs.  The
+//     counter is reset by that CTA, so the counters are zero between calls.
+// Roles (512 threads, registers rebalanced per warpgroup with setmaxnreg):
+// warp 0 TMA producer (weight tile, zero points and the token tile of each
+// group into a ring of stages), warp 1 MMA issuer (one commit per group),
+// warp 2 scale tables (this CTA's groups, loaded once), warps 4-11 4-bit
+// unpack into the swizzled int8 operand (with few tokens it is the longest
+// per-group step), warps 12-15 epilogue (one TMEM lane quadrant each).  Every
+// wait is bounded as in the tiled kernel.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cudaTypedefs.h>
+#include <cstdint>
+
+#include "launch.h"
+#include "ptx_sm100.cuh"
+
+namespace mixllm {
+
+constexpr int kSmThreads = 512;
+constexpr int kSmUnpackWarps = 8;  // warps 4..11
+// registers per thread after setmaxnreg, per warpgroup: control, unpack (two), epilogue;
+// 128 * kSmRegsCtl + 256 * kSmRegsUnpack + 128 * kSmRegsEpi <= 512 * 128
+constexpr int kSmRegsCtl = 88, kSmRegsUnpack = 72, kSmRegsEpi = 200;
+static_assert(128 * kSmRegsCtl + 256 * kSmRegsUnpack + 128 * kSmRegsEpi <= 65536, "register split");
+constexpr int kSmGroupsMax = 32;  // groups per CTA (bounds the scale tables)
+
+template <int MP>
+struct SmallMCfg {
+  static_assert(MP == 16 || MP == 32 || MP == 64, "token tile");
+  // The ring holds as many stages as fit (all of a CTA's groups when they
+  // fit, so one round of loads covers the whole K range): a stage is the
+  // weight tile (int8 16 KB, or packed 4-bit 8 KB) followed by the token tile.
+  static constexpr int kRingBytes = 160 * 1024;
+  static constexpr int kMaxStages = 16;
+  static constexpr int kTBufs = 2;
+  static constexpr int kAccBufs = 4;
+  static constexpr int kDone = kMaxStages;              // >= every ring released through it
+  static_assert(kDone >= kTBufs && kDone >= kAccBufs, "done ring");
+  static constexpr int kWBytes = 128 * 128;             // int8 weight tile (W8), or the unpacked 4-bit tile
+  static constexpr int kW4Bytes = 128 * 64;             // packed 4-bit tile
+  static constexpr int kXBytes = MP * 128;              // token tile of one group
+  static constexpr int kTmemCols = kAccBufs * MP < 32 ? 32 : kAccBufs * MP;
+  // shared-memory layout (offsets from a 1024-byte aligned base)
+  static constexpr int kOffStages = 0;
+  static constexpr int kOffTBuf = kOffStages + kRingBytes;
+  static constexpr int kOffZ = kOffTBuf + kTBufs * kWBytes;
+  static constexpr int kOffSw = kOffZ + kMaxStages * 64;               // fp16 s_w [groups][128]
+  static constexpr int kOffSa = kOffSw + kSmGroupsMax * 128 * 4;       // fp32 s_a [groups][MP]
+  static constexpr int kOffBar = kOffSa + kSmGroupsMax * MP * 4;
+  static constexpr int kNumBars = kMaxStages + kDone + kTBufs + kAccBufs + 2;  // + table ready, drain
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16;
+  static constexpr int kSmemAlloc = kSmemBytes + 1024;
+  static_assert(kXBytes % 1024 == 0 && kRingBytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+  static_assert(kWBytes + kXBytes <= kRingBytes, "one stage must fit");
+  static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
+};
+
+// Workspace of one call: S x tiles x MP x 128 fp32 partial sums (scratch),
+// then one int32 counter per tile (zero between calls).
+struct SmallMPlan {
+  int mp, nt4, nt8, splits, groups;
+  size_t part_floats, counters;
+  size_t bytes() const { return part_floats * 4 + counters * 4; }
+};
+
+// Atomic add at GPU scope with acquire-release semantics; returns the old value.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int *p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// bytes of w with 0x80 set, minus z in every byte, then back to two's complement:
+// byte i of the result is (w_i - z) as int8 for w_i, z in [0, 15].
+__device__ __forceinline__ uint32_t sm_sub_zero_bytes(uint32_t w, uint32_t zz) {
+  return ((w | 0x80808080u) - zz) ^ 0x80808080u;
+}
+
+// MP consecutive TMEM columns of this warp's 32 lanes into r (x16 / x32 loads).
+template <int MP>
+__device__ __forceinline__ void sm_tmem_ld(uint32_t taddr, uint32_t (&r)[MP]) {
+  if constexpr (MP == 16) {
+    tmem_ld_32x32b_x16(taddr, r);
+  } else {
+#pragma unroll
+    for (int c = 0; c < MP / 32; ++c) tmem_ld_32x32b_x32(taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * c));
+  }
+}
+template <int MP>
+__device__ __forceinline__ void sm_tmem_fill(uint32_t taddr, uint32_t v) {
+  if constexpr (MP == 16) {
+    tmem_st_32x32b_x16_fill(taddr, v);
+  } else {
+#pragma unroll
+    for (int c = 0; c < MP / 32; ++c) tmem_st_32x32b_x32_fill(taddr + 32 * c, v);
+  }
+}
+template <int MP>
+__device__ __forceinline__ void sm_reg_fence(uint32_t (&r)[MP]) {
+  if constexpr (MP == 16) {
+    reg_fence(r);
+  } else {
+#pragma unroll
+    for (int c = 0; c < MP / 32; ++c) reg_fence(*reinterpret_cast<uint32_t(*)[32]>(r + 32 * c));
+  }
+}
+
+template <int MP>
+__global__ void __launch_bounds__(kSmThreads, 1)
+    gemm_small_m_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW4,
+                        const __grid_constant__ CUtensorMap tmW8, const float *__restrict__ s_a,
+                        const uint8_t *__restrict__ z4, const __half *__restrict__ s_w4,
+                        const int32_t *__restrict__ idx4, const __half *__restrict__ s_w8,
+                        const int32_t *__restrict__ idx8, int M, int K, int N4, int N8, int N4p, int N8p, int nt4,
+                        int ntiles, int S, __half *__restrict__ Y, float *__restrict__ ws_part,
+                        int *__restrict__ ws_cnt) {
+  using C = SmallMCfg<MP>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
+  uint64_t *full = bars;                      // TMA -> unpack / MMA   (per stage)
+  uint64_t *done = full + C::kMaxStages;      // MMA commit of local group i (ring of kDone)
+  uint64_t *tfull = done + C::kDone;          // unpack -> MMA         (per unpacked buffer)
+  uint64_t *accempty = tfull + C::kTBufs;     // epilogue -> MMA       (per accumulator)
+  uint64_t *tabready = accempty + C::kAccBufs;  // scale tables loaded
+  uint64_t *drain = tabready + 1;             // MMA issuer's final commit
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kOffMisc + 4);
+  volatile int *last_flag = reinterpret_cast<volatile int *>(smem + C::kOffMisc + 8);
+  float *tab_sw = reinterpret_cast<float *>(smem + C::kOffSw);
+  float *tab_sa = reinterpret_cast<float *>(smem + C::kOffSa);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x / S, split = blockIdx.x - tile * S;
+  const bool is4 = tile < nt4;
+  const int n0 = (is4 ? tile : tile - nt4) * 128;
+  const int G = K >> 7;
+  const int g0 = static_cast<int>((static_cast<int64_t>(split) * G) / S);
+  const int g1 = static_cast<int>((static_cast<int64_t>(split + 1) * G) / S);
+  const int ng = g1 - g0;  // 1 .. kSmGroupsMax (the host sizes S so)
+  const int Nset = is4 ? N4 : N8;
+  const int Np = is4 ? N4p : N8p;
+  const int N = N4 + N8;
+  const __half *s_w = is4 ? s_w4 : s_w8;
+  const int32_t *idx = is4 ? idx4 : idx8;
+
+  // stage = weight tile (packed 4-bit or int8) + token tile; as many as fit
+  const int wbytes = is4 ? C::kW4Bytes : C::kWBytes;
+  const int stage_sz = wbytes + C::kXBytes;  // a multiple of 1024
+  const int nst = C::kRingBytes / stage_sz < C::kMaxStages ? C::kRingBytes / stage_sz : C::kMaxStages;
+  auto stage_w = [&](int s) { return smem + C::kOffStages + s * stage_sz; };
+  auto stage_x = [&](int s) { return smem + C::kOffStages + s * stage_sz + wbytes; };
+  auto tbuf = [&](int b) { return smem + C::kOffTBuf + b * C::kWBytes; };
+  auto zmeta = [&](int s) { return smem + C::kOffZ + s * 64; };
+  const uint32_t stage_bytes = static_cast<uint32_t>(C::kXBytes + (is4 ? C::kW4Bytes + 64 : C::kWBytes));
+  auto load = [&](int i) {  // local group i of this CTA into stage i % nst
+    const int s = i % nst, g = g0 + i;
+    mbar_arrive_expect_tx(&full[s], stage_bytes);
+    tma_load_2d(stage_x(s), &tmX, &full[s], g * 128, 0);
+    if (is4) {
+      tma_load_2d(stage_w(s), &tmW4, &full[s], g * 64, n0);
+      bulk_load(zmeta(s), z4 + static_cast<int64_t>(g) * (N4p >> 1) + (n0 >> 1), 64, &full[s]);
+    } else {
+      tma_load_2d(stage_w(s), &tmW8, &full[s], g * 128, n0);
+    }
+  };
+
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmX);
+    if (is4) prefetch_tmap(&tmW4); else prefetch_tmap(&tmW8);
+    for (int s = 0; s < C::kMaxStages; ++s) mbar_init(&full[s], 1);
+    for (int i = 0; i < C::kDone; ++i) mbar_init(&done[i], 1);
+    for (int b = 0; b < C::kTBufs; ++b) mbar_init(&tfull[b], kSmUnpackWarps);
+    for (int a = 0; a < C::kAccBufs; ++a) mbar_init(&accempty[a], 4);
+    mbar_init(tabready, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *last_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp < 4) {
+    regs_dec<kSmRegsCtl>();
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      // every global read of this grid comes after this wait (here, in the
+      // scale warp, or in roles ordered after these loads by barriers)
+      pdl_wait();
+      int issued = ng < nst ? ng : nst;
+      for (int i = 0; i < issued; ++i) load(i);
+      for (int i = nst; i < ng; ++i) {
+        const int ip = i - nst;  // the stage last held local group ip
+        if (!mbar_wait(&done[ip % C::kDone], (ip / C::kDone) & 1, abort_flag)) break;
+        load(i);
+        issued = i + 1;
+      }
+      for (int i = (issued > nst ? issued - nst : 0); i < issued; ++i)
+        (void)mbar_wait_drain(&full[i % nst], (i / nst) & 1, 1ll << 26);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(128, MP);
+      for (int i = 0; i < ng; ++i) {
+        const int s = i % nst, b = i % C::kTBufs, a = i % C::kAccBufs;
+        if (!mbar_wait(&full[s], (i / nst) & 1, abort_flag)) break;
+        if (is4 && !mbar_wait(&tfull[b], (i / C::kTBufs) & 1, abort_flag)) break;
+        // phase 0 of accempty[a] is the epilogue's bias fill, phase u+1 its drain of use u
+        if (!mbar_wait(&accempty[a], (i / C::kAccBufs) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(is4 ? tbuf(b) : stage_w(s));  // weights: 128 channels x 128 k
+        const uint32_t b_addr = smem_u32(stage_x(s));                   // tokens: MP rows x 128 k
+        const uint32_t d = tmem_base + static_cast<uint32_t>(a * MP);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_i8(d, sw128_kmajor_desc(a_addr + 32 * kk), sw128_kmajor_desc(b_addr + 32 * kk), idesc, 1u);
+        mma_commit(&done[i % C::kDone]);
+      }
+      mma_commit(drain);
+      (void)mbar_wait_drain(drain, 0, 1ll << 28);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ scale tables
+    // One batch of asynchronous copies for all of this CTA's groups, then a
+    // single wait: s_w (fp16, 8 bytes per lane per group, contiguous per
+    // group) and s_a (4 bytes per token per group; zero for padding tokens).
+    pdl_wait();
+    __half *tsw = reinterpret_cast<__half *>(tab_sw);
+    for (int i = 0; i < ng; ++i)
+      cp_async_8(tsw + i * 128 + 4 * lane, s_w + static_cast<int64_t>(g0 + i) * Np + n0 + 4 * lane);
+    for (int e = lane; e < ng * MP; e += 32) {
+      const int i = e / MP, t = e - i * MP;
+      const bool in = t < M;
+      cp_async_4(tab_sa + e, s_a + (in ? static_cast<int64_t>(t) * G + g0 + i : 0), in ? 4u : 0u);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(tabready);
+  }
+  } else if (warp < 12) {
+    regs_dec<kSmRegsUnpack>();
+    // ------------------------------------------------------------ 4-bit unpack
+    // Thread tt owns the 16-byte column chunk c = tt % 4 (32 weights) of rows
+    // r0 and r0 + 64 (r0 = tt / 4).
+    if (is4) {
+      const int tt = threadIdx.x - 128;  // 0..255
+      const int c = tt & 3, r0 = tt >> 2;
+      const int zshift = (r0 & 1) * 4;
+      const int sw = r0 & 7;
+      for (int i = 0; i < ng; ++i) {
+        const int s = i % nst, b = i % C::kTBufs;
+        if (!warp_wait(&full[s], (i / nst) & 1, abort_flag)) break;
+        if (i >= C::kTBufs) {  // buffer b last held local group i - kTBufs
+          const int ip = i - C::kTBufs;
+          if (!warp_wait(&done[ip % C::kDone], (ip / C::kDone) & 1, abort_flag)) break;
+        }
+        const uint8_t *raw = stage_w(s);
+        const uint8_t *zb = zmeta(s);
+        uint8_t *dst = tbuf(b);
+        uint4 x[2];
+        uint32_t zz[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int rr = r0 + 64 * k;
+          x[k] = *reinterpret_cast<const uint4 *>(raw + rr * 64 + c * 16);
+          zz[k] = ((static_cast<uint32_t>(zb[rr >> 1]) >> zshift) & 0xFu) * 0x01010101u;
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int rr = r0 + 64 * k;
+          uint4 lo, hi;
+          lo.x = sm_sub_zero_bytes(x[k].x & 0x0F0F0F0Fu, zz[k]);
+          lo.y = sm_sub_zero_bytes(x[k].y & 0x0F0F0F0Fu, zz[k]);
+          lo.z = sm_sub_zero_bytes(x[k].z & 0x0F0F0F0Fu, zz[k]);
+          lo.w = sm_sub_zero_bytes(x[k].w & 0x0F0F0F0Fu, zz[k]);
+          hi.x = sm_sub_zero_bytes((x[k].x >> 4) & 0x0F0F0F0Fu, zz[k]);
+          hi.y = sm_sub_zero_bytes((x[k].y >> 4) & 0x0F0F0F0Fu, zz[k]);
+          hi.z = sm_sub_zero_bytes((x[k].z >> 4) & 0x0F0F0F0Fu, zz[k]);
+          hi.w = sm_sub_zero_bytes((x[k].w >> 4) & 0x0F0F0F0Fu, zz[k]);
+          *reinterpret_cast<uint4 *>(dst + rr * 128 + (((2 * c) ^ sw) << 4)) = lo;
+          *reinterpret_cast<uint4 *>(dst + rr * 128 + (((2 * c + 1) ^ sw) << 4)) = hi;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tfull[b]);
+      }
+    }
+  } else {
+    regs_inc<kSmRegsEpi>();
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;        // TMEM lane quadrant: channels q*32 .. q*32+31 of the tile
+    const int c = q * 32 + lane;   // this thread's channel in the tile
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    // Every accumulator starts at the bias 0x4b400000 and is reset to it after
+    // each drain, so the int32 sum read as a float is 1.5*2^23 + P exactly.
+#pragma unroll
+    for (int a = 0; a < C::kAccBufs; ++a) sm_tmem_fill<MP>(lane_base + static_cast<uint32_t>(a * MP), kI2FBiasBits);
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0)
+      for (int a = 0; a < C::kAccBufs; ++a) mbar_arrive(&accempty[a]);
+
+    float acc[MP];
+#pragma unroll
+    for (int t = 0; t < MP; ++t) acc[t] = 0.0f;
+    bool live = warp_wait(tabready, 0, abort_flag);
+    for (int i = 0; live && i < ng; ++i) {
+      const int a = i % C::kAccBufs;
+      if (!warp_wait(&done[i % C::kDone], (i / C::kDone) & 1, abort_flag)) {
+        live = false;
+        break;
+      }
+      tc_fence_after();
+      // v = bits of (1.5*2^23 + P) as float; u = fma(v, s_w, -1.5*2^23*s_w) is
+      // exactly fl(P * s_w) (the bias term is exact for an fp16-valued s_w);
+      // then acc[t] += u * s_a[t] for every token t.
+      const float sw = __half2float(reinterpret_cast<const __half *>(tab_sw)[i * 128 + c]);
+      const float2 sw2 = make_float2(sw, sw);
+      const float2 cb2 = make_float2(-kI2FBias * sw, -kI2FBias * sw);
+      const float2 *sa2 = reinterpret_cast<const float2 *>(tab_sa + i * MP);
+      constexpr int CH = 16;  // columns per tcgen05.ld
+#pragma unroll
+      for (int h = 0; h < MP / CH; ++h) {
+        uint32_t r[CH];
+        const uint32_t col = lane_base + static_cast<uint32_t>(a * MP + h * CH);
+        sm_tmem_ld<CH>(col, r);
+        tmem_ld_wait();
+        sm_reg_fence<CH>(r);
+        sm_tmem_fill<CH>(col, kI2FBiasBits);  // hand the columns back preset to the bias
+#pragma unroll
+        for (int t = 0; t < CH; t += 2) {
+          const int tt = h * CH + t;
+          const float2 v = make_float2(__uint_as_float(r[t]), __uint_as_float(r[t + 1]));
+          const float2 u = __ffma2_rn(v, sw2, cb2);
+          const float2 o = __ffma2_rn(u, sa2[tt >> 1], make_float2(acc[tt], acc[tt + 1]));
+          acc[tt] = o.x;
+          acc[tt + 1] = o.y;
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[a]);
+    }
+    tmem_ld_wait();
+
+    // Stage the sums in shared memory (the stage ring is idle now: every load
+    // was consumed by an MMA that has completed), so the stores below run in a
+    // plain loop over the tokens.
+    float *stg = reinterpret_cast<float *>(smem + C::kOffStages) + c;
+#pragma unroll
+    for (int t = 0; t < MP; ++t) stg[t * 128] = acc[t];
+    // One decision for all four epilogue warps (the barriers below need all
+    // of them): a failed wait anywhere in the CTA has set the abort flag.
+    (void)live;
+    named_bar_sync(1, 128);
+    if (threadIdx.x == 384) *last_flag = *abort_flag ? 2 : 0;
+    named_bar_sync(1, 128);
+    if (*last_flag == 0) {
+      const bool ch_ok = n0 + c < Nset;
+      const int col_out = ch_ok ? __ldg(idx + n0 + c) : 0;
+      const int mt = M < MP ? M : MP;
+      if (S == 1) {
+        if (ch_ok)
+          for (int t = 0; t < mt; ++t) Y[static_cast<int64_t>(t) * N + col_out] = __float2half_rn(stg[t * 128]);
+      } else {
+        // this split's partial sums; the last of the tile's S CTAs adds them
+        float *part = ws_part + (static_cast<size_t>(split) * ntiles + tile) * (MP * 128) + c;
+        for (int t = 0; t < mt; ++t) part[t * 128] = stg[t * 128];
+        // The barrier orders the four warps' partial stores before the
+        // counter update, whose release (GPU scope, cumulative) publishes
+        // them; its acquire makes the other splits' partials visible to this
+        // thread, and the second barrier to the other three warps.
+        named_bar_sync(1, 128);
+        if (threadIdx.x == 384) *last_flag = atom_add_acq_rel_gpu(ws_cnt + tile, 1) == S - 1 ? 1 : 0;
+        named_bar_sync(1, 128);
+        if (*last_flag) {
+          const float *p0 = ws_part + static_cast<size_t>(tile) * (MP * 128) + c;
+          const size_t split_stride = static_cast<size_t>(ntiles) * (MP * 128);
+          // eight tokens at a time, so that many loads are in flight at once
+          for (int t0 = 0; t0 < mt; t0 += 8) {
+            float y[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) y[j] = t0 + j < mt ? __ldcg(p0 + (t0 + j) * 128) : 0.0f;
+            for (int sp = 1; sp < S; ++sp) {
+              const float *ps = p0 + sp * split_stride;
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                if (t0 + j < mt) y[j] += __ldcg(ps + (t0 + j) * 128);
+            }
+            if (ch_ok)
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                if (t0 + j < mt) Y[static_cast<int64_t>(t0 + j) * N + col_out] = __float2half_rn(y[j]);
+          }
+          if (threadIdx.x == 384) ws_cnt[tile] = 0;  // leave the workspace as it was found
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+constexpr int kSmWave = 148;  // SMs of a B200: split-K fills one wave of CTAs
+
+SmallMPlan plan_small_m(int64_t M, int64_t N4, int64_t N8, int64_t K) {
+  SmallMPlan p{};
+  p.mp = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+  p.nt4 = static_cast<int>((N4 + 127) / 128);
+  p.nt8 = static_cast<int>((N8 + 127) / 128);
+  p.groups = static_cast<int>(K / 128);
+  const int tiles = p.nt4 + p.nt8;
+  int S = tiles > 0 ? kSmWave / tiles : 1;
+  if (S < 1) S = 1;
+  const int s_min = (p.groups + kSmGroupsMax - 1) / kSmGroupsMax;  // groups per CTA <= kSmGroupsMax
+  if (S < s_min) S = s_min;
+  if (S > p.groups) S = p.groups;
+  p.splits = S;
+  p.part_floats = S > 1 ? static_cast<size_t>(S) * tiles * p.mp * 128 : 0;
+  p.counters = S > 1 ? static_cast<size_t>(tiles) : 0;
+  return p;
+}
+
+template <int MP>
+static cudaError_t launch_small_m_mp(const GemmArgs &a, const SmallMPlan &p, void *ws, cudaStream_t stream,
+                                     const char **msg) {
+  using C = SmallMCfg<MP>;
+  auto enc = get_encode_fn();
+  if (!enc) {
+    *msg = "cuTensorMapEncodeTiled is not available from the driver";
+    return cudaErrorNotSupported;
+  }
+  CUtensorMap tmX, tmW4, tmW8;
+  memset(&tmX, 0, sizeof(tmX));
+  memset(&tmW4, 0, sizeof(tmW4));
+  memset(&tmW8, 0, sizeof(tmW8));
+  if (!encode_2d_u8(enc, &tmX, a.A_q, a.K, a.M, 128, MP, true)) {
+    *msg = "tensor map encoding of A_q failed";
+    return cudaErrorInvalidValue;
+  }
+  if (a.N4 > 0 && !encode_2d_u8(enc, &tmW4, a.W4, a.K / 2, a.N4, 64, 128, false)) {
+    *msg = "tensor map encoding of W4 failed";
+    return cudaErrorInvalidValue;
+  }
+  if (a.N8 > 0 && !encode_2d_u8(enc, &tmW8, a.W8, a.K, a.N8, 128, 128, true)) {
+    *msg = "tensor map encoding of W8 failed";
+    return cudaErrorInvalidValue;
+  }
+  const int tiles = p.nt4 + p.nt8;
+  const int64_t grid = static_cast<int64_t>(tiles) * p.splits;
+  if (grid > 0x7FFFFFFF) {
+    *msg = "too many tiles";
+    return cudaErrorInvalidValue;
+  }
+  auto kern = gemm_small_m_kernel<MP>;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static unsigned long long configured = 0;  // one bit per device ordinal
+  if (dev < 64 && !(configured & (1ull << dev))) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
+    if (e != cudaSuccess) {
+      *msg = "cudaFuncSetAttribute(MaxDynamicSharedMemorySize) failed";
+      return e;
+    }
+    configured |= 1ull << dev;
+  }
+  float *ws_part = static_cast<float *>(ws);
+  int *ws_cnt = p.splits > 1 ? reinterpret_cast<int *>(ws_part + p.part_floats) : nullptr;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kSmThreads);
+  cfg.dynamicSmemBytes = C::kSmemAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(
+      &cfg, kern, tmX, tmW4, tmW8, a.s_a, a.z4, static_cast<const __half *>(a.s_w4), a.idx4,
+      static_cast<const __half *>(a.s_w8), a.idx8, static_cast<int>(a.M), static_cast<int>(a.K),
+      static_cast<int>(a.N4), static_cast<int>(a.N8), static_cast<int>(padded_channels(a.N4)),
+      static_cast<int>(padded_channels(a.N8)), p.nt4, tiles, p.splits, static_cast<__half *>(a.Y), ws_part, ws_cnt);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) *msg = "launch of the small-M GEMM failed";
+  return e;
+}
+
+size_t small_m_workspace_bytes(int64_t M, int64_t N4, int64_t N8, int64_t K) {
+  return plan_small_m(M, N4, N8, K).bytes();
+}
+
+cudaError_t launch_gemm_small_m(const GemmArgs &a, void *ws, size_t ws_bytes, cudaStream_t stream, const char **msg) {
+  const SmallMPlan p = plan_small_m(a.M, a.N4, a.N8, a.K);
+  if (ws_bytes < p.bytes() || (p.bytes() > 0 && !ws)) {
+    *msg = "workspace too small for this shape";
+    return cudaErrorInvalidValue;
+  }
+  if (p.mp == 16) return launch_small_m_mp<16>(a, p, ws, stream, msg);
+  if (p.mp == 32) return launch_small_m_mp<32>(a, p, ws, stream, msg);
+  return launch_small_m_mp<64>(a, p, ws, stream, msg);
+}
+
+}  // namespace mixllm

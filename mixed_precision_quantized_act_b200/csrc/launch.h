@@ -39,6 +39,13 @@ struct GemmArgs {
 // is unavailable.  *msg receives a static description on failure.
 cudaError_t launch_gemm_w4w8a8(const GemmArgs &a, cudaStream_t stream, const char **msg);
 
+// Few-token variant (M <= 64): split-K over the groups with a workspace of
+// small_m_workspace_bytes() bytes: fp32 partial sums, then one int32 counter
+// per tile (zero before the first call; every call returns them to zero).
+// Y only; no debug partials.
+cudaError_t launch_gemm_small_m(const GemmArgs &a, void *ws, size_t ws_bytes, cudaStream_t stream, const char **msg);
+size_t small_m_workspace_bytes(int64_t M, int64_t N4, int64_t N8, int64_t K);
+
 cudaError_t launch_selftest_wait_timeout(uint32_t limit_us, cudaStream_t stream);
 
 int64_t padded_channels(int64_t n);  // n rounded up to a multiple of 256

@@ -11,6 +11,7 @@
 
 #include "../../include/mixllm.h"
 #include "gemm_w4w8a8.cuh"
+#include "gemm_small_m.cuh"
 #include "launch.h"
 #include "quant.cuh"
 
@@ -59,15 +60,21 @@ mixllm_status check_device() {
   return MIXLLM_OK;
 }
 
-mixllm_status gemm_common(const int8_t *A_q, const float *s_a, int64_t M, int64_t K, const uint8_t *W4,
-                          const uint8_t *z4, const void *s_w4, const int32_t *idx4, int64_t N4, const int8_t *W8,
-                          const void *s_w8, const int32_t *idx8, int64_t N8, void *Y, int32_t *P, void *stream) {
+// Argument checks of the GEMM entry points.  Returns MIXLLM_OK with *empty
+// set when there is nothing to compute.
+mixllm_status check_gemm(const int8_t *A_q, const float *s_a, int64_t M, int64_t K, const uint8_t *W4,
+                         const uint8_t *z4, const void *s_w4, const int32_t *idx4, int64_t N4, const int8_t *W8,
+                         const void *s_w8, const int32_t *idx8, int64_t N8, void *Y, int32_t *P, bool *empty) {
+  *empty = false;
   mixllm_status st = check_k(K, MIXLLM_GROUP);
   if (st != MIXLLM_OK) return st;
   if (M < 0 || N4 < 0 || N8 < 0) return fail(MIXLLM_ERR_INVALID_ARG, "negative size");
   if (M > 0x7FFFFFFF || N4 + N8 > 0x7FFFFFF0)
     return fail(MIXLLM_ERR_INVALID_ARG, "M or N beyond the supported 2^31 range");
-  if (M == 0 || N4 + N8 == 0) return ok();
+  if (M == 0 || N4 + N8 == 0) {
+    *empty = true;
+    return MIXLLM_OK;
+  }
   if (!A_q || !s_a || !(Y || P)) return fail(MIXLLM_ERR_INVALID_ARG, "null A_q, s_a or output");
   if (!aligned(A_q, 16)) return fail(MIXLLM_ERR_INVALID_ARG, "A_q must be 16-byte aligned");
   if (!aligned(s_a, 4)) return fail(MIXLLM_ERR_INVALID_ARG, "s_a must be 4-byte aligned");
@@ -83,8 +90,16 @@ mixllm_status gemm_common(const int8_t *A_q, const float *s_a, int64_t M, int64_
     if (!aligned(W8, 16) || !aligned(s_w8, 16) || !aligned(idx8, 4))
       return fail(MIXLLM_ERR_INVALID_ARG, "8-bit set buffers must be 16-byte aligned (idx8: 4)");
   }
-  st = check_device();
+  return check_device();
+}
+
+mixllm_status gemm_common(const int8_t *A_q, const float *s_a, int64_t M, int64_t K, const uint8_t *W4,
+                          const uint8_t *z4, const void *s_w4, const int32_t *idx4, int64_t N4, const int8_t *W8,
+                          const void *s_w8, const int32_t *idx8, int64_t N8, void *Y, int32_t *P, void *stream) {
+  bool empty = false;
+  mixllm_status st = check_gemm(A_q, s_a, M, K, W4, z4, s_w4, idx4, N4, W8, s_w8, idx8, N8, Y, P, &empty);
   if (st != MIXLLM_OK) return st;
+  if (empty) return ok();
   mixllm::GemmArgs a{A_q, s_a, M, K, W4, z4, s_w4, idx4, N4, W8, s_w8, idx8, N8, Y, P};
   const char *msg = "";
   cudaError_t e = mixllm::launch_gemm_w4w8a8(a, static_cast<cudaStream_t>(stream), &msg);
@@ -197,6 +212,42 @@ mixllm_status mixllm_gemm_debug_partials(const int8_t *A_q, const float *s_a, in
                                          const int32_t *idx8, int64_t N8, int32_t *P, void *stream) {
   if (!P && M > 0 && N4 + N8 > 0) return fail(MIXLLM_ERR_INVALID_ARG, "null P");
   return gemm_common(A_q, s_a, M, K, W4, z4, s_w4_f16, idx4, N4, W8, s_w8_f16, idx8, N8, nullptr, P, stream);
+}
+
+mixllm_status mixllm_small_m_workspace_bytes(int64_t M, int64_t K, int64_t N4, int64_t N8, size_t *bytes) {
+  mixllm_status st = check_k(K, MIXLLM_GROUP);
+  if (st != MIXLLM_OK) return st;
+  if (!bytes) return fail(MIXLLM_ERR_INVALID_ARG, "null bytes");
+  if (M < 1 || M > 64) return fail(MIXLLM_ERR_INVALID_ARG, "the small-M path takes 1 <= M <= 64");
+  if (N4 < 0 || N8 < 0 || N4 + N8 > 0x7FFFFFF0) return fail(MIXLLM_ERR_INVALID_ARG, "bad N4 / N8");
+  *bytes = mixllm::small_m_workspace_bytes(M, N4, N8, K);
+  return ok();
+}
+
+mixllm_status mixllm_gemm_w4w8a8_small_m(const int8_t *A_q, const float *s_a, int64_t M, int64_t K,
+                                         const uint8_t *W4, const uint8_t *z4, const void *s_w4_f16,
+                                         const int32_t *idx4, int64_t N4, const int8_t *W8, const void *s_w8_f16,
+                                         const int32_t *idx8, int64_t N8, void *Y_f16, void *workspace,
+                                         size_t workspace_bytes, void *stream) {
+  if (M > 64) return fail(MIXLLM_ERR_INVALID_ARG, "the small-M path takes M <= 64 (M = %lld)", static_cast<long long>(M));
+  if (!Y_f16 && M > 0 && N4 + N8 > 0) return fail(MIXLLM_ERR_INVALID_ARG, "null Y");
+  bool empty = false;
+  mixllm_status st =
+      check_gemm(A_q, s_a, M, K, W4, z4, s_w4_f16, idx4, N4, W8, s_w8_f16, idx8, N8, Y_f16, nullptr, &empty);
+  if (st != MIXLLM_OK) return st;
+  if (empty) return ok();
+  const size_t need = mixllm::small_m_workspace_bytes(M, N4, N8, K);
+  if (workspace_bytes < need)
+    return fail(MIXLLM_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu this shape needs",
+                workspace_bytes, need);
+  if (need > 0 && (!workspace || !aligned(workspace, 16)))
+    return fail(MIXLLM_ERR_INVALID_ARG, "workspace must be a 16-byte aligned device buffer");
+  mixllm::GemmArgs a{A_q, s_a, M, K, W4, z4, s_w4_f16, idx4, N4, W8, s_w8_f16, idx8, N8, Y_f16, nullptr};
+  const char *msg = "";
+  cudaError_t e = mixllm::launch_gemm_small_m(a, workspace, workspace_bytes, static_cast<cudaStream_t>(stream), &msg);
+  if (e == cudaErrorNotSupported) return fail(MIXLLM_ERR_UNSUPPORTED, "%s", msg);
+  if (e != cudaSuccess) return fail(MIXLLM_ERR_CUDA, "%s: %s", msg, cudaGetErrorString(e));
+  return ok();
 }
 
 mixllm_status mixllm_sync_status(void *stream) {

@@ -115,3 +115,30 @@ def test_binding_raises_without_cuda_tensors(L):
     with pytest.raises(ValueError):
         _lib.quantize_act_into(torch.zeros(2, 128, dtype=torch.float16), torch.zeros(2, 128, dtype=torch.int8),
                                torch.zeros(2, 1), None)
+
+
+def test_small_m_workspace_plan(L):
+    """Workspace of the few-token path: S splits x tiles x (token tile x 128)
+    fp32 partials + one int32 counter per 128-channel tile; S fills one wave
+    of 148 CTAs and caps a CTA at 32 groups; no workspace without a split."""
+    def ws(M, K, N4, N8):
+        out = ctypes.c_size_t(0)
+        st = L.mixllm_small_m_workspace_bytes(M, K, N4, N8, ctypes.byref(out))
+        return st, out.value
+
+    # q_proj p10 at M=1: 29 + 4 tiles, S = 148 // 33 = 4, token tile 16
+    assert ws(1, 4096, 3686, 410) == (_lib.OK, 4 * 33 * 16 * 128 * 4 + 33 * 4)
+    # token tiles 32 and 64
+    assert ws(17, 4096, 3686, 410) == (_lib.OK, 4 * 33 * 32 * 128 * 4 + 33 * 4)
+    assert ws(64, 4096, 3686, 410) == (_lib.OK, 4 * 33 * 64 * 128 * 4 + 33 * 4)
+    # 225 tiles: more than one wave, no split, no workspace
+    assert ws(16, 4096, 27238, 1434) == (_lib.OK, 0)
+    # K = 28672 (224 groups), 58 + 7 tiles: S = max(148 // 65, 224 / 32) = 7
+    assert ws(16, 28672, 7373, 819) == (_lib.OK, 7 * 65 * 16 * 128 * 4 + 65 * 4)
+    # one group: nothing to split
+    assert ws(3, 128, 300, 84) == (_lib.OK, 0)
+    assert ws(65, 4096, 100, 10)[0] == _lib.ERR_INVALID_ARG
+    assert ws(0, 4096, 100, 10)[0] == _lib.ERR_INVALID_ARG
+    assert ws(8, 100, 100, 10)[0] == _lib.ERR_UNSUPPORTED
+    null = L.mixllm_small_m_workspace_bytes(8, 4096, 100, 10, None)
+    assert null == _lib.ERR_INVALID_ARG

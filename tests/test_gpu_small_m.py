@@ -1,0 +1,136 @@
+"""Parity of the few-token GEMM (mixllm_gemm_w4w8a8_small_m, M <= 64) with the
+CPU oracle.  GPU only.
+
+Y within |dY| <= 2^-9 * |y_oracle| + 1e-3 * rms(y_oracle), per element; the
+split-K reduction adds the splits in a fixed order, so repeated calls are
+bit-identical, and every call returns the workspace's tile counters to zero.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle  # noqa: E402
+import mixed_precision_quantized_act_b200 as mx  # noqa: E402
+from mixed_precision_quantized_act_b200 import _lib  # noqa: E402
+from mixed_precision_quantized_act_b200 import workloads as wl  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+REL, ABS_RMS = 2.0 ** -9, 1e-3
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    mx.load()
+    return torch.device("cuda:0")
+
+
+def assert_y_close(Y, Y_ref, what=""):
+    Y = np.asarray(Y, np.float64)
+    Y_ref = np.asarray(Y_ref, np.float64)
+    assert Y.shape == Y_ref.shape
+    rms = float(np.sqrt(np.mean(Y_ref ** 2))) if Y_ref.size else 0.0
+    err = np.abs(Y - Y_ref)
+    bad = err > REL * np.abs(Y_ref) + ABS_RMS * rms
+    assert not bad.any(), (f"{what}: {int(bad.sum())} of {Y.size} outside tolerance, "
+                           f"max excess {float(np.max(err - REL * np.abs(Y_ref) - ABS_RMS * rms)):.3g}")
+
+
+def _layer(name, M, N, K, n8, outliers=4):
+    return wl.Linear(name, M, N, K, ((0, N, n8),), outliers)
+
+
+# token tiles 16 / 32 / 64, ragged N, one set empty, one 8-bit channel,
+# split counts from 1 (wide N) to the group cap (long K)
+CASES = [
+    wl.Q_PROJ_P10.with_m(1),
+    wl.Q_PROJ_P10.with_m(16),
+    wl.Q_PROJ_P10.with_m(64),
+    _layer("sm_m5_ragged", 5, 300, 384, 37),
+    _layer("sm_m17", 17, 1000, 1024, 101),
+    _layer("sm_m33", 33, 640, 1024, 64),
+    _layer("sm_m7_p0", 7, 512, 512, 0),
+    _layer("sm_m7_p100", 7, 512, 512, 512),
+    _layer("sm_m2_one_8bit", 2, 260, 256, 1),
+    _layer("sm_m3_k128", 3, 384, 128, 40),
+]
+
+
+def counters_zero(ws, p, M, K):
+    need = mx.small_m_workspace_bytes(M, K, p.N4, p.N8)
+    tiles = -(-p.N4 // 128) + -(-p.N8 // 128)
+    return need == 0 or not ws[need - 4 * tiles: need].any()
+
+
+def _run(dev, layer, seed):
+    X, W, is8 = wl.make_x(layer, seed), wl.make_w(layer, seed), wl.make_bitmap(layer, seed)
+    A_q, s_a = mx.quantize_act(torch.from_numpy(X).to(dev))
+    p = mx.pack_weights(torch.from_numpy(W).to(dev), torch.from_numpy(is8).to(dev))
+    ws = mx.small_m_workspace(layer.M, p, dev)
+    Y = mx.gemm_w4w8a8_small_m(A_q, s_a, p, ws)
+    mx.sync_status()
+    return X, W, is8, A_q, s_a, p, ws, Y
+
+
+@pytest.mark.parametrize("layer", CASES, ids=lambda l: l.name)
+def test_small_m_matches_oracle(dev, layer):
+    X, W, is8, A_q, s_a, p, ws, Y = _run(dev, layer, 11)
+    A_ref, s_ref = oracle.quantize_act(X)
+    Y_ref = oracle.gemm_w4w8a8(A_ref, s_ref, oracle.Quantized(W, is8))
+    assert_y_close(Y.cpu().numpy(), Y_ref, layer.name)
+    assert counters_zero(ws, p, layer.M, layer.K), "the tile counters must be back at zero"
+
+
+@pytest.mark.parametrize("layer", [wl.Q_PROJ_P10.with_m(16), _layer("sm_m33", 33, 640, 1024, 64)],
+                         ids=lambda l: l.name)
+def test_small_m_deterministic_and_close_to_tiled(dev, layer):
+    X, W, is8, A_q, s_a, p, ws, Y1 = _run(dev, layer, 12)
+    Y2 = torch.empty_like(Y1)
+    for _ in range(5):
+        mx.gemm_w4w8a8_small_m_into(A_q, s_a, p, Y2, ws)
+    Yt = mx.gemm_w4w8a8(A_q, s_a, p)
+    mx.sync_status()
+    assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
+    assert counters_zero(ws, p, layer.M, layer.K)
+    # the tiled kernel computes the same layer with another fp32 order
+    A_ref, s_ref = oracle.quantize_act(X)
+    Y_ref = oracle.gemm_w4w8a8(A_ref, s_ref, oracle.Quantized(W, is8))
+    assert_y_close(Yt.cpu().numpy(), Y_ref, layer.name + " tiled")
+    assert_y_close(Y1.cpu().numpy(), Y_ref, layer.name + " small-M")
+
+
+@pytest.mark.parametrize("layer", [wl.LLAMA8B_LAYER[2].with_m(8), wl.LLAMA70B[3].with_m(4)],
+                         ids=lambda l: l.name)
+def test_small_m_wide_and_long_layers(dev, layer):
+    """8B gate_up (N = 28672: more tiles than SMs, no split) and 70B down
+    (K = 28672: the split count set by the per-CTA group cap); a random
+    subset of the columns against the oracle."""
+    X, W, is8, A_q, s_a, p, ws, Y = _run(dev, layer, 13)
+    cols = np.sort(np.random.default_rng(3).choice(layer.N, 2048, replace=False))
+    A_ref, s_ref = oracle.quantize_act(X)
+    Y_ref = oracle.gemm_w4w8a8(A_ref, s_ref, oracle.Quantized(W[cols], is8[cols]))
+    assert_y_close(Y.cpu().numpy()[:, cols], Y_ref, layer.name)
+    assert torch.isfinite(Y).all()
+    assert counters_zero(ws, p, layer.M, layer.K)
+
+
+def test_small_m_linear_dispatch_and_validation(dev):
+    layer = _layer("sm_m5_ragged", 5, 300, 384, 37)
+    X, W, is8, A_q, s_a, p, ws, Y = _run(dev, layer, 14)
+    Y_lin = mx.linear(torch.from_numpy(X).to(dev), p, workspace=ws)
+    mx.sync_status()
+    assert torch.equal(Y.view(torch.int16), Y_lin.view(torch.int16))
+    need = mx.small_m_workspace_bytes(layer.M, layer.K, p.N4, p.N8)
+    assert need > 0
+    with pytest.raises(_lib.MixLLMError) as ei:
+        mx.gemm_w4w8a8_small_m_into(A_q, s_a, p, torch.empty_like(Y), ws[: need - 4])
+    assert ei.value.status == _lib.ERR_INVALID_ARG
+    X65 = torch.from_numpy(wl.make_x(layer.with_m(65), 1)).to(dev)
+    A65, s65 = mx.quantize_act(X65)
+    with pytest.raises(_lib.MixLLMError) as ei:
+        mx.gemm_w4w8a8_small_m(A65, s65, p, ws)
+    assert ei.value.status == _lib.ERR_INVALID_ARG
+    mx.sync_status()
