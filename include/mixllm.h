@@ -221,6 +221,29 @@ MIXLLM_API mixllm_status mixllm_gemm_w4w8a8_small_m(const int8_t *A_q, const flo
                                          void *stream);
 
 /*
+ * mixllm_gemm_w4w8a8_small_m without a workspace argument and without any
+ * allocation: the split partial sums and tile counters live in a fixed 8 MiB
+ * scratch array in the library's static device memory (one per device,
+ * created with the module).  An engineering variant for callers that cannot
+ * hand over device memory; the paper has no counterpart.  Same arguments,
+ * result and rounding as mixllm_gemm_w4w8a8_small_m otherwise.
+ *   * The tile counters are cleared on `stream` before every launch (an
+ *     asynchronous memset of the scratch, no allocation).
+ *   * Calls that overlap in time on one device share the scratch and race:
+ *     issue them to one stream, or order them with events.
+ *   * Returns MIXLLM_ERR_UNSUPPORTED when the shape needs more scratch than
+ *     the array holds (see mixllm_small_m_workspace_bytes), and
+ *     MIXLLM_ERR_INVALID_ARG for M > 64.
+ * Asynchronous on `stream`.
+ */
+MIXLLM_API mixllm_status mixllm_gemm_w4w8a8_small_m_noalloc(const int8_t *A_q, const float *s_a, int64_t M,
+                                                 int64_t K, const uint8_t *W4, const uint8_t *z4,
+                                                 const void *s_w4_f16, const int32_t *idx4, int64_t N4,
+                                                 const int8_t *W8, const void *s_w8_f16,
+                                                 const int32_t *idx8, int64_t N8,
+                                                 void *Y_f16, void *stream);
+
+/*
  * Waits for `stream`, then reads and clears the device status word of the
  * current device.  Returns MIXLLM_ERR_TIMEOUT if a kernel of this library
  * gave up a wait since the last call, MIXLLM_ERR_CUDA if the stream reports

@@ -14,6 +14,7 @@ from ._lib import (  # noqa: F401
     gemm_w4w8a8,
     gemm_w4w8a8_into,
     gemm_w4w8a8_small_m,
+    gemm_w4w8a8_small_m_noalloc_into,
     gemm_w4w8a8_small_m_into,
     linear,
     load,

@@ -36,6 +36,8 @@ SIGNATURES = {
     "mixllm_small_m_workspace_bytes": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(ctypes.c_size_t)]),
     "mixllm_gemm_w4w8a8_small_m": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64,
                                                   _vp, _vp, _vp, _i64, _vp, _vp, ctypes.c_size_t, _vp]),
+    "mixllm_gemm_w4w8a8_small_m_noalloc": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64,
+                                                          _vp, _vp, _vp, _i64, _vp, _vp]),
     "mixllm_sync_status": (ctypes.c_int, [_vp]),
     "mixllm_selftest_wait_timeout": (ctypes.c_int, [_u32, _vp]),
 }
@@ -240,6 +242,18 @@ def gemm_w4w8a8_small_m(A_q, s_a, p: PackedLinear, workspace: torch.Tensor = Non
     Y = torch.empty((M, p.N), dtype=torch.float16, device=A_q.device)
     gemm_w4w8a8_small_m_into(A_q, s_a, p, Y, workspace, stream)
     return Y
+
+
+def gemm_w4w8a8_small_m_noalloc_into(A_q, s_a, p: PackedLinear, Y, stream=None):
+    """The few-token GEMM on the library's static device scratch (no workspace,
+    no allocation); calls must not overlap in time on one device."""
+    _need_cuda(A_q, s_a, Y)
+    M, K = A_q.shape
+    assert K == p.K and Y.shape == (M, p.N) and Y.dtype == torch.float16 and Y.is_contiguous()
+    _check(load().mixllm_gemm_w4w8a8_small_m_noalloc(_ptr(A_q), _ptr(s_a), M, K, _ptr(p.W4), _ptr(p.z4),
+                                                     _ptr(p.s_w4), _ptr(p.idx4), p.N4, _ptr(p.W8), _ptr(p.s_w8),
+                                                     _ptr(p.idx8), p.N8, _ptr(Y), _stream(stream)),
+           "mixllm_gemm_w4w8a8_small_m_noalloc")
 
 
 def linear(X: torch.Tensor, p: PackedLinear, stream=None, workspace: torch.Tensor = None) -> torch.Tensor:

@@ -545,4 +545,43 @@ cudaError_t launch_gemm_small_m(const GemmArgs &a, void *ws, size_t ws_bytes, cu
   return launch_small_m_mp<64>(a, p, ws, stream, msg);
 }
 
+// ---------------------------------------------------------------------------
+// The same path with no caller workspace and no allocation: a fixed scratch
+// array in the module's static device memory (one copy per device, created
+// when the module loads and zero-initialized).  Calls that run at the same
+// time on one device (different streams or host threads) would share it, so
+// they must be ordered, e.g. issued to one stream.
+// ---------------------------------------------------------------------------
+
+constexpr size_t kSmallMScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) unsigned char g_small_m_scratch[kSmallMScratchBytes];
+
+size_t small_m_scratch_capacity() { return kSmallMScratchBytes; }
+
+cudaError_t launch_gemm_small_m_noalloc(const GemmArgs &a, cudaStream_t stream, const char **msg) {
+  const SmallMPlan p = plan_small_m(a.M, a.N4, a.N8, a.K);
+  if (p.bytes() > kSmallMScratchBytes) {
+    *msg = "shape needs more scratch than the static buffer holds";
+    return cudaErrorInvalidValue;
+  }
+  void *ws = nullptr;
+  if (p.bytes() > 0) {
+    // the device's own copy of the array
+    cudaError_t e = cudaGetSymbolAddress(&ws, g_small_m_scratch);
+    if (e != cudaSuccess) {
+      *msg = "cudaGetSymbolAddress of the static scratch failed";
+      return e;
+    }
+    // The tile counters must start at zero.  Every call returns them to zero,
+    // but one that gave up (a timeout) may not have: clear them each time.
+    e = cudaMemsetAsync(static_cast<unsigned char *>(ws) + p.part_floats * sizeof(float), 0,
+                        p.counters * sizeof(int), stream);
+    if (e != cudaSuccess) {
+      *msg = "clearing the tile counters failed";
+      return e;
+    }
+  }
+  return launch_gemm_small_m(a, ws, kSmallMScratchBytes, stream, msg);
+}
+
 }  // namespace mixllm

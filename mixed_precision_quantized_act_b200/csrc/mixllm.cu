@@ -250,6 +250,30 @@ mixllm_status mixllm_gemm_w4w8a8_small_m(const int8_t *A_q, const float *s_a, in
   return ok();
 }
 
+mixllm_status mixllm_gemm_w4w8a8_small_m_noalloc(const int8_t *A_q, const float *s_a, int64_t M, int64_t K,
+                                                 const uint8_t *W4, const uint8_t *z4, const void *s_w4_f16,
+                                                 const int32_t *idx4, int64_t N4, const int8_t *W8,
+                                                 const void *s_w8_f16, const int32_t *idx8, int64_t N8, void *Y_f16,
+                                                 void *stream) {
+  if (M > 64) return fail(MIXLLM_ERR_INVALID_ARG, "the small-M path takes M <= 64 (M = %lld)", static_cast<long long>(M));
+  if (!Y_f16 && M > 0 && N4 + N8 > 0) return fail(MIXLLM_ERR_INVALID_ARG, "null Y");
+  bool empty = false;
+  mixllm_status st =
+      check_gemm(A_q, s_a, M, K, W4, z4, s_w4_f16, idx4, N4, W8, s_w8_f16, idx8, N8, Y_f16, nullptr, &empty);
+  if (st != MIXLLM_OK) return st;
+  if (empty) return ok();
+  const size_t need = mixllm::small_m_workspace_bytes(M, N4, N8, K);
+  if (need > mixllm::small_m_scratch_capacity())
+    return fail(MIXLLM_ERR_UNSUPPORTED, "this shape needs %zu bytes of scratch; the static buffer holds %zu", need,
+                mixllm::small_m_scratch_capacity());
+  mixllm::GemmArgs a{A_q, s_a, M, K, W4, z4, s_w4_f16, idx4, N4, W8, s_w8_f16, idx8, N8, Y_f16, nullptr};
+  const char *msg = "";
+  cudaError_t e = mixllm::launch_gemm_small_m_noalloc(a, static_cast<cudaStream_t>(stream), &msg);
+  if (e == cudaErrorNotSupported) return fail(MIXLLM_ERR_UNSUPPORTED, "%s", msg);
+  if (e != cudaSuccess) return fail(MIXLLM_ERR_CUDA, "%s: %s", msg, cudaGetErrorString(e));
+  return ok();
+}
+
 mixllm_status mixllm_sync_status(void *stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
