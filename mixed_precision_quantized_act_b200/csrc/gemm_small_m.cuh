@@ -21,7 +21,8 @@
 //     counter is reset by that CTA, so the counters are zero between calls.
 // Roles (512 threads, registers rebalanced per warpgroup with setmaxnreg):
 // warp 0 TMA producer (weight tile, zero points and the token tile of each
-// group into a ring of stages), warp 1 MMA issuer (one commit per group),
+// group into a ring of stages), warps 1 and 3 MMA issuers (alternate groups,
+// one commit per group),
 // warp 2 scale tables (this CTA's groups, loaded once), warps 4-11 4-bit
 // unpack into the swizzled int8 operand (with few tokens it is the longest
 // per-group step), warps 12-15 epilogue (one TMEM lane quadrant each).  Every
@@ -52,9 +53,12 @@ struct SmallMCfg {
   // The ring holds as many stages as fit (all of a CTA's groups when they
   // fit, so one round of loads covers the whole K range): a stage is the
   // weight tile (int8 16 KB, or packed 4-bit 8 KB) followed by the token tile.
-  static constexpr int kRingBytes = 160 * 1024;
+  static constexpr int kRingBytes = 128 * 1024;
   static constexpr int kMaxStages = 16;
-  static constexpr int kTBufs = 2;
+  // Unpacked 4-bit tiles: buffer i % kTBufs is free again only when the MMAs
+  // of group i - kTBufs have completed (~800 cycles after their commit), so
+  // the unpack needs several in flight.
+  static constexpr int kTBufs = 4;
   static constexpr int kAccBufs = 4;
   static constexpr int kDone = kMaxStages;              // >= every ring released through it
   static_assert(kDone >= kTBufs && kDone >= kAccBufs, "done ring");
@@ -69,7 +73,11 @@ struct SmallMCfg {
   static constexpr int kOffSw = kOffZ + kMaxStages * 64;               // fp16 s_w [groups][128]
   static constexpr int kOffSa = kOffSw + kSmGroupsMax * 128 * 4;       // fp32 s_a [groups][MP]
   static constexpr int kOffBar = kOffSa + kSmGroupsMax * MP * 4;
-  static constexpr int kNumBars = kMaxStages + kDone + kTBufs + kAccBufs + 2;  // + table ready, drain
+  static constexpr int kNumBars = kMaxStages + kDone + kTBufs + kAccBufs + 3;  // + table ready, 2 drains
+  // Two threads issue the MMAs of alternate groups; a ring they wait on must
+  // give each slot to one of them (even slot counts), or a parity wait could
+  // see a phase meant for the other one.
+  static_assert(kTBufs % 2 == 0 && kAccBufs % 2 == 0 && kMaxStages % 2 == 0, "rings the issuers wait on");
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;
@@ -146,7 +154,7 @@ __global__ void __launch_bounds__(kSmThreads, 1)
   uint64_t *tfull = done + C::kDone;          // unpack -> MMA         (per unpacked buffer)
   uint64_t *accempty = tfull + C::kTBufs;     // epilogue -> MMA       (per accumulator)
   uint64_t *tabready = accempty + C::kAccBufs;  // scale tables loaded
-  uint64_t *drain = tabready + 1;             // MMA issuer's final commit
+  uint64_t *drain = tabready + 1;             // [2]: each MMA issuer's final commit
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kOffMisc + 4);
   volatile int *last_flag = reinterpret_cast<volatile int *>(smem + C::kOffMisc + 8);
@@ -170,7 +178,8 @@ __global__ void __launch_bounds__(kSmThreads, 1)
   // stage = weight tile (packed 4-bit or int8) + token tile; as many as fit
   const int wbytes = is4 ? C::kW4Bytes : C::kWBytes;
   const int stage_sz = wbytes + C::kXBytes;  // a multiple of 1024
-  const int nst = C::kRingBytes / stage_sz < C::kMaxStages ? C::kRingBytes / stage_sz : C::kMaxStages;
+  int nst = C::kRingBytes / stage_sz < C::kMaxStages ? C::kRingBytes / stage_sz : C::kMaxStages;
+  nst &= ~1;  // even: every stage belongs to one MMA issuer
   auto stage_w = [&](int s) { return smem + C::kOffStages + s * stage_sz; };
   auto stage_x = [&](int s) { return smem + C::kOffStages + s * stage_sz + wbytes; };
   auto tbuf = [&](int b) { return smem + C::kOffTBuf + b * C::kWBytes; };
@@ -196,7 +205,8 @@ __global__ void __launch_bounds__(kSmThreads, 1)
     for (int b = 0; b < C::kTBufs; ++b) mbar_init(&tfull[b], kSmUnpackWarps);
     for (int a = 0; a < C::kAccBufs; ++a) mbar_init(&accempty[a], 4);
     mbar_init(tabready, 1);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     *last_flag = 0;
     fence_mbar_init();
@@ -229,11 +239,14 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       for (int i = (issued > nst ? issued - nst : 0); i < issued; ++i)
         (void)mbar_wait_drain(&full[i % nst], (i / nst) & 1, 1ll << 26);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------------------------------------ MMA issuers
+    // warp 1 the even local groups, warp 3 the odd ones: one thread pays for
+    // every tcgen05.mma and commit it issues, two keep the tensor pipe fed.
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_i8(128, MP);
-      for (int i = 0; i < ng; ++i) {
+      const int who = warp == 1 ? 0 : 1;
+      for (int i = who; i < ng; i += 2) {
         const int s = i % nst, b = i % C::kTBufs, a = i % C::kAccBufs;
         if (!mbar_wait(&full[s], (i / nst) & 1, abort_flag)) break;
         if (is4 && !mbar_wait(&tfull[b], (i / C::kTBufs) & 1, abort_flag)) break;
@@ -248,8 +261,8 @@ __global__ void __launch_bounds__(kSmThreads, 1)
           mma_i8(d, sw128_kmajor_desc(a_addr + 32 * kk), sw128_kmajor_desc(b_addr + 32 * kk), idesc, 1u);
         mma_commit(&done[i % C::kDone]);
       }
-      mma_commit(drain);
-      (void)mbar_wait_drain(drain, 0, 1ll << 28);
+      mma_commit(&drain[who]);
+      (void)mbar_wait_drain(&drain[who], 0, 1ll << 28);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ scale tables

@@ -53,6 +53,7 @@
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 #include <cstdint>
+#include <mutex>
 
 #include "launch.h"
 #include "ptx_sm100.cuh"
@@ -612,8 +613,9 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-static bool encode_2d_u8(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *map, const void *base, uint64_t inner,
-                         uint64_t outer, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+static bool encode_2d_u8_uncached(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *map, const void *base,
+                                  uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+                                  bool swizzle128) {
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {inner};
   const cuuint32_t box[2] = {box_inner, box_outer};
@@ -623,6 +625,35 @@ static bool encode_2d_u8(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *map
                          swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// The descriptor is a pure function of its arguments, so encoded ones are
+// kept (a small round-robin table) and reused: a layer called again with the
+// same buffers skips the host-side encoding.
+static bool encode_2d_u8(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *map, const void *base, uint64_t inner,
+                         uint64_t outer, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  struct Entry {
+    const void *base;
+    uint64_t inner, outer;
+    uint32_t box_inner, box_outer;
+    bool swizzle;
+    bool valid;
+    CUtensorMap map;
+  };
+  static Entry table[64];
+  static int next = 0;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry &e : table)
+    if (e.valid && e.base == base && e.inner == inner && e.outer == outer && e.box_inner == box_inner &&
+        e.box_outer == box_outer && e.swizzle == swizzle128) {
+      *map = e.map;
+      return true;
+    }
+  if (!encode_2d_u8_uncached(enc, map, base, inner, outer, box_inner, box_outer, swizzle128)) return false;
+  table[next] = Entry{base, inner, outer, box_inner, box_outer, swizzle128, true, *map};
+  next = (next + 1) % 64;
+  return true;
 }
 
 template <int BN, bool kDebugP>
