@@ -69,7 +69,8 @@ MIXLLM_API const char *mixllm_last_error(void);
 /*
  * Byte sizes of the seven packed-weight buffers for N output channels, of
  * which N8 are 8-bit, and inner size K:
- *   out_bytes[0] W4    uint8 [N4, K/2]   4-bit codes, two per byte
+ *   out_bytes[0] W4    uint8 [T4, G, 128, 64]  4-bit codes, two per byte,
+ *                      T4 = ceil(N4/128) tiles of 128 rows
  *   out_bytes[1] z4    uint8 [G, N4p/2]  4-bit zero points, two per byte
  *   out_bytes[2] s_w4  fp16  [G, N4p]    4-bit set scales
  *   out_bytes[3] idx4  int32 [N4]        output column of each 4-bit row
@@ -113,9 +114,11 @@ MIXLLM_API mixllm_status mixllm_quantize_act(const void *X_f16, int64_t M, int64
  *   8-bit, per (channel, group): s = fp16(min(amax/127, 65504)),
  *     q = clamp(rne(w/s), -127, 127); s == 0 gives q = 0.
  * Packed layout (the buffers of mixllm_packed_sizes):
- *   W4: row r holds channel idx4[r]; in each run of 32 consecutive k, byte
- *       i (0..15) holds code k = 32c+i in its low nibble and k = 32c+16+i
- *       in its high nibble.
+ *   W4: row r (channel idx4[r]) of group g is the 64 bytes at
+ *       ((r/128)*G + g)*8192 + (r%128)*64, so that each 128-channel tile's
+ *       group is one contiguous 8 KiB block; in each run c of 32 consecutive
+ *       k, byte 16c+i (i = 0..15) holds code k = 32c+i in its low nibble and
+ *       k = 32c+16+i in its high nibble; rows past N4 are 0.
  *   z4: zero point of row r, group g in byte g*N4p/2 + r/2, low nibble for
  *       even r, high for odd r; padding rows are 0.
  *   s_w4 / s_w8: scale of row r, group g at g*Np + r; padding rows are 0.

@@ -131,7 +131,7 @@ class PackedLinear:
     K: int
     N4: int
     N8: int
-    W4: torch.Tensor    # uint8 [N4, K/2]
+    W4: torch.Tensor    # uint8 [ceil(N4/128), K/128, 128, 64]: one block per (128-channel tile, group)
     z4: torch.Tensor    # uint8 [G, N4p/2]
     s_w4: torch.Tensor  # fp16 [G, N4p]
     idx4: torch.Tensor  # int32 [N4]
@@ -153,7 +153,7 @@ def empty_packed(N: int, K: int, N8: int, device) -> PackedLinear:
     u8, i8, f16, i32 = torch.uint8, torch.int8, torch.float16, torch.int32
     return PackedLinear(
         N, K, N4, N8,
-        torch.empty((N4, K // 2), dtype=u8, device=device),
+        torch.empty(((N4 + 127) // 128, G, 128, 64), dtype=u8, device=device),
         torch.empty((G, padded(N4) // 2), dtype=u8, device=device),
         torch.empty((G, padded(N4)), dtype=f16, device=device),
         torch.empty((N4,), dtype=i32, device=device),

@@ -138,7 +138,7 @@ __device__ __forceinline__ void sm_reg_fence(uint32_t (&r)[MP]) {
 
 template <int MP>
 __global__ void __launch_bounds__(kSmThreads, 1)
-    gemm_small_m_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW4,
+    gemm_small_m_kernel(const __grid_constant__ CUtensorMap tmX, const uint8_t *__restrict__ W4,
                         const __grid_constant__ CUtensorMap tmW8, const float *__restrict__ s_a,
                         const uint8_t *__restrict__ z4, const __half *__restrict__ s_w4,
                         const int32_t *__restrict__ idx4, const __half *__restrict__ s_w8,
@@ -190,7 +190,8 @@ __global__ void __launch_bounds__(kSmThreads, 1)
     mbar_arrive_expect_tx(&full[s], stage_bytes);
     tma_load_2d(stage_x(s), &tmX, &full[s], g * 128, 0);
     if (is4) {
-      tma_load_2d(stage_w(s), &tmW4, &full[s], g * 64, n0);
+      // the tile's packed group is one contiguous 8 KB block: one bulk copy
+      bulk_load(stage_w(s), W4 + (static_cast<int64_t>(n0 >> 7) * G + g) * C::kW4Bytes, C::kW4Bytes, &full[s]);
       bulk_load(zmeta(s), z4 + static_cast<int64_t>(g) * (N4p >> 1) + (n0 >> 1), 64, &full[s]);
     } else {
       tma_load_2d(stage_w(s), &tmW8, &full[s], g * 128, n0);
@@ -199,7 +200,7 @@ __global__ void __launch_bounds__(kSmThreads, 1)
 
   if (threadIdx.x == 0) {
     prefetch_tmap(&tmX);
-    if (is4) prefetch_tmap(&tmW4); else prefetch_tmap(&tmW8);
+    if (!is4) prefetch_tmap(&tmW8);
     for (int s = 0; s < C::kMaxStages; ++s) mbar_init(&full[s], 1);
     for (int i = 0; i < C::kDone; ++i) mbar_init(&done[i], 1);
     for (int b = 0; b < C::kTBufs; ++b) mbar_init(&tfull[b], kSmUnpackWarps);
@@ -487,16 +488,11 @@ static cudaError_t launch_small_m_mp(const GemmArgs &a, const SmallMPlan &p, voi
     *msg = "cuTensorMapEncodeTiled is not available from the driver";
     return cudaErrorNotSupported;
   }
-  CUtensorMap tmX, tmW4, tmW8;
+  CUtensorMap tmX, tmW8;
   memset(&tmX, 0, sizeof(tmX));
-  memset(&tmW4, 0, sizeof(tmW4));
   memset(&tmW8, 0, sizeof(tmW8));
   if (!encode_2d_u8(enc, &tmX, a.A_q, a.K, a.M, 128, MP, true)) {
     *msg = "tensor map encoding of A_q failed";
-    return cudaErrorInvalidValue;
-  }
-  if (a.N4 > 0 && !encode_2d_u8(enc, &tmW4, a.W4, a.K / 2, a.N4, 64, 128, false)) {
-    *msg = "tensor map encoding of W4 failed";
     return cudaErrorInvalidValue;
   }
   if (a.N8 > 0 && !encode_2d_u8(enc, &tmW8, a.W8, a.K, a.N8, 128, 128, true)) {
@@ -534,7 +530,7 @@ static cudaError_t launch_small_m_mp(const GemmArgs &a, const SmallMPlan &p, voi
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(
-      &cfg, kern, tmX, tmW4, tmW8, a.s_a, a.z4, static_cast<const __half *>(a.s_w4), a.idx4,
+      &cfg, kern, tmX, a.W4, tmW8, a.s_a, a.z4, static_cast<const __half *>(a.s_w4), a.idx4,
       static_cast<const __half *>(a.s_w8), a.idx8, static_cast<int>(a.M), static_cast<int>(a.K),
       static_cast<int>(a.N4), static_cast<int>(a.N8), static_cast<int>(padded_channels(a.N4)),
       static_cast<int>(padded_channels(a.N8)), p.nt4, tiles, p.splits, static_cast<__half *>(a.Y), ws_part, ws_cnt);

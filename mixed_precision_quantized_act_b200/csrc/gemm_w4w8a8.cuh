@@ -14,9 +14,9 @@
 //   warp 0      TMA producer: the A_q tile [128 x 128] (128-byte swizzle) of
 //               every group -- together with the int8 weight tile [BN x 128]
 //               on 8-bit tiles -- into a ring of stages, and on 4-bit tiles
-//               the packed uint4 weight tile [BN x 64 B] and the group's zero
-//               points into a ring of their own; L2 prefetch of the boxes a few
-//               groups further on.
+//               the packed uint4 weight tile [BN x 64 B] (one contiguous 8 KB
+//               block per tile and group: a single bulk copy) and the group's
+//               zero points into a ring of their own.
 //   warps 1, 3  one thread each issues the MMAs of alternate groups: 4 x
 //               tcgen05.mma.kind::i8 (K = 32 each) into one of kAccBufs int32
 //               accumulators in tensor memory (TMEM), then one commit to the
@@ -111,8 +111,6 @@ struct GemmCfg {
   static constexpr int kStgSlots = 12;                         // raw scale staging ring
   static constexpr int kStgDist = 10;                          // groups prefetched ahead
   static constexpr int kStgBytes = BN * 2 + kBM * 4;           // raw fp16 s_w + fp32 s_a
-  // L2 prefetch distance in groups, past the loads the ring already holds
-  static constexpr int kPrefetchAhead = 4;
   // shared-memory layout (offsets from a 1024-byte aligned base)
   static constexpr int kOffRing = 0;
   static constexpr int kOffZ = kOffRing + kRingBytes;
@@ -140,7 +138,7 @@ __device__ __forceinline__ uint32_t sub_zero_bytes(uint32_t w, uint32_t zz) {
 
 template <int BN, bool kDebugP>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_w4w8a8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW4,
+    gemm_w4w8a8_kernel(const __grid_constant__ CUtensorMap tmA, const uint8_t *__restrict__ W4,
                        const __grid_constant__ CUtensorMap tmW8, const float *__restrict__ s_a,
                        const uint8_t *__restrict__ z4, const __half *__restrict__ s_w4,
                        const int32_t *__restrict__ idx4, const __half *__restrict__ s_w8,
@@ -205,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     prefetch_tmap(&tmA);
-    if (is4) prefetch_tmap(&tmW4); else prefetch_tmap(&tmW8);
+    if (!is4) prefetch_tmap(&tmW8);
     for (int s = 0; s < C::kMaxStages; ++s) mbar_init(&full[s], 1);
     for (int i = 0; i < C::kDone; ++i) mbar_init(&done[i], 1);
     for (int r = 0; r < C::kRaw; ++r) {
@@ -222,12 +220,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
-    // Weights do not depend on the kernel before this one: hint the first
-    // tiles into L2 while it may still be running (launched as a programmatic
-    // dependent, this CTA can start before the activation quantizer ends).
-    for (int g = 0; g < S && g < G; ++g) {
-      if (is4) tma_prefetch_l2_2d(&tmW4, g * (kKG / 2), n0); else tma_prefetch_l2_2d(&tmW8, g * kKG, n0);
-    }
     // Every global read of this grid comes after this wait: here, in the
     // table warp, and in the roles ordered after these loads by barriers.
     pdl_wait();
@@ -250,26 +242,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // One thread feeds both rings: the A stages (with W8 on 8-bit tiles),
       // each refilled once the MMAs of the group that held it are done, and on
       // 4-bit tiles the packed W4 tiles, each refilled once unpacked.  It
-      // polls both, so neither ring waits on the other, and keeps L2
-      // prefetches kPrefetchAhead groups ahead of each.
+      // polls both, so neither ring waits on the other.  (L2 prefetch hints
+      // ahead of the rings measured slower: they compete with the loads for
+      // the TMA unit's requests.)
       if (lane == 0) {
-        auto prefetch_a = [&](int g) {
-          if (g < G) {
-            tma_prefetch_l2_2d(&tmA, g * kKG, m0);
-            if (!is4) tma_prefetch_l2_2d(&tmW8, g * kKG, n0);
-          }
-        };
-        auto prefetch_w4 = [&](int g) {
-          if (g < G) {
-            tma_prefetch_l2_2d(&tmW4, g * (kKG / 2), n0);
-            bulk_prefetch_l2(z4 + static_cast<int64_t>(g) * (N4p >> 1) + (n0 >> 1), C::kZBytes);
-          }
-        };
         int ga = S < G ? S : G;  // next A group; the prologue issued groups 0 .. S-1
         int gw = is4 ? 0 : G;    // next packed W4 group
-        for (int g = ga; g < ga + C::kPrefetchAhead; ++g) prefetch_a(g);
-        if (is4)
-          for (int g = 0; g < C::kRaw + C::kPrefetchAhead; ++g) prefetch_w4(g);
         long long idle_since = -1;
         while (ga < G || gw < G) {
           bool progressed = false;
@@ -278,16 +256,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               (gw < C::kRaw || mbar_try_wait(smem_u32(&rempty[gw % C::kRaw]), ((gw / C::kRaw) - 1) & 1))) {
             const int r = gw % C::kRaw;
             mbar_arrive_expect_tx(&rfull[r], static_cast<uint32_t>(C::kW4Bytes + C::kZBytes));
-            tma_load_2d(raw_w4(r), &tmW4, &rfull[r], gw * (kKG / 2), n0);
+            // the tile's packed group is one contiguous block: one bulk copy
+            bulk_load(raw_w4(r), W4 + (static_cast<int64_t>(n0 >> 7) * G + gw) * C::kW4Bytes, C::kW4Bytes, &rfull[r]);
             bulk_load(zmeta(r), z4 + static_cast<int64_t>(gw) * (N4p >> 1) + (n0 >> 1), C::kZBytes, &rfull[r]);
-            prefetch_w4(gw + C::kRaw + C::kPrefetchAhead);
             ++gw;
             progressed = true;
           }
           // A stage ga % S last held group ga - S; it is free once that group is done
           if (ga < G && mbar_try_wait(smem_u32(&done[(ga - S) % C::kDone]), ((ga - S) / C::kDone) & 1)) {
             load_a(ga);
-            prefetch_a(ga + C::kPrefetchAhead);
             ++ga;
             progressed = true;
           }
@@ -664,16 +641,11 @@ static cudaError_t launch_gemm_bn(const GemmArgs &a, cudaStream_t stream, const 
     *msg = "cuTensorMapEncodeTiled is not available from the driver";
     return cudaErrorNotSupported;
   }
-  CUtensorMap tmA, tmW4, tmW8;
+  CUtensorMap tmA, tmW8;
   memset(&tmA, 0, sizeof(tmA));
-  memset(&tmW4, 0, sizeof(tmW4));
   memset(&tmW8, 0, sizeof(tmW8));
   if (!encode_2d_u8(enc, &tmA, a.A_q, a.K, a.M, kKG, kBM, true)) {
     *msg = "tensor map encoding of A_q failed";
-    return cudaErrorInvalidValue;
-  }
-  if (a.N4 > 0 && !encode_2d_u8(enc, &tmW4, a.W4, a.K / 2, a.N4, kKG / 2, BN, false)) {
-    *msg = "tensor map encoding of W4 failed";
     return cudaErrorInvalidValue;
   }
   if (a.N8 > 0 && !encode_2d_u8(enc, &tmW8, a.W8, a.K, a.N8, kKG, BN, true)) {
@@ -714,7 +686,7 @@ static cudaError_t launch_gemm_bn(const GemmArgs &a, cudaStream_t stream, const 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(
-      &cfg, kern, tmA, tmW4, tmW8, a.s_a, a.z4, static_cast<const __half *>(a.s_w4), a.idx4,
+      &cfg, kern, tmA, a.W4, tmW8, a.s_a, a.z4, static_cast<const __half *>(a.s_w4), a.idx4,
       static_cast<const __half *>(a.s_w8), a.idx8, static_cast<int>(a.M), static_cast<int>(a.K),
       static_cast<int>(a.N4), static_cast<int>(a.N8), static_cast<int>(padded_channels(a.N4)),
       static_cast<int>(padded_channels(a.N8)), mt, nt4, static_cast<__half *>(a.Y), a.P);

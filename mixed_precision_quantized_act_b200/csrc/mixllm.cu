@@ -123,7 +123,7 @@ mixllm_status mixllm_packed_sizes(int64_t N, int64_t K, int64_t N8, int32_t grou
   if (N < 0 || N8 < 0 || N8 > N) return fail(MIXLLM_ERR_INVALID_ARG, "need 0 <= N8 <= N");
   const int64_t N4 = N - N8, G = K / MIXLLM_GROUP;
   const int64_t N4p = mixllm::padded_channels(N4), N8p = mixllm::padded_channels(N8);
-  out_bytes[0] = static_cast<size_t>(N4 * (K / 2));
+  out_bytes[0] = static_cast<size_t>((N4 + 127) / 128 * 128 * (K / 2));  // whole 128-channel tiles
   out_bytes[1] = static_cast<size_t>(G * (N4p / 2));
   out_bytes[2] = static_cast<size_t>(G * N4p * 2);
   out_bytes[3] = static_cast<size_t>(N4 * 4);

@@ -148,9 +148,12 @@ __device__ __forceinline__ float warp_max(float v) {
 
 // ---------------------------------------------------------------------------
 // 4-bit asymmetric pack.  One warp per (pair of packed rows, group): the two
-// rows share the zero-point byte.  Lane l writes packed bytes 2l and 2l+1 of
-// the row's 64-byte group slice; byte b = 16c + i of a 32-k run c holds codes
-// k = 32c + i (low nibble) and k = 32c + 16 + i (high nibble).
+// rows share the zero-point byte.  The codes of row r, group g go to the
+// 64-byte row r % 128 of block (r / 128, g) -- each 128-channel tile's group
+// is one contiguous 8 KB block, loaded by the GEMM with a single bulk copy --
+// and lane l writes bytes 2l and 2l+1 of it: byte b = 16c + i of a 32-k run c
+// holds codes k = 32c + i (low nibble) and k = 32c + 16 + i (high nibble).
+// Rows of the last tile past N4 are written as zeros.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) pack_w4_kernel(const float *__restrict__ W, int64_t N, int64_t K,
                                                       const int32_t *__restrict__ idx4, int64_t N4, int64_t N4p,
@@ -192,11 +195,14 @@ __global__ void __launch_bounds__(256) pack_w4_kernel(const float *__restrict__ 
         for (int i = 0; i < 4; ++i) q[i] = static_cast<uint32_t>(max(0, min(15, __float2int_rn(__fdiv_rn(v[i], sf)) + z)));
       }
       const uint32_t two = (q[0] | (q[1] << 4)) | ((q[2] | (q[3] << 4)) << 8);
-      *reinterpret_cast<uint16_t *>(W4 + r * (K >> 1) + (g << 6) + 2 * lane) = static_cast<uint16_t>(two);
+      *reinterpret_cast<uint16_t *>(W4 + (((r >> 7) * G + g) * 128 + (r & 127)) * 64 + 2 * lane) =
+          static_cast<uint16_t>(two);
       if (lane == 0) s_w4[g * N4p + r] = sh;
       zpair |= static_cast<uint32_t>(z) << (4 * e);
-    } else if (lane == 0) {
-      s_w4[g * N4p + r] = __float2half_rn(0.0f);
+    } else {
+      if (r < ((N4 + 127) & ~int64_t(127)))  // padding row of the last tile
+        *reinterpret_cast<uint16_t *>(W4 + (((r >> 7) * G + g) * 128 + (r & 127)) * 64 + 2 * lane) = 0;
+      if (lane == 0) s_w4[g * N4p + r] = __float2half_rn(0.0f);
     }
   }
   if (lane == 0) z4[g * (N4p >> 1) + p] = static_cast<uint8_t>(zpair);

@@ -215,9 +215,10 @@ def padded(n: int) -> int:
 
 
 def pack_w4(q4: np.ndarray) -> np.ndarray:
+    """Packed 4-bit codes, [tiles of 128 channels, G, 128, 64] bytes."""
     q4 = _c(q4, np.uint8)
     N4, K = q4.shape
-    out = np.empty((N4, K // 2), np.uint8)
+    out = np.empty(((N4 + 127) // 128, K // 128, 128, 64), np.uint8)
     lib().oracle_pack_w4(_p(q4), N4, K, _p(out))
     return out
 

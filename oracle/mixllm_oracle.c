@@ -386,9 +386,11 @@ void oracle_group_partials(const int8_t *A_q, int64_t M, int64_t K,
 /* ------------------------------------------------------------------ */
 /* The library's packed weight layout, restated from its specification  */
 /* (a storage format, so both sides must agree on it byte for byte):    */
-/*   W4 bytes [N4, K/2]: in each run of 32 consecutive k of a row, byte */
-/*      i (0..15) holds element i in its low nibble and element i+16 in */
-/*      its high nibble.                                                 */
+/*   W4 bytes [ceil(N4/128)][G][128][64]: tile t, group g is one block  */
+/*      of 128 rows (channels 128t .. 128t+127 of the 4-bit set; rows   */
+/*      past N4 are zero) by the 64 bytes of the group's 128 codes; in  */
+/*      each run of 32 consecutive k, byte i (0..15) holds element i in */
+/*      its low nibble and element i+16 in its high nibble.             */
 /*   z4 bytes [G, Np/2]: zero point of channel n, group g, in byte      */
 /*      g*Np/2 + n/2, low nibble for even n, high nibble for odd n.     */
 /*   s (either set) fp16 [G, Np]: scale of channel n, group g at g*Np+n. */
@@ -397,13 +399,22 @@ void oracle_group_partials(const int8_t *A_q, int64_t M, int64_t K,
 
 void oracle_pack_w4(const uint8_t *q, int64_t N4, int64_t K, uint8_t *W4)
 {
-    for (int64_t n = 0; n < N4; ++n)
-        for (int64_t base = 0; base < K; base += 32)
-            for (int i = 0; i < 16; ++i) {
-                uint8_t lo = q[n * K + base + i] & 0x0F;
-                uint8_t hi = q[n * K + base + 16 + i] & 0x0F;
-                W4[n * (K / 2) + base / 2 + i] = (uint8_t)(lo | (hi << 4));
+    const int64_t G = K / 128, tiles = (N4 + 127) / 128;
+    memset(W4, 0, (size_t)(tiles * G * 128 * 64));
+    for (int64_t n = 0; n < N4; ++n) {
+        const int64_t t = n / 128, r = n % 128;
+        for (int64_t g = 0; g < G; ++g) {
+            uint8_t *row = W4 + ((t * G + g) * 128 + r) * 64;
+            for (int64_t run = 0; run < 4; ++run) {
+                const int64_t base = g * 128 + run * 32;
+                for (int i = 0; i < 16; ++i) {
+                    uint8_t lo = q[n * K + base + i] & 0x0F;
+                    uint8_t hi = q[n * K + base + 16 + i] & 0x0F;
+                    row[run * 16 + i] = (uint8_t)(lo | (hi << 4));
+                }
             }
+        }
+    }
 }
 
 void oracle_pack_zeros(const uint8_t *z, int64_t N, int64_t G, int64_t Np, uint8_t *z_packed)

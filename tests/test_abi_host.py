@@ -55,7 +55,8 @@ def test_packed_sizes_footprint(L):
     s = _lib.packed_sizes(N, K, N8)
     N4, G = N - N8, K // 128
     N4p, N8p = 3840, 512
-    assert s == [N4 * K // 2, G * N4p // 2, G * N4p * 2, N4 * 4, N8 * K, G * N8p * 2, N8 * 4]
+    T4 = (N4 + 127) // 128  # W4 is stored as whole 128-channel tiles (rows past N4 are zero)
+    assert s == [T4 * 128 * K // 2, G * N4p // 2, G * N4p * 2, N4 * 4, N8 * K, G * N8p * 2, N8 * 4]
     # without padding the per-weight footprints are the pages' 0.5 + 2.5/G and 1 + 2/G
     s2 = _lib.packed_sizes(512, 1024, 256)
     assert (s2[0] + s2[1] + s2[2]) / (256 * 1024) == 0.5 + 2.5 / 128

@@ -307,16 +307,23 @@ def test_moving_a_channel_changes_only_its_column(oracle_mod):
 
 def test_packed_nibbles_round_trip(oracle_mod):
     rng = np.random.default_rng(7)
-    q = rng.integers(0, 16, size=(5, 256)).astype(np.uint8)
+    N4, K = 133, 256  # two tiles of 128 channels, the second one ragged
+    q = rng.integers(0, 16, size=(N4, K)).astype(np.uint8)
     P = oracle_mod.pack_w4(q)
-    assert P.shape == (5, 128)
-    # unpack by the layout's definition: run of 32 -> byte i = (k_i, k_{i+16})
-    lo, hi = P & 0x0F, P >> 4
-    r = np.empty_like(q)
-    for base in range(0, 256, 32):
-        r[:, base:base + 16] = lo[:, base // 2: base // 2 + 16]
-        r[:, base + 16:base + 32] = hi[:, base // 2: base // 2 + 16]
-    assert np.array_equal(r, q)
+    assert P.shape == (2, 2, 128, 64)
+    # unpack by the layout's definition: tile t, group g is a [128 rows x 64 B]
+    # block; in a run of 32 codes, byte i = (k_i low, k_{i+16} high)
+    r = np.zeros((256, K), np.uint8)
+    for t in range(2):
+        for g in range(2):
+            blk = P[t, g]
+            lo, hi = blk & 0x0F, blk >> 4
+            for run in range(4):
+                k0 = g * 128 + run * 32
+                r[t * 128:(t + 1) * 128, k0:k0 + 16] = lo[:, run * 16:(run + 1) * 16]
+                r[t * 128:(t + 1) * 128, k0 + 16:k0 + 32] = hi[:, run * 16:(run + 1) * 16]
+    assert np.array_equal(r[:N4], q)
+    assert not r[N4:].any()  # rows past the set are zero
     z = rng.integers(0, 16, size=(5, 2)).astype(np.uint8)
     zp = oracle_mod.pack_zeros(z)
     assert zp.shape == (2, 128)
