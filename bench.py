@@ -367,12 +367,90 @@ def max_over_ranks(x, world):
     return dp.max_over_ranks(x, world, device="cuda")
 
 
+LAYER_WORKLOAD = "llama3.1-8b_layer"  # the four linears of one decoder layer, "@M<m>" picks M
+
+
+def run_layer(args, rank, world, local_rank):
+    """The decoder layer's four linears (qkv, o_proj, gate_up, down), each as
+    quantize + GEMM, replayed as one CUDA graph per step; L2 flushed before
+    each step, outside the graph.  Reports TOPS over the four GEMMs."""
+    import torch
+    import mixed_precision_quantized_act_b200 as mx
+    from mixed_precision_quantized_act_b200.layer import LinearChain
+
+    M = int(args.workload.split("@M")[1]) if "@M" in args.workload else 512
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    mx.load()
+    layers = [l.with_m(M) for l in wl.LLAMA8B_LAYER]
+    packed = [mx.pack_weights(torch.from_numpy(wl.make_w(l, args.seed)).to(dev),
+                              torch.from_numpy(wl.make_bitmap(l, args.seed)).to(dev)) for l in layers]
+    chain = LinearChain(packed, M, dev)
+    for l, x in zip(layers, chain.inputs):
+        x.copy_(torch.from_numpy(wl.make_x(l, dp.batch_seed(args.seed, rank))))
+    chain.capture()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1)
+        chain.replay()
+    mx.sync_status(stream)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            chain.replay()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    mx.sync_status(stream)
+    t_step = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / K, world)
+    chain.release()
+    ops = chain.ops()
+    if rank != 0:
+        return None
+    return {
+        "metric": "W4.4A8 decoder-layer linears (qkv, o_proj, gate_up, down) effective TOPS",
+        "value": ops * world / (t_step * 1e-3) / 1e12, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic (seeded N(0,1) X with x20 outlier columns, N(0,0.02) W, random 8-bit channel sets)",
+        "config": {"workload": f"{LAYER_WORKLOAD}@M{M}", "M": M, "linears": [l.name.split("_M")[0] for l in layers],
+                   "l2": "flushed by a 256 MiB device write before every timed step",
+                   "parallelism": f"dp{world} (weights replicated, M tokens per GPU)"},
+        "step": "8 kernels (4 x quantize_act + fused GEMM) replayed as one CUDA graph",
+        "gpu_launches": 8 * K,
+        "clocks": clocks.summary(),
+    }
+
+
 def main():
     args = parse()
-    layer = layer_for(args.workload)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.workload.startswith(LAYER_WORKLOAD):
+        if args.impl == "reference":
+            if rank == 0:
+                print(json.dumps({"impl": "reference", "unavailable": "the decoder-layer workload has no "
+                                  "CPU reference arm; use a single-linear workload"}), flush=True)
+            return
+        if world > 1:
+            import torch
+            torch.cuda.set_device(local_rank)
+            dp.init("nccl", timeout_s=120, device=torch.device("cuda", local_rank))
+        try:
+            line = run_layer(args, rank, world, local_rank)
+            if line is not None:
+                print(json.dumps(line), flush=True)
+        finally:
+            dp.shutdown(world)
+        return
+    layer = layer_for(args.workload)
     if args.impl == "reference":
         run_reference(args, layer, rank, world)
         return
