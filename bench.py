@@ -56,16 +56,24 @@ def parse():
 
 
 def layer_for(name):
-    for l in wl.ALL:
-        if l.name == name:
-            return l
-    raise SystemExit(f"unknown workload {name}")
+    try:
+        return wl.by_name(name)
+    except KeyError:
+        raise SystemExit(f"unknown workload {name}")
 
 
-def config_of(layer, n_gpus):
+# Few-token (decode) steps read a few MB of weights: instead of a flush, the
+# timed steps cycle over enough copies of the packed weights to exceed L2
+# twice over, as the layers of a decoder do, and run as one CUDA graph (the
+# host cannot issue eager launches as fast as the device runs them).
+ROTATE_BYTES = 300 * 1024 * 1024
+
+
+def config_of(layer, n_gpus, rotate=0):
+    l2 = (f"inputs larger than L2: {rotate} copies of the packed weights, step i uses copy i mod {rotate}"
+          if rotate else "flushed by a 256 MiB device write before every timed step")
     return {"workload": layer.name, "M": layer.M, "N": layer.N, "K": layer.K, "N8": layer.N8,
-            "N4": layer.N4, "group": 128,
-            "l2": "flushed by a 256 MiB device write before every timed step",
+            "N4": layer.N4, "group": 128, "l2": l2,
             "parallelism": f"dp{n_gpus} (weights replicated, M tokens per GPU)"}
 
 
@@ -225,59 +233,124 @@ def run_ours(args, layer, rank, world, local_rank):
 
     # few tokens (decode): the split-K path with its workspace; otherwise the tiled kernel
     small = layer.M <= mx.SMALL_M_MAX
+    copies = [p]
     if small:
         ws = mx.small_m_workspace(layer.M, p, dev)
+        ncopy = max(2, -(-ROTATE_BYTES // p.nbytes()))
+        copies += [mx.PackedLinear(**{k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in vars(p).items()})
+                   for _ in range(ncopy - 1)]
 
-        def gemm():
-            mx.gemm_w4w8a8_small_m_into(A_q, s_a, p, Y, ws, stream)
+        def gemm(i=0):
+            mx.gemm_w4w8a8_small_m_into(A_q, s_a, copies[i % len(copies)], Y, ws, stream)
     else:
-        def gemm():
+        def gemm(i=0):
             mx.gemm_w4w8a8_into(A_q, s_a, p, Y, stream)
 
-    def step():
+    def step(i=0):
         mx.quantize_act_into(Xd, A_q, s_a, stream)
-        gemm()
+        gemm(i)
 
-    for _ in range(max(args.warmup, 3)):
-        flush.fill_(1)
-        step()
+    for i in range(max(args.warmup, 3)):
+        if not small:
+            flush.fill_(1)
+        step(i)
     mx.sync_status(stream)
 
-    # Timed region: whole steps.  The GEMM is launched as a programmatic
-    # dependent of the quantizer, so nothing is recorded between the two.
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clocks:
-        for i in range(K):
-            flush.fill_(i & 0xFF)
-            ev[i][0].record(stream)
-            step()
-            ev[i][1].record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
-    mx.sync_status(stream)
-    t_step = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / K, world)
+    if small:
+        # Timed region: one graph of exactly K steps (the GEMM of each is a
+        # programmatic dependent of its quantizer), then one of Kk GEMMs alone
+        # for the per-kernel duration (its launch gaps included).
+        def captured(fn, n):
+            g = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream(device=dev)
+            side.wait_stream(torch.cuda.current_stream(dev))
+            with torch.cuda.stream(side):
+                fn(0)  # warm the library's cached descriptors on the capturing stream
+            torch.cuda.current_stream(dev).wait_stream(side)
+            with torch.cuda.graph(g, stream=side):
+                for i in range(n):
+                    fn(i)
+            return g
 
-    # Per-kernel durations for the roofline: the same steps with an event
-    # between the two kernels (which also keeps the GEMM from starting early,
-    # so this is its stand-alone duration).
-    Kk = min(K, 500)
-    ek = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(Kk)]
-    torch.cuda.synchronize()
-    for i in range(Kk):
-        flush.fill_(i & 0xFF)
-        ek[i][0].record(stream)
-        mx.quantize_act_into(Xd, A_q, s_a, stream)
-        ek[i][1].record(stream)
-        gemm()
-        ek[i][2].record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    mx.sync_status(stream)
-    t_gemm = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ek) / Kk, world)
-    t_quant = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ek) / Kk, world)
+        def graph_step(i):
+            mx.quantize_act_into(Xd, A_q, s_a, None)
+            mx.gemm_w4w8a8_small_m_into(A_q, s_a, copies[i % len(copies)], Y, ws, None)
+
+        def graph_gemm(i):
+            mx.gemm_w4w8a8_small_m_into(A_q, s_a, copies[i % len(copies)], Y, ws, None)
+
+        g_steps = captured(graph_step, K)
+        g_steps.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        with ClockSampler(local_rank) as clocks:
+            e0.record(stream)
+            g_steps.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+        barrier(world)
+        mx.sync_status(stream)
+        t_step = max_over_ranks(e0.elapsed_time(e1) / K, world)
+        del g_steps
+
+        Kk = min(K, 500)
+        g_gemm = captured(graph_gemm, Kk)
+        g_gemm.replay()
+        g_q = captured(lambda i: mx.quantize_act_into(Xd, A_q, s_a, None), Kk)
+        g_q.replay()
+        torch.cuda.synchronize()
+        e2, e3, e4 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e2.record(stream)
+        g_gemm.replay()
+        e3.record(stream)
+        g_q.replay()
+        e4.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        mx.sync_status(stream)
+        t_gemm = max_over_ranks(e2.elapsed_time(e3) / Kk, world)
+        t_quant = max_over_ranks(e3.elapsed_time(e4) / Kk, world)
+        del g_gemm, g_q
+        gemm_timed = f"{Kk} launches in one CUDA graph on rotating weight copies (launch gaps included)"
+    else:
+        # Timed region: whole steps.  The GEMM is launched as a programmatic
+        # dependent of the quantizer, so nothing is recorded between the two.
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        barrier(world)
+        torch.cuda.synchronize()
+        with ClockSampler(local_rank) as clocks:
+            for i in range(K):
+                flush.fill_(i & 0xFF)
+                ev[i][0].record(stream)
+                step()
+                ev[i][1].record(stream)
+            torch.cuda.synchronize()
+        barrier(world)
+        mx.sync_status(stream)
+        t_step = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / K, world)
+
+        # Per-kernel durations for the roofline: the same steps with an event
+        # between the two kernels (which also keeps the GEMM from starting early,
+        # so this is its stand-alone duration).
+        Kk = min(K, 500)
+        ek = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(Kk)]
+        torch.cuda.synchronize()
+        for i in range(Kk):
+            flush.fill_(i & 0xFF)
+            ek[i][0].record(stream)
+            mx.quantize_act_into(Xd, A_q, s_a, stream)
+            ek[i][1].record(stream)
+            gemm()
+            ek[i][2].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        mx.sync_status(stream)
+        t_gemm = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ek) / Kk, world)
+        t_quant = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ek) / Kk, world)
+        gemm_timed = f"{Kk} launches with an event before and after each, L2 flushed before each"
 
     # end to end through the public API: pinned host X in, host Y out
     Xh = torch.from_numpy(X).pin_memory()
@@ -291,10 +364,11 @@ def run_ours(args, layer, rank, world, local_rank):
     barrier(world)
     torch.cuda.synchronize()
     for i in range(Ke):
-        flush.fill_(i & 0xFF)
+        if not small:
+            flush.fill_(i & 0xFF)
         ee[i][0].record(stream)
         Xd.copy_(Xh, non_blocking=True)
-        step()
+        step(i)
         Yh.copy_(Y, non_blocking=True)
         ee[i][1].record(stream)
     torch.cuda.synchronize()
@@ -339,11 +413,12 @@ def run_ours(args, layer, rank, world, local_rank):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded N(0,1) X with x20 outlier "
-            "columns, N(0,0.02) W, random 8-bit channel set)", "config": config_of(layer, world),
-            "gemm_kernel": {"path": "few-token split-K" if small else "tiled", "ms": t_gemm, "tops": gemm_tops,
+            "columns, N(0,0.02) W, random 8-bit channel set)", "config": config_of(layer, world, len(copies) if small else 0),
+            "gemm_kernel": {"path": ("GEMV split-K" if layer.M <= 8 else "few-token split-K") if small else "tiled",
+                            "ms": t_gemm, "tops": gemm_tops,
                             "frac_of_int8_peak": gemm_tops / int8_peak,
                             "frac_of_nominal_4500": gemm_tops / 4500.0,
-                            "timed": f"{Kk} launches with an event before and after each, L2 flushed before each"},
+                            "timed": gemm_timed},
             "quantize_act_kernel": {"ms": t_quant,
                                     "gbs": (layer.M * layer.K * 3 + layer.M * layer.G * 4) / (t_quant * 1e-3) / 1e9},
             "roofline": roofline,
@@ -353,7 +428,8 @@ def run_ours(args, layer, rank, world, local_rank):
             "gpu_launches": 2 * K,
             "step": "quantize_act then the fused GEMM, launched as its programmatic dependent (its "
                     "prologue overlaps the quantizer's tail; it reads A_q and s_a only after the quantizer ends)"
-                    + ("; M <= 64 runs the few-token split-K path" if small else ""),
+                    + ("; M <= 8 runs the GEMV, 9 <= M <= 64 the few-token tensor-core kernel (both split-K)"
+                       if small else ""),
             "clocks": clocks.summary(),
         }
     return line

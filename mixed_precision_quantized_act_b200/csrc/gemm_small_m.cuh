@@ -27,6 +27,8 @@
 // unpack into the swizzled int8 operand (with few tokens it is the longest
 // per-group step), warps 12-15 epilogue (one TMEM lane quadrant each).  Every
 // wait is bounded as in the tiled kernel.
+// Up to kGemvMaxM tokens the entry points below run the GEMV kernel instead
+// (gemv_w4w8a8.cuh): the same plan, workspace layout and split reduction.
 #pragma once
 
 #include <cuda.h>
@@ -34,6 +36,8 @@
 #include <cudaTypedefs.h>
 #include <cstdint>
 
+#include "gemm_w4w8a8.cuh"
+#include "gemv_w4w8a8.cuh"
 #include "launch.h"
 #include "ptx_sm100.cuh"
 
@@ -87,9 +91,13 @@ struct SmallMCfg {
 };
 
 // Workspace of one call: S x tiles x MP x 128 fp32 partial sums (scratch),
-// then one int32 counter per tile (zero between calls).
+// then one int32 counter per tile (zero between calls).  gemv: the call runs
+// the GEMV kernel (M <= kGemvMaxM) with a token bound of MP in 1, 2, 4, 8,
+// `splits` splits per 4-bit tile and `splits8` per 8-bit tile (S above is
+// the larger); the tensor-core kernel uses `splits` for both sets.
 struct SmallMPlan {
-  int mp, nt4, nt8, splits, groups;
+  int mp, nt4, nt8, splits, splits8, groups;
+  bool gemv;
   size_t part_floats, counters;
   size_t bytes() const { return part_floats * 4 + counters * 4; }
 };
@@ -459,23 +467,45 @@ __global__ void __launch_bounds__(kSmThreads, 1)
 // host side
 // ---------------------------------------------------------------------------
 
-constexpr int kSmWave = 148;  // SMs of a B200: split-K fills one wave of CTAs
+constexpr int kSmWave = 148;      // SMs of a B200: split-K fills one wave of CTAs
+constexpr int kGemvMaxM = 8;      // up to this many tokens the GEMV kernel runs
+// GEMV grid target: the CTAs that are resident at once on the 148 SMs
+constexpr int gemv_cta_target(int mt) { return kSmWave * gemv_min_blocks(mt); }
+constexpr int gemv_groups_max(int mt) {
+  return mt == 1 ? GvCfg<1>::kGroupsMax
+                 : (mt == 2 ? GvCfg<2>::kGroupsMax : (mt == 4 ? GvCfg<4>::kGroupsMax : GvCfg<8>::kGroupsMax));
+}
 
 SmallMPlan plan_small_m(int64_t M, int64_t N4, int64_t N8, int64_t K) {
   SmallMPlan p{};
-  p.mp = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+  p.gemv = M <= kGemvMaxM;
+  if (p.gemv)
+    p.mp = M <= 1 ? 1 : (M <= 2 ? 2 : (M <= 4 ? 4 : 8));
+  else
+    p.mp = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
   p.nt4 = static_cast<int>((N4 + 127) / 128);
   p.nt8 = static_cast<int>((N8 + 127) / 128);
   p.groups = static_cast<int>(K / 128);
   const int tiles = p.nt4 + p.nt8;
-  int S = tiles > 0 ? kSmWave / tiles : 1;
-  if (S < 1) S = 1;
-  const int s_min = (p.groups + kSmGroupsMax - 1) / kSmGroupsMax;  // groups per CTA <= kSmGroupsMax
-  if (S < s_min) S = s_min;
-  if (S > p.groups) S = p.groups;
-  p.splits = S;
-  p.part_floats = S > 1 ? static_cast<size_t>(S) * tiles * p.mp * 128 : 0;
-  p.counters = S > 1 ? static_cast<size_t>(tiles) : 0;
+  // groups per CTA <= the kernel's cap
+  const int gmax = p.gemv ? gemv_groups_max(p.mp) : kSmGroupsMax;
+  const int s_min = (p.groups + gmax - 1) / gmax;
+  auto clamp_s = [&](int S) { return S < s_min ? s_min : (S > p.groups ? p.groups : S); };
+  if (p.gemv) {
+    // an 8-bit tile has twice the bytes of a 4-bit one: it counts twice and gets twice the splits
+    const int units = p.nt4 + 2 * p.nt8;
+    int base = units > 0 ? gemv_cta_target(p.mp) / units : 1;
+    if (base < 1) base = 1;
+    p.splits = clamp_s(base);
+    p.splits8 = clamp_s(2 * base);
+  } else {
+    int S = tiles > 0 ? kSmWave / tiles : 1;
+    if (S < 1) S = 1;
+    p.splits = p.splits8 = clamp_s(S);
+  }
+  const int smax = p.splits > p.splits8 ? p.splits : p.splits8;
+  p.part_floats = smax > 1 ? static_cast<size_t>(smax) * tiles * p.mp * 128 : 0;
+  p.counters = smax > 1 ? static_cast<size_t>(tiles) : 0;
   return p;
 }
 
@@ -539,6 +569,98 @@ static cudaError_t launch_small_m_mp(const GemmArgs &a, const SmallMPlan &p, voi
   return e;
 }
 
+// W8 [N8, K] int8 as a 3-D tensor (k within a group, row, group) with
+// 128 x 128 x groups_per_box boxes: whole groups of a 128-row tile, each
+// 128-byte row swizzled.  Encodings are cached by (base, K, N8, box).
+static bool encode_w8_groups_3d(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *map, const void *W8, int64_t K,
+                                int64_t N8, int groups_per_box) {
+  struct Entry {
+    const void *base;
+    int64_t K, N8;
+    int gpb;
+    bool valid;
+    CUtensorMap map;
+  };
+  static Entry table[32];
+  static int next = 0;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry &e : table)
+    if (e.valid && e.base == W8 && e.K == K && e.N8 == N8 && e.gpb == groups_per_box) {
+      *map = e.map;
+      return true;
+    }
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(N8), static_cast<cuuint64_t>(K / 128)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K), 128};  // bytes, dims 1 and 2
+  const cuuint32_t box[3] = {128, 128, static_cast<cuuint32_t>(groups_per_box)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(W8), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  table[next] = Entry{W8, K, N8, groups_per_box, true, *map};
+  next = (next + 1) % 32;
+  return true;
+}
+
+template <int MT>
+static cudaError_t launch_gemv_mt(const GemmArgs &a, const SmallMPlan &p, void *ws, cudaStream_t stream,
+                                  const char **msg) {
+  static_assert(gemv_min_blocks(MT) * (gemv_smem_bytes<MT>() + 1024) <= 228 * 1024, "resident CTAs per SM");
+  CUtensorMap tmW8;
+  memset(&tmW8, 0, sizeof(tmW8));
+  if (a.N8 > 0) {
+    auto enc = get_encode_fn();
+    if (!enc) {
+      *msg = "cuTensorMapEncodeTiled is not available from the driver";
+      return cudaErrorNotSupported;
+    }
+    if (!encode_w8_groups_3d(enc, &tmW8, a.W8, a.K, a.N8, GvCfg<MT>::kChunk8)) {
+      *msg = "tensor map encoding of W8 failed";
+      return cudaErrorInvalidValue;
+    }
+  }
+  const int tiles = p.nt4 + p.nt8;
+  const int64_t grid = static_cast<int64_t>(p.nt4) * p.splits + static_cast<int64_t>(p.nt8) * p.splits8;
+  if (grid > 0x7FFFFFFF) {
+    *msg = "too many tiles";
+    return cudaErrorInvalidValue;
+  }
+  auto kern = gemv_w4w8a8_kernel<MT>;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static unsigned long long configured = 0;  // one bit per device ordinal
+  if (dev < 64 && !(configured & (1ull << dev))) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gemv_smem_bytes<MT>());
+    if (e != cudaSuccess) {
+      *msg = "cudaFuncSetAttribute(MaxDynamicSharedMemorySize) failed";
+      return e;
+    }
+    configured |= 1ull << dev;
+  }
+  float *ws_part = static_cast<float *>(ws);
+  int *ws_cnt = p.counters > 0 ? reinterpret_cast<int *>(ws_part + p.part_floats) : nullptr;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kGvThreads);
+  cfg.dynamicSmemBytes = gemv_smem_bytes<MT>();
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(
+      &cfg, kern, tmW8, a.A_q, a.s_a, a.W4, a.z4, static_cast<const __half *>(a.s_w4), a.idx4,
+      static_cast<const __half *>(a.s_w8), a.idx8, static_cast<int>(a.M), static_cast<int>(a.K),
+      static_cast<int>(a.N4), static_cast<int>(a.N8), static_cast<int>(padded_channels(a.N4)),
+      static_cast<int>(padded_channels(a.N8)), p.nt4, tiles, p.splits, p.splits8, static_cast<__half *>(a.Y), ws_part,
+      ws_cnt);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) *msg = "launch of the GEMV failed";
+  return e;
+}
+
 size_t small_m_workspace_bytes(int64_t M, int64_t N4, int64_t N8, int64_t K) {
   return plan_small_m(M, N4, N8, K).bytes();
 }
@@ -548,6 +670,12 @@ cudaError_t launch_gemm_small_m(const GemmArgs &a, void *ws, size_t ws_bytes, cu
   if (ws_bytes < p.bytes() || (p.bytes() > 0 && !ws)) {
     *msg = "workspace too small for this shape";
     return cudaErrorInvalidValue;
+  }
+  if (p.gemv) {
+    if (p.mp == 1) return launch_gemv_mt<1>(a, p, ws, stream, msg);
+    if (p.mp == 2) return launch_gemv_mt<2>(a, p, ws, stream, msg);
+    if (p.mp == 4) return launch_gemv_mt<4>(a, p, ws, stream, msg);
+    return launch_gemv_mt<8>(a, p, ws, stream, msg);
   }
   if (p.mp == 16) return launch_small_m_mp<16>(a, p, ws, stream, msg);
   if (p.mp == 32) return launch_small_m_mp<32>(a, p, ws, stream, msg);

@@ -135,6 +135,15 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *m, uin
       : "memory");
 }
 
+// 3-D tiled load of one box into shared memory; completes on `bar` (tx bytes).
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *m, uint64_t *bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
 // Hint: bring one box of a tensor into L2 ahead of its load (no shared memory,
 // no completion to wait for).
 __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *m, int x, int y) {

@@ -142,7 +142,14 @@ def make_bitmap(layer: Linear, seed: int = 0) -> np.ndarray:
 
 
 def by_name(name: str) -> Linear:
+    """A workload of ALL by name, or any of them with another token count as
+    `<name>@M<m>`."""
     for layer in ALL:
         if layer.name == name:
             return layer
+    base, sep, m = name.rpartition("@M")
+    if sep and m.isdigit() and int(m) > 0:
+        for layer in ALL:
+            if layer.name == base:
+                return layer.with_m(int(m))
     raise KeyError(name)

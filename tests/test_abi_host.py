@@ -120,15 +120,29 @@ def test_binding_raises_without_cuda_tensors(L):
 
 def test_small_m_workspace_plan(L):
     """Workspace of the few-token path: S splits x tiles x (token tile x 128)
-    fp32 partials + one int32 counter per 128-channel tile; S fills one wave
-    of 148 CTAs and caps a CTA at 32 groups; no workspace without a split."""
+    fp32 partials + one int32 counter per 128-channel tile; no workspace
+    without a split; a CTA takes at most 32 groups.  Tensor-core kernel
+    (M > 8): S fills one wave of 148 CTAs, token tiles 16 / 32 / 64.  GEMV
+    (M <= 8): token bounds 1 / 2 / 4 / 8; an 8-bit tile counts as two 4-bit
+    ones, S4 = 296 // (nt4 + 2 nt8) splits per 4-bit tile and twice that per
+    8-bit tile, S the larger."""
     def ws(M, K, N4, N8):
         out = ctypes.c_size_t(0)
         st = L.mixllm_small_m_workspace_bytes(M, K, N4, N8, ctypes.byref(out))
         return st, out.value
 
-    # q_proj p10 at M=1: 29 + 4 tiles, S = 148 // 33 = 4, token tile 16
-    assert ws(1, 4096, 3686, 410) == (_lib.OK, 4 * 33 * 16 * 128 * 4 + 33 * 4)
+    # q_proj p10, 29 + 4 tiles.  GEMV: S4 = 296 // 37 = 8, S8 = 16
+    for M, bound in ((1, 1), (2, 2), (3, 4), (8, 8)):
+        assert ws(M, 4096, 3686, 410) == (_lib.OK, 16 * 33 * bound * 128 * 4 + 33 * 4)
+    # tensor-core kernel: M=9 -> S = 148 // 33 = 4, token tile 16
+    assert ws(9, 4096, 3686, 410) == (_lib.OK, 4 * 33 * 16 * 128 * 4 + 33 * 4)
+    # GEMV, 213 + 12 tiles: S4 = 296 // 237 = 1, S8 = 2
+    assert ws(1, 4096, 27238, 1434) == (_lib.OK, 2 * 225 * 1 * 128 * 4 + 225 * 4)
+    # GEMV, K = 28672 (224 groups), 58 + 7 tiles: S4 = max(296 // 72, 224 / 32) = 7, S8 = 8
+    assert ws(8, 28672, 7373, 819) == (_lib.OK, 8 * 65 * 8 * 128 * 4 + 65 * 4)
+    # GEMV, one 4-bit tile only: S4 = 296 (capped at G = 32); one 8-bit tile only: S8 = 2 * 148 -> 32
+    assert ws(1, 4096, 100, 0) == (_lib.OK, 32 * 1 * 1 * 128 * 4 + 1 * 4)
+    assert ws(1, 4096, 0, 100) == (_lib.OK, 32 * 1 * 1 * 128 * 4 + 1 * 4)
     # token tiles 32 and 64
     assert ws(17, 4096, 3686, 410) == (_lib.OK, 4 * 33 * 32 * 128 * 4 + 33 * 4)
     assert ws(64, 4096, 3686, 410) == (_lib.OK, 4 * 33 * 64 * 128 * 4 + 33 * 4)

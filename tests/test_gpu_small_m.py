@@ -43,10 +43,14 @@ def _layer(name, M, N, K, n8, outliers=4):
     return wl.Linear(name, M, N, K, ((0, N, n8),), outliers)
 
 
-# token tiles 16 / 32 / 64, ragged N, one set empty, one 8-bit channel,
-# split counts from 1 (wide N) to the group cap (long K)
+# GEMV (M <= 8: token bounds 1 / 2 / 4 / 8) and tensor-core kernel (token
+# tiles 16 / 32 / 64) on either side of M = 8, ragged N, one set empty, one
+# 8-bit channel, split counts from 1 (wide N) to the group cap (long K)
 CASES = [
     wl.Q_PROJ_P10.with_m(1),
+    wl.Q_PROJ_P10.with_m(2),
+    wl.Q_PROJ_P10.with_m(8),
+    wl.Q_PROJ_P10.with_m(9),
     wl.Q_PROJ_P10.with_m(16),
     wl.Q_PROJ_P10.with_m(64),
     _layer("sm_m5_ragged", 5, 300, 384, 37),
@@ -56,6 +60,8 @@ CASES = [
     _layer("sm_m7_p100", 7, 512, 512, 512),
     _layer("sm_m2_one_8bit", 2, 260, 256, 1),
     _layer("sm_m3_k128", 3, 384, 128, 40),
+    _layer("sm_m1_k8960", 1, 200, 8960, 30),
+    _layer("sm_m4_g33", 4, 640, 33 * 128, 70),
 ]
 
 
@@ -84,7 +90,8 @@ def test_small_m_matches_oracle(dev, layer):
     assert counters_zero(ws, p, layer.M, layer.K), "the tile counters must be back at zero"
 
 
-@pytest.mark.parametrize("layer", [wl.Q_PROJ_P10.with_m(16), _layer("sm_m33", 33, 640, 1024, 64)],
+@pytest.mark.parametrize("layer", [wl.Q_PROJ_P10.with_m(16), _layer("sm_m33", 33, 640, 1024, 64),
+                                   wl.Q_PROJ_P10.with_m(1), _layer("sm_m6", 6, 1000, 2048, 100)],
                          ids=lambda l: l.name)
 def test_small_m_deterministic_and_close_to_tiled(dev, layer):
     X, W, is8, A_q, s_a, p, ws, Y1 = _run(dev, layer, 12)
@@ -102,12 +109,14 @@ def test_small_m_deterministic_and_close_to_tiled(dev, layer):
     assert_y_close(Y1.cpu().numpy(), Y_ref, layer.name + " small-M")
 
 
-@pytest.mark.parametrize("layer", [wl.LLAMA8B_LAYER[2].with_m(8), wl.LLAMA70B[3].with_m(4)],
+@pytest.mark.parametrize("layer", [wl.LLAMA8B_LAYER[2].with_m(8), wl.LLAMA70B[3].with_m(4),
+                                   wl.LLAMA8B_LAYER[2].with_m(16), wl.LLAMA70B[3].with_m(12)],
                          ids=lambda l: l.name)
 def test_small_m_wide_and_long_layers(dev, layer):
     """8B gate_up (N = 28672: more tiles than SMs, no split) and 70B down
-    (K = 28672: the split count set by the per-CTA group cap); a random
-    subset of the columns against the oracle."""
+    (K = 28672: the split count set by the per-CTA group cap), on the GEMV
+    (M <= 8) and on the tensor-core kernel; a random subset of the columns
+    against the oracle."""
     X, W, is8, A_q, s_a, p, ws, Y = _run(dev, layer, 13)
     cols = np.sort(np.random.default_rng(3).choice(layer.N, 2048, replace=False))
     A_ref, s_ref = oracle.quantize_act(X)
