@@ -98,6 +98,10 @@ struct SmallMCfg {
 struct SmallMPlan {
   int mp, nt4, nt8, splits, splits8, groups;
   bool gemv;
+  // persistent GEMV (M <= kGemvMaxM and M*K within its resident-token bound):
+  // `ctas` CTAs share `units` 32 KiB units evenly; workspace [ctas][2][MP][128]
+  bool persistent;
+  int units, ctas, chunks4, chunks8;
   size_t part_floats, counters;
   size_t bytes() const { return part_floats * 4 + counters * 4; }
 };
@@ -471,6 +475,7 @@ constexpr int kSmWave = 148;      // SMs of a B200: split-K fills one wave of CT
 constexpr int kGemvMaxM = 8;      // up to this many tokens the GEMV kernel runs
 // GEMV grid target: the CTAs that are resident at once on the 148 SMs
 constexpr int gemv_cta_target(int mt) { return kSmWave * gemv_min_blocks(mt); }
+constexpr int kGvpMinUnitsPerCta = 8;  // the persistent GEMV from this many 32 KiB units per CTA
 constexpr int gemv_groups_max(int mt) {
   return mt == 1 ? GvCfg<1>::kGroupsMax
                  : (mt == 2 ? GvCfg<2>::kGroupsMax : (mt == 4 ? GvCfg<4>::kGroupsMax : GvCfg<8>::kGroupsMax));
@@ -491,6 +496,24 @@ SmallMPlan plan_small_m(int64_t M, int64_t N4, int64_t N8, int64_t K) {
   const int gmax = p.gemv ? gemv_groups_max(p.mp) : kSmGroupsMax;
   const int s_min = (p.groups + gmax - 1) / gmax;
   auto clamp_s = [&](int S) { return S < s_min ? s_min : (S > p.groups ? p.groups : S); };
+  // The persistent GEMV pays for its even shares with a reduction for every
+  // tile that two CTAs share; measured on B200 it wins from about 8 units per
+  // CTA (Llama 3.1 70B gate_up, down at M=1: 27 and 14 units per CTA, 19 % and
+  // 16 % faster) and loses below (8B gate_up, 6 units: 8 % slower).
+  const int chunks4 = (p.groups + 3) / 4, chunks8 = (p.groups + 1) / 2;
+  const int64_t U = static_cast<int64_t>(p.nt4) * chunks4 + static_cast<int64_t>(p.nt8) * chunks8;
+  if (p.gemv && p.mp <= kGvpMaxTokens && static_cast<int64_t>(p.mp) * K <= kGvpMaxTokenBytes &&
+      U >= static_cast<int64_t>(kGvpMinUnitsPerCta) * gemv_cta_target(p.mp)) {
+    p.persistent = true;
+    p.chunks4 = chunks4;
+    p.chunks8 = chunks8;
+    p.units = static_cast<int>(U);
+    p.ctas = static_cast<int>(U < gemv_cta_target(p.mp) ? U : gemv_cta_target(p.mp));
+    p.splits = p.splits8 = 1;
+    p.part_floats = static_cast<size_t>(p.ctas) * 2 * p.mp * 128;
+    p.counters = static_cast<size_t>(tiles);
+    return p;
+  }
   if (p.gemv) {
     // an 8-bit tile has twice the bytes of a 4-bit one: it counts twice and gets twice the splits
     const int units = p.nt4 + 2 * p.nt8;
@@ -661,6 +684,58 @@ static cudaError_t launch_gemv_mt(const GemmArgs &a, const SmallMPlan &p, void *
   return e;
 }
 
+template <int MT>
+static cudaError_t launch_gemv_persistent_mt(const GemmArgs &a, const SmallMPlan &p, void *ws, cudaStream_t stream,
+                                             const char **msg) {
+  static_assert(2 * (gvp_smem_bytes_max<MT>() + 1024) <= 228 * 1024, "two CTAs per SM");
+  CUtensorMap tmW8;
+  memset(&tmW8, 0, sizeof(tmW8));
+  if (a.N8 > 0) {
+    auto enc = get_encode_fn();
+    if (!enc) {
+      *msg = "cuTensorMapEncodeTiled is not available from the driver";
+      return cudaErrorNotSupported;
+    }
+    if (!encode_w8_groups_3d(enc, &tmW8, a.W8, a.K, a.N8, 2)) {
+      *msg = "tensor map encoding of W8 failed";
+      return cudaErrorInvalidValue;
+    }
+  }
+  auto kern = gemv_w4w8a8_persistent_kernel<MT>;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static unsigned long long configured = 0;  // one bit per device ordinal
+  if (dev < 64 && !(configured & (1ull << dev))) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gvp_smem_bytes_max<MT>());
+    if (e != cudaSuccess) {
+      *msg = "cudaFuncSetAttribute(MaxDynamicSharedMemorySize) failed";
+      return e;
+    }
+    configured |= 1ull << dev;
+  }
+  GvpGeom geo{p.nt4, p.chunks4, p.chunks8, p.units, p.ctas};
+  float *ws_part = static_cast<float *>(ws);
+  int *ws_cnt = reinterpret_cast<int *>(ws_part + p.part_floats);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.ctas));
+  cfg.blockDim = dim3(kGvThreads);
+  cfg.dynamicSmemBytes = 1024 + gvp_layout(MT, static_cast<int>(a.K)).total;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(
+      &cfg, kern, tmW8, a.A_q, a.s_a, a.W4, a.z4, static_cast<const __half *>(a.s_w4), a.idx4,
+      static_cast<const __half *>(a.s_w8), a.idx8, static_cast<int>(a.M), static_cast<int>(a.K),
+      static_cast<int>(a.N4), static_cast<int>(a.N8), static_cast<int>(padded_channels(a.N4)),
+      static_cast<int>(padded_channels(a.N8)), geo, static_cast<__half *>(a.Y), ws_part, ws_cnt);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) *msg = "launch of the persistent GEMV failed";
+  return e;
+}
+
 size_t small_m_workspace_bytes(int64_t M, int64_t N4, int64_t N8, int64_t K) {
   return plan_small_m(M, N4, N8, K).bytes();
 }
@@ -670,6 +745,12 @@ cudaError_t launch_gemm_small_m(const GemmArgs &a, void *ws, size_t ws_bytes, cu
   if (ws_bytes < p.bytes() || (p.bytes() > 0 && !ws)) {
     *msg = "workspace too small for this shape";
     return cudaErrorInvalidValue;
+  }
+  if (p.persistent) {
+    static_assert(kGvpMaxTokens == 4, "token bounds of the persistent GEMV");
+    if (p.mp == 1) return launch_gemv_persistent_mt<1>(a, p, ws, stream, msg);
+    if (p.mp == 2) return launch_gemv_persistent_mt<2>(a, p, ws, stream, msg);
+    return launch_gemv_persistent_mt<4>(a, p, ws, stream, msg);
   }
   if (p.gemv) {
     if (p.mp == 1) return launch_gemv_mt<1>(a, p, ws, stream, msg);

@@ -119,28 +119,35 @@ def test_binding_raises_without_cuda_tensors(L):
 
 
 def test_small_m_workspace_plan(L):
-    """Workspace of the few-token path: S splits x tiles x (token tile x 128)
-    fp32 partials + one int32 counter per 128-channel tile; no workspace
-    without a split; a CTA takes at most 32 groups.  Tensor-core kernel
-    (M > 8): S fills one wave of 148 CTAs, token tiles 16 / 32 / 64.  GEMV
-    (M <= 8): token bounds 1 / 2 / 4 / 8; an 8-bit tile counts as two 4-bit
-    ones, S4 = 296 // (nt4 + 2 nt8) splits per 4-bit tile and twice that per
-    8-bit tile, S the larger."""
+    """Workspace of the few-token path.  Tensor-core kernel (M > 8) and the
+    split GEMV: S splits x tiles x (token tile x 128) fp32 partials + one int32
+    counter per 128-channel tile, none without a split, at most 32 groups per
+    CTA; the tensor-core kernel's S fills one wave of 148 CTAs (token tiles
+    16 / 32 / 64), the split GEMV's S4 = 296 // (nt4 + 2 nt8) per 4-bit tile
+    and twice that per 8-bit tile.  Persistent GEMV (M <= 4, bound*K <= 32 KiB
+    and U >= 8 * 296 units, U = nt4*ceil(G/4) + nt8*ceil(G/2)): P = 296 CTAs,
+    [P][2][bound][128] fp32 partials + one counter per tile."""
     def ws(M, K, N4, N8):
         out = ctypes.c_size_t(0)
         st = L.mixllm_small_m_workspace_bytes(M, K, N4, N8, ctypes.byref(out))
         return st, out.value
 
-    # q_proj p10, 29 + 4 tiles.  GEMV: S4 = 296 // 37 = 8, S8 = 16
+    # q_proj p10, 29 + 4 tiles (U = 296, too few units for the persistent GEMV):
+    # split, S4 = 296 // 37 = 8, S8 = 16
     for M, bound in ((1, 1), (2, 2), (3, 4), (8, 8)):
         assert ws(M, 4096, 3686, 410) == (_lib.OK, 16 * 33 * bound * 128 * 4 + 33 * 4)
     # tensor-core kernel: M=9 -> S = 148 // 33 = 4, token tile 16
     assert ws(9, 4096, 3686, 410) == (_lib.OK, 4 * 33 * 16 * 128 * 4 + 33 * 4)
-    # GEMV, 213 + 12 tiles: S4 = 296 // 237 = 1, S8 = 2
+    # split, 213 + 12 tiles: S4 = 296 // 237 = 1, S8 = 2
     assert ws(1, 4096, 27238, 1434) == (_lib.OK, 2 * 225 * 1 * 128 * 4 + 225 * 4)
-    # GEMV, K = 28672 (224 groups), 58 + 7 tiles: S4 = max(296 // 72, 224 / 32) = 7, S8 = 8
+    # persistent, 70B gate_up (404 + 45 tiles, G = 64): U = 404*16 + 45*32 = 7904
+    assert ws(1, 8192, 51610, 5734) == (_lib.OK, 296 * 2 * 1 * 128 * 4 + 449 * 4)
+    assert ws(4, 8192, 51610, 5734) == (_lib.OK, 296 * 2 * 4 * 128 * 4 + 449 * 4)
+    # ... but not at M = 5 (token bound 8): split, S4 = max(296 // 494, 1) = 1, S8 = 2
+    assert ws(5, 8192, 51610, 5734) == (_lib.OK, 2 * 449 * 8 * 128 * 4 + 449 * 4)
+    # split GEMV (8 x 28672 > 32 KiB), 58 + 7 tiles: S4 = max(296 // 72, 224 / 32) = 7, S8 = 8
     assert ws(8, 28672, 7373, 819) == (_lib.OK, 8 * 65 * 8 * 128 * 4 + 65 * 4)
-    # GEMV, one 4-bit tile only: S4 = 296 (capped at G = 32); one 8-bit tile only: S8 = 2 * 148 -> 32
+    # split, one 4-bit tile only: S4 = 296 (capped at G = 32); one 8-bit tile only: S8 = 592 -> 32
     assert ws(1, 4096, 100, 0) == (_lib.OK, 32 * 1 * 1 * 128 * 4 + 1 * 4)
     assert ws(1, 4096, 0, 100) == (_lib.OK, 32 * 1 * 1 * 128 * 4 + 1 * 4)
     # token tiles 32 and 64
@@ -152,6 +159,7 @@ def test_small_m_workspace_plan(L):
     assert ws(16, 28672, 7373, 819) == (_lib.OK, 7 * 65 * 16 * 128 * 4 + 65 * 4)
     # one group: nothing to split
     assert ws(3, 128, 300, 84) == (_lib.OK, 0)
+    assert ws(9, 128, 300, 84) == (_lib.OK, 0)
     assert ws(65, 4096, 100, 10)[0] == _lib.ERR_INVALID_ARG
     assert ws(0, 4096, 100, 10)[0] == _lib.ERR_INVALID_ARG
     assert ws(8, 100, 100, 10)[0] == _lib.ERR_UNSUPPORTED

@@ -110,13 +110,16 @@ def test_small_m_deterministic_and_close_to_tiled(dev, layer):
 
 
 @pytest.mark.parametrize("layer", [wl.LLAMA8B_LAYER[2].with_m(8), wl.LLAMA70B[3].with_m(4),
+                                   wl.LLAMA70B[3].with_m(1), wl.LLAMA70B[2].with_m(3), wl.LLAMA8B_LAYER[3].with_m(2),
                                    wl.LLAMA8B_LAYER[2].with_m(16), wl.LLAMA70B[3].with_m(12)],
                          ids=lambda l: l.name)
 def test_small_m_wide_and_long_layers(dev, layer):
-    """8B gate_up (N = 28672: more tiles than SMs, no split) and 70B down
-    (K = 28672: the split count set by the per-CTA group cap), on the GEMV
-    (M <= 8) and on the tensor-core kernel; a random subset of the columns
-    against the oracle."""
+    """8B / 70B gate_up (N = 28672 / 57344) and 70B / 8B down (K = 28672 /
+    14336): the persistent GEMV, whose CTAs take units of several tiles and
+    share tiles with their neighbours (70B down M=1, 70B gate_up M=3), the
+    split GEMV (8B gate_up M=8, 70B down M=4, 8B down M=2) and the
+    tensor-core kernel (M=16, 12); a random subset of the columns against the
+    oracle."""
     X, W, is8, A_q, s_a, p, ws, Y = _run(dev, layer, 13)
     cols = np.sort(np.random.default_rng(3).choice(layer.N, 2048, replace=False))
     A_ref, s_ref = oracle.quantize_act(X)
