@@ -39,7 +39,9 @@ METRIC = "W4.4A8 GEMM effective TOPS at M=512,N=K=4096; % of B200 int8 TC peak"
 UNIT = "TOPS"
 NOMINAL_INT8_OVER_BF16 = 4.5 / 2.25  # dense tensor peaks, ops per bf16 flop
 GEMM_SRC = os.path.join(ROOT, "mixed_precision_quantized_act_b200", "csrc", "gemm_w4w8a8.cuh")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemm_w4w8a8_traffic.json")
+# ncu DRAM traffic per launch of the dominant kernel, per workload: a single
+# entry or {"entries": [...]}, used while its source hash matches the CUDA sources
+TRAFFIC_FILES = [os.path.join(ROOT, "profiles", f) for f in ("gemm_w4w8a8_traffic.json", "gemv_w4w8a8_traffic.json")]
 
 
 def parse():
@@ -77,10 +79,13 @@ def config_of(layer, n_gpus, rotate=0):
             "parallelism": f"dp{n_gpus} (weights replicated, M tokens per GPU)"}
 
 
-def source_hash():
+def source_hash(files=None):
+    """sha256 (16 hex digits) of CUDA sources of the library, in the order
+    given (default: every file of csrc/, sorted)."""
+    d = os.path.dirname(GEMM_SRC)
     h = hashlib.sha256()
-    for f in sorted(os.listdir(os.path.dirname(GEMM_SRC))):
-        with open(os.path.join(os.path.dirname(GEMM_SRC), f), "rb") as fh:
+    for f in files if files is not None else sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
@@ -381,13 +386,19 @@ def run_ours(args, layer, rank, world, local_rank):
     peaks, peak_src = measured_peaks()
     int8_peak = peaks["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
     traffic = None
-    try:
-        with open(TRAFFIC_FILE) as f:
-            tr = json.load(f)
-        if tr.get("source_hash") == source_hash() and tr.get("workload") == layer.name:
-            traffic = tr["dram_bytes_per_launch"]
-    except (OSError, ValueError, KeyError):
-        pass
+    for path in TRAFFIC_FILES:
+        try:
+            with open(path) as f:
+                tr = json.load(f)
+        except (OSError, ValueError):
+            continue
+        for e in tr.get("entries", [tr]):
+            try:
+                current = source_hash(e.get("sources"))
+            except OSError:
+                continue
+            if e.get("source_hash") == current and e.get("workload") == layer.name:
+                traffic = e.get("dram_bytes_per_launch")
 
     if small:  # HBM-bound: the packed weights are nearly all the bytes
         gemm_gbs = layer.algorithmic_bytes() / (t_gemm * 1e-3) / 1e9
@@ -414,7 +425,7 @@ def run_ours(args, layer, rank, world, local_rank):
             "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded N(0,1) X with x20 outlier "
             "columns, N(0,0.02) W, random 8-bit channel set)", "config": config_of(layer, world, len(copies) if small else 0),
-            "gemm_kernel": {"path": ("GEMV split-K" if layer.M <= 8 else "few-token split-K") if small else "tiled",
+            "gemm_kernel": {"path": mx.small_m_kernel(layer.M, layer.K, p.N4, p.N8) if small else "tiled",
                             "ms": t_gemm, "tops": gemm_tops,
                             "frac_of_int8_peak": gemm_tops / int8_peak,
                             "frac_of_nominal_4500": gemm_tops / 4500.0,

@@ -191,14 +191,36 @@ MIXLLM_API mixllm_status mixllm_small_m_workspace_bytes(int64_t M, int64_t K, in
                                              size_t *bytes);
 
 /*
+ * Which kernel mixllm_gemm_w4w8a8_small_m (and its _noalloc form) runs for a
+ * shape, in *kind:
+ *   MIXLLM_SMALL_M_TENSOR_CORE     9 <= M <= 64: int8 tensor-core tiles, split-K;
+ *   MIXLLM_SMALL_M_GEMV_SPLIT      M <= 8: the GEMV, split-K over each tile's groups;
+ *   MIXLLM_SMALL_M_GEMV_PERSISTENT M <= 4 with M*K <= 32768 and at least
+ *                                  8 x 296 units of 32 KiB of weights: the
+ *                                  GEMV with an even share of units per CTA.
+ * Pure host function, with the arguments and errors of
+ * mixllm_small_m_workspace_bytes (kind must not be NULL).  The pages have no
+ * counterpart: it reports the library's own choice, for logs and benchmarks.
+ */
+typedef enum {
+  MIXLLM_SMALL_M_TENSOR_CORE = 0,
+  MIXLLM_SMALL_M_GEMV_SPLIT = 1,
+  MIXLLM_SMALL_M_GEMV_PERSISTENT = 2
+} mixllm_small_m_kind;
+MIXLLM_API mixllm_status mixllm_small_m_kernel(int64_t M, int64_t K, int64_t N4, int64_t N8, int32_t *kind);
+
+/*
  * The same layer and the same result rule as mixllm_gemm_w4w8a8, laid out
  * for few tokens (1 <= M <= 64, the decode regime, where the packed weights
- * are nearly all the bytes and HBM bandwidth bounds the layer): the weight
- * tile is the tensor core's 128-row side and the tokens its 16/32/64-column
- * side, and the groups of every 128-channel tile are split among several
- * CTAs so the grid fills the GPU.  Each split writes fp32 partial sums to the
- * workspace; the last split of a tile to finish adds them in split order (the
- * result does not depend on timing) and writes Y.  The rounding differs from
+ * are nearly all the bytes and HBM bandwidth bounds the layer).  For
+ * 9 <= M <= 64 the weight tile is the tensor core's 128-row side and the
+ * tokens its 16/32/64-column side; for M <= 8 a GEMV streams the packed
+ * weights through shared memory and forms the exact int32 group partials
+ * with dp4a (mixllm_small_m_kernel says which).  Either way the groups of
+ * every 128-channel tile are split among several CTAs so the grid fills the
+ * GPU: each part writes fp32 partial sums to the workspace, and the last one
+ * of a tile to finish adds them in K order (the result does not depend on
+ * timing) and writes Y.  The rounding differs from
  * mixllm_gemm_w4w8a8 only in the order of the fp32 operations (Y is within
  * the same tolerance of the reference definition).
  * Arguments: as mixllm_gemm_w4w8a8, plus

@@ -23,6 +23,7 @@ from ._lib import (  # noqa: F401
     quantize_act,
     quantize_act_into,
     selftest_wait_timeout,
+    small_m_kernel,
     small_m_workspace,
     small_m_workspace_bytes,
     sync_status,

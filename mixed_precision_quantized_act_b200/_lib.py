@@ -34,6 +34,7 @@ SIGNATURES = {
     "mixllm_gemm_debug_partials": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64,
                                                   _vp, _vp, _vp, _i64, _vp, _vp]),
     "mixllm_small_m_workspace_bytes": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(ctypes.c_size_t)]),
+    "mixllm_small_m_kernel": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(ctypes.c_int32)]),
     "mixllm_gemm_w4w8a8_small_m": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64,
                                                   _vp, _vp, _vp, _i64, _vp, _vp, ctypes.c_size_t, _vp]),
     "mixllm_gemm_w4w8a8_small_m_noalloc": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64,
@@ -215,6 +216,16 @@ def small_m_workspace_bytes(M: int, K: int, N4: int, N8: int) -> int:
     out = ctypes.c_size_t(0)
     _check(load().mixllm_small_m_workspace_bytes(M, K, N4, N8, ctypes.byref(out)), "mixllm_small_m_workspace_bytes")
     return out.value
+
+
+SMALL_M_KERNELS = ("tensor-core split-K", "GEMV split-K", "GEMV persistent")
+
+
+def small_m_kernel(M: int, K: int, N4: int, N8: int) -> str:
+    """The few-token kernel the library runs for this shape (mixllm_small_m_kernel)."""
+    out = ctypes.c_int32(-1)
+    _check(load().mixllm_small_m_kernel(M, K, N4, N8, ctypes.byref(out)), "mixllm_small_m_kernel")
+    return SMALL_M_KERNELS[out.value]
 
 
 def small_m_workspace(M: int, p: PackedLinear, device) -> torch.Tensor:

@@ -740,6 +740,11 @@ size_t small_m_workspace_bytes(int64_t M, int64_t N4, int64_t N8, int64_t K) {
   return plan_small_m(M, N4, N8, K).bytes();
 }
 
+int small_m_kernel_kind(int64_t M, int64_t N4, int64_t N8, int64_t K) {
+  const SmallMPlan p = plan_small_m(M, N4, N8, K);
+  return p.persistent ? 2 : (p.gemv ? 1 : 0);
+}
+
 cudaError_t launch_gemm_small_m(const GemmArgs &a, void *ws, size_t ws_bytes, cudaStream_t stream, const char **msg) {
   const SmallMPlan p = plan_small_m(a.M, a.N4, a.N8, a.K);
   if (ws_bytes < p.bytes() || (p.bytes() > 0 && !ws)) {

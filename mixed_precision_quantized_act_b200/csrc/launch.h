@@ -45,6 +45,8 @@ cudaError_t launch_gemm_w4w8a8(const GemmArgs &a, cudaStream_t stream, const cha
 // Y only; no debug partials.
 cudaError_t launch_gemm_small_m(const GemmArgs &a, void *ws, size_t ws_bytes, cudaStream_t stream, const char **msg);
 size_t small_m_workspace_bytes(int64_t M, int64_t N4, int64_t N8, int64_t K);
+// 0: tensor-core kernel, 1: split GEMV, 2: persistent GEMV (mixllm_small_m_kind)
+int small_m_kernel_kind(int64_t M, int64_t N4, int64_t N8, int64_t K);
 // The same with a static device scratch instead of a workspace (no allocation);
 // fails with cudaErrorInvalidValue when the shape needs more than it holds.
 cudaError_t launch_gemm_small_m_noalloc(const GemmArgs &a, cudaStream_t stream, const char **msg);

@@ -224,6 +224,16 @@ mixllm_status mixllm_small_m_workspace_bytes(int64_t M, int64_t K, int64_t N4, i
   return ok();
 }
 
+mixllm_status mixllm_small_m_kernel(int64_t M, int64_t K, int64_t N4, int64_t N8, int32_t *kind) {
+  mixllm_status st = check_k(K, MIXLLM_GROUP);
+  if (st != MIXLLM_OK) return st;
+  if (!kind) return fail(MIXLLM_ERR_INVALID_ARG, "null kind");
+  if (M < 1 || M > 64) return fail(MIXLLM_ERR_INVALID_ARG, "the small-M path takes 1 <= M <= 64");
+  if (N4 < 0 || N8 < 0 || N4 + N8 > 0x7FFFFFF0) return fail(MIXLLM_ERR_INVALID_ARG, "bad N4 / N8");
+  *kind = mixllm::small_m_kernel_kind(M, N4, N8, K);
+  return ok();
+}
+
 mixllm_status mixllm_gemm_w4w8a8_small_m(const int8_t *A_q, const float *s_a, int64_t M, int64_t K,
                                          const uint8_t *W4, const uint8_t *z4, const void *s_w4_f16,
                                          const int32_t *idx4, int64_t N4, const int8_t *W8, const void *s_w8_f16,

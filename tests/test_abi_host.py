@@ -118,6 +118,30 @@ def test_binding_raises_without_cuda_tensors(L):
                                torch.zeros(2, 1), None)
 
 
+def test_small_m_kernel_choice(L):
+    """mixllm_small_m_kernel: tensor cores from M = 9, the GEMV below; the
+    persistent GEMV only for M <= 4, M*K <= 32 KiB and >= 8 x 296 units."""
+    def kind(M, K, N4, N8):
+        out = ctypes.c_int32(-1)
+        st = L.mixllm_small_m_kernel(M, K, N4, N8, ctypes.byref(out))
+        return st, out.value
+
+    assert kind(9, 4096, 3686, 410) == (_lib.OK, 0)
+    assert kind(64, 4096, 3686, 410) == (_lib.OK, 0)
+    assert kind(1, 4096, 3686, 410) == (_lib.OK, 1)       # q_proj: 296 units
+    assert kind(8, 4096, 27238, 1434) == (_lib.OK, 1)     # 8B gate_up: 1896 units
+    assert kind(1, 8192, 51610, 5734) == (_lib.OK, 2)     # 70B gate_up: 7904 units
+    assert kind(4, 8192, 51610, 5734) == (_lib.OK, 2)
+    assert kind(5, 8192, 51610, 5734) == (_lib.OK, 1)     # token bound 8
+    assert kind(1, 28672, 7373, 819) == (_lib.OK, 2)      # 70B down: 4032 units, 1 x 28672 bytes of codes
+    assert kind(2, 28672, 7373, 819) == (_lib.OK, 1)      # 2 x 28672 > 32 KiB
+    assert kind(0, 4096, 100, 10)[0] == _lib.ERR_INVALID_ARG
+    assert kind(65, 4096, 100, 10)[0] == _lib.ERR_INVALID_ARG
+    assert kind(8, 100, 100, 10)[0] == _lib.ERR_UNSUPPORTED
+    assert L.mixllm_small_m_kernel(1, 4096, 100, 10, None) == _lib.ERR_INVALID_ARG
+    assert _lib.small_m_kernel(1, 8192, 51610, 5734) == "GEMV persistent"
+
+
 def test_small_m_workspace_plan(L):
     """Workspace of the few-token path.  Tensor-core kernel (M > 8) and the
     split GEMV: S splits x tiles x (token tile x 128) fp32 partials + one int32
