@@ -69,6 +69,8 @@ def configure(L):
     L.oracle_pack_w4.argtypes = [vp, i64, i64, vp]
     L.oracle_pack_zeros.argtypes = [vp, i64, i64, i64, vp]
     L.oracle_pack_scales.argtypes = [vp, i64, i64, i64, vp]
+    L.oracle_channel_salience.argtypes = [vp, i64, i64, vp, i64, vp]
+    L.oracle_select_top_t.argtypes = [vp, i64, i64, vp]
     return L
 
 
@@ -253,3 +255,27 @@ def packed(Wq: Quantized) -> dict:
         "s_w8": pack_scales(Wq.s8),
         "idx8": Wq.idx8.copy(),
     }
+
+
+# ---------------------------------------------------------------- global search
+
+def channel_salience(W: np.ndarray, G: np.ndarray) -> np.ndarray:
+    """Salience S [N] (fp64) of every output channel of one layer:
+    W fp32 [N, K], G fp32 [D, N, K] per-sample gradients."""
+    W = _c(W, np.float32)
+    G = _c(G, np.float32)
+    N, K = W.shape
+    D = G.shape[0]
+    assert G.shape == (D, N, K)
+    S = np.zeros(N, np.float64)
+    lib().oracle_channel_salience(_p(W), N, K, _p(G), D, _p(S))
+    return S
+
+
+def select_top_t(S: np.ndarray, T: int) -> np.ndarray:
+    """Bit map [Ntot] (uint8) of the T channels of largest fp32 salience,
+    equal saliences in index order."""
+    S = _c(S, np.float32)
+    is8 = np.zeros(S.size, np.uint8)
+    lib().oracle_select_top_t(_p(S), S.size, int(T), _p(is8))
+    return is8

@@ -38,8 +38,12 @@
  *   R4 two-step GEMM: P = sum_{k in g} (Wq - z)*Aq in exact integers; then
  *      acc = acc + (float)P * (s_w * s_a), groups in ascending order, fp32;
  *      Y = fp16(acc).
+ *   R5 channel salience: c_q is the channel's 4-bit asymmetric quantization
+ *      (R2), dequantized as s*(q - z); the gradients are inputs; fp64.
+ *   R6 top-T selection: equal saliences in list order (lower index first).
  */
 #include <math.h>
+#include <stdlib.h>
 #include <stdint.h>
 #include <string.h>
 
@@ -435,4 +439,77 @@ void oracle_pack_scales(const uint16_t *s, int64_t N, int64_t G, int64_t Np, uin
     for (int64_t g = 0; g < G; ++g)
         for (int64_t n = 0; n < N; ++n)
             s_packed[g * Np + n] = s[n * G + g];
+}
+
+/* ------------------------------------------------------------------ */
+/* Global mixed-precision search, step 1: the salience of every output  */
+/* channel (MLSys 2026 talk notes on MixLLM, notes.yuuk.io,             */
+/* §グローバル混合精度探索).  The loss change of quantizing channel c   */
+/* alone, expanded to second order with the Fisher approximation of the */
+/* Hessian, reduces to                                                  */
+/*   S_c = (1/|D|) sum_d | g_d^T (c_q - c_0) + 1/2 (g_d^T (c_q - c_0))^2 | */
+/* with g_d the gradient of the loss on sample d with respect to the    */
+/* channel's weights, c_0 the channel's weights and c_q the channel     */
+/* after quantization.  Reading taken: c_q is the low-bit form of the   */
+/* layer, the 4-bit asymmetric group quantization of                    */
+/* oracle_quantize_w4, dequantized as s * (q - z).                      */
+/* W fp32 [N, K]; G fp32 [D, N, K]; S fp64 [N].  Everything in fp64.    */
+/* ------------------------------------------------------------------ */
+void oracle_channel_salience(const float *W, int64_t N, int64_t K, const float *G, int64_t D, double *S)
+{
+    const int64_t Gr = K / ORACLE_GROUP;
+    uint8_t *q = (uint8_t *)malloc((size_t)(N * K));
+    uint8_t *z = (uint8_t *)malloc((size_t)(N * Gr));
+    uint16_t *s = (uint16_t *)malloc((size_t)(N * Gr) * sizeof(uint16_t));
+    double *delta = (double *)malloc((size_t)K * sizeof(double));
+    oracle_quantize_w4(W, N, K, q, z, s);
+    for (int64_t n = 0; n < N; ++n) {
+        /* c_q - c_0, exact in fp64 */
+        for (int64_t k = 0; k < K; ++k) {
+            const int64_t g = k / ORACLE_GROUP;
+            const double cq = (double)oracle_f16_to_f32(s[n * Gr + g]) * (double)((int)q[n * K + k] - (int)z[n * Gr + g]);
+            delta[k] = cq - (double)W[n * K + k];
+        }
+        double acc = 0.0;
+        for (int64_t d = 0; d < D; ++d) {
+            const float *gd = G + (d * N + n) * K;
+            double t = 0.0;
+            for (int64_t k = 0; k < K; ++k) t += (double)gd[k] * delta[k];
+            acc += fabs(t + 0.5 * t * t);
+        }
+        S[n] = D > 0 ? acc / (double)D : 0.0;
+    }
+    free(q);
+    free(z);
+    free(s);
+    free(delta);
+}
+
+/* ------------------------------------------------------------------ */
+/* Global mixed-precision search, step 2 (Algorithm 1 of the same      */
+/* notes): all output channels of all layers in one list, sorted by    */
+/* salience in descending order; the first T are given 8 bits.         */
+/* Reading taken: equal saliences keep their list order (the lower     */
+/* index first), so the set is unique.  S fp32 [Ntot] (both sides take */
+/* this integer decision from the same fp32 keys); is8 [Ntot].         */
+/* ------------------------------------------------------------------ */
+static const float *g_sel_keys;
+static int sel_cmp(const void *a, const void *b)
+{
+    const int64_t i = *(const int64_t *)a, j = *(const int64_t *)b;
+    const float si = g_sel_keys[i], sj = g_sel_keys[j];
+    if (si > sj) return -1;
+    if (si < sj) return 1;
+    return i < j ? -1 : (i > j ? 1 : 0);
+}
+
+void oracle_select_top_t(const float *S, int64_t Ntot, int64_t T, uint8_t *is8)
+{
+    int64_t *order = (int64_t *)malloc((size_t)(Ntot > 0 ? Ntot : 1) * sizeof(int64_t));
+    for (int64_t i = 0; i < Ntot; ++i) order[i] = i;
+    g_sel_keys = S;
+    qsort(order, (size_t)Ntot, sizeof(int64_t), sel_cmp);
+    for (int64_t i = 0; i < Ntot; ++i) is8[i] = 0;
+    for (int64_t r = 0; r < T && r < Ntot; ++r) is8[order[r]] = 1;
+    free(order);
 }

@@ -11,6 +11,7 @@ import pytest
 
 import oracle
 from tests import test_oracle_pins as pins
+from tests import test_oracle_salience as sal
 
 MUTATIONS = {
     "zero_point_sign_in_gemm": ("p += ((int32_t)q[i] - (int32_t)zp) * (int32_t)a[i];",
@@ -34,6 +35,11 @@ MUTATIONS = {
     "w4_scale_not_rounded_to_fp16": (
         "            float sf = oracle_f16_to_f32(sh);\n            int zi = 0;",
         "            float sf = sc;\n            int zi = 0;"),
+    "salience_delta_sign": ("delta[k] = cq - (double)W[n * K + k];", "delta[k] = (double)W[n * K + k] - cq;"),
+    "salience_second_order_not_halved": ("acc += fabs(t + 0.5 * t * t);", "acc += fabs(t + t * t);"),
+    "salience_no_absolute_value": ("acc += fabs(t + 0.5 * t * t);", "acc += (t + 0.5 * t * t);"),
+    "salience_first_group_scale": ("(double)oracle_f16_to_f32(s[n * Gr + g])", "(double)oracle_f16_to_f32(s[n * Gr])"),
+    "top_t_ties_high_index_first": ("return i < j ? -1 : (i > j ? 1 : 0);", "return i > j ? -1 : (i < j ? 1 : 0);"),
     "w8_scale_from_wrong_group": ("float v = fabsf(w[i]);\n                if (v > amax) amax = v;\n            }\n            float sc = amax / 127.0f;",
                                   "float v = fabsf(w[i % 64]);\n                if (v > amax) amax = v;\n            }\n            float sc = amax / 127.0f;"),
 }
@@ -52,6 +58,13 @@ def _pins():
         yield pins.test_gemm_matches_fp64_brute_force, case
     yield pins.test_group_partials_int64_brute_force, ()
     yield pins.test_partial_bounds_fit_bias_window, ()
+    # the global search pins call the module directly (the swapped library)
+    for fn in (sal.test_channel_on_the_grid_has_zero_salience, sal.test_zero_gradients_give_zero_salience,
+               sal.test_each_group_uses_its_own_scale_and_the_dot_product_spans_the_row,
+               sal.test_channels_are_independent, sal.test_top_t_ties_and_bounds, sal.test_top_t_selects_the_largest):
+        yield (lambda _o, f=fn: f()), ()
+    for eps in (0.25 * sal.S_GRID, -0.375 * sal.S_GRID):
+        yield (lambda _o, e=eps: sal.test_one_perturbed_weight_closed_form(e)), ()
 
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
