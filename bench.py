@@ -515,8 +515,129 @@ def run_layer(args, rank, world, local_rank):
     }
 
 
+SEARCH_WORKLOAD = "llama3.1-8b_search_q_gate_D16"  # global salience search over two layers' channels
+
+
+def run_search(args, rank, world, local_rank):
+    """The global mixed-precision search (salience of every output channel,
+    then the global top 10 %) over a q_proj-shaped (4096 x 4096) and a
+    gate_proj-shaped (14336 x 4096) layer with 16 synthetic gradient samples
+    per channel: 4.8 GB of gradients, larger than L2, so no flush."""
+    import numpy as np
+    import torch
+    import mixed_precision_quantized_act_b200 as mx
+    from mixed_precision_quantized_act_b200 import _lib
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    mx.load()
+    D, K = 16, 4096
+    Ns = [4096, 14336]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(args.seed * 1000 + rank)
+    Ws = [torch.randn(N, K, device=dev, generator=gen) * 0.02 for N in Ns]
+    Gs = [torch.randn(D, N, K, device=dev, generator=gen) for N in Ns]
+    n_all = sum(Ns)
+    T = n_all // 10
+    S = torch.empty(n_all, dtype=torch.float32, device=dev)
+    is8 = torch.empty(n_all, dtype=torch.uint8, device=dev)
+    ws = _lib.select_top_t_workspace(n_all, dev)
+    stream = torch.cuda.current_stream()
+    offs = [0, Ns[0]]
+
+    def salience():
+        for W, G, o, N in zip(Ws, Gs, offs, Ns):
+            _lib.channel_salience_into(W, G, S[o:o + N], stream)
+
+    def step():
+        salience()
+        _lib.select_top_t_into(S, T, is8, ws, stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    mx.sync_status(stream)
+    Kst = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(Kst)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        for i in range(Kst):
+            ev[i][0].record(stream)
+            salience()
+            ev[i][1].record(stream)
+            _lib.select_top_t_into(S, T, is8, ws, stream)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    mx.sync_status(stream)
+    t_step = max_over_ranks(sum(e[0].elapsed_time(e[2]) for e in ev) / Kst, world)
+    t_sal = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / Kst, world)
+    t_sel = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ev) / Kst, world)
+    sal_bytes = sum(D * N * K * 4 + N * K * 4 + N * 4 for N in Ns)
+    step_bytes = sal_bytes + n_all * (6 * 4 + 1)  # + the selection: six passes over the scores, the bit map
+
+    # end to end: gradients from pinned host memory every step, the bit map back
+    Gh = [G.cpu().pin_memory() for G in Gs]
+    is8_h = torch.empty(n_all, dtype=torch.uint8).pin_memory()
+    Ke = min(Kst, 3)
+    ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Ke)]
+    torch.cuda.synchronize()
+    for i in range(Ke):
+        ee[i][0].record(stream)
+        for G, h in zip(Gs, Gh):
+            G.copy_(h, non_blocking=True)
+        step()
+        is8_h.copy_(is8, non_blocking=True)
+        ee[i][1].record(stream)
+    torch.cuda.synchronize()
+    t_e2e = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ee) / Ke, world)
+
+    if rank != 0:
+        return None
+    # the oracle on a sample of channels of the first layer
+    rows = 512
+    Wn = Ws[0][:rows].cpu().numpy()
+    Gn = Gs[0][:, :rows].cpu().numpy()
+    t0 = time.perf_counter()
+    import oracle
+    oracle.channel_salience(Wn, Gn)
+    secs = time.perf_counter() - t0
+    cpu_gbs = (D * rows * K * 4 + rows * K * 4) / secs / 1e9
+    peaks, peak_src = measured_peaks()
+    gbs = step_bytes * world / (t_step * 1e-3) / 1e9
+    sal_gbs = sal_bytes / (t_sal * 1e-3) / 1e9
+    return {
+        "metric": "global salience search (channel salience of two layers + global top 10 %), bytes moved per second",
+        "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": Kst, "warmup": args.warmup,
+        "ms_per_step": t_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded N(0,0.02) W, N(0,1) per-sample gradients)",
+        "config": {"workload": SEARCH_WORKLOAD, "layers": [[N, K] for N in Ns], "samples": D, "T": T,
+                   "l2": "inputs larger than L2 (4.8 GB of gradients)", "parallelism": f"dp{world}"},
+        "salience_kernels": {"ms": t_sal, "gbs": sal_gbs}, "select_kernels": {"ms": t_sel},
+        "roofline": {"bound": "hbm", "achieved": sal_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": sal_gbs / peaks["hbm_gbs"], "traffic": None,
+                     "peak_source": f"{peak_src} HBM copy {peaks['hbm_gbs']} GB/s", "algorithmic_bytes": sal_bytes},
+        "cpu_baseline": {"value": cpu_gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{rows} channels of the 4096 x 4096 layer x {D} samples, fp64, {secs:.2f} s"},
+        "e2e": {"value": step_bytes / (t_e2e * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": sum(G.numel() * 4 for G in Gs), "d2h_bytes_per_step": n_all},
+        "gpu_launches": 14 * Kst,
+        "step": "2 x channel_salience_kernel, then the radix select (init, 4 x (histogram + pick), count, scan, mark)",
+        "clocks": clocks.summary(),
+    }
+
+
 def main():
     args = parse()
+    if args.workload == SEARCH_WORKLOAD:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the search workload has no reference arm; "
+                              "its cpu_baseline is the oracle on a channel sample"}), flush=True)
+            return
+        line = run_search(args, int(os.environ.get("RANK", "0")), 1, int(os.environ.get("LOCAL_RANK", "0")))
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

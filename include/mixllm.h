@@ -269,6 +269,44 @@ MIXLLM_API mixllm_status mixllm_gemm_w4w8a8_small_m_noalloc(const int8_t *A_q, c
                                                  void *Y_f16, void *stream);
 
 /*
+ * Global mixed-precision search, step 1 (MLSys 2026 talk notes on MixLLM,
+ * notes.yuuk.io, §グローバル混合精度探索): the salience of every output channel
+ * n of one linear layer,
+ *   S[n] = (1/D) sum_d | t_d + t_d^2 / 2 |,  t_d = sum_k G[d, n, k] (c_q - c_0)[n, k],
+ * the loss change of quantizing channel n alone to second order, with the
+ * Hessian approximated by the Fisher matrix.  c_0 is the channel's weights and
+ * c_q their 4-bit asymmetric group quantization (the one
+ * mixllm_pack_weights applies), dequantized as s * (q - z).
+ *   W   device fp32 [N, K] row-major, 16-byte aligned (the layer's weights).
+ *   G   device fp32 [D, N, K], 16-byte aligned: G[d, n, :] is the gradient of
+ *       the loss on calibration sample d with respect to channel n's weights.
+ *   S   device fp32 [N], written.
+ * K a positive multiple of 128 up to 56832 (the row of c_q - c_0 is held in
+ * shared memory); D >= 1.  fp32 arithmetic in a fixed order: the result is
+ * deterministic and within the rounding of an fp32 dot product of the exact
+ * value.  Asynchronous on `stream`; the caller owns every buffer.
+ */
+MIXLLM_API mixllm_status mixllm_channel_salience(const float *W, int64_t N, int64_t K, const float *G, int64_t D,
+                                                 float *S, void *stream);
+
+/* Workspace bytes of mixllm_select_top_t for n scores.  Pure host function. */
+MIXLLM_API mixllm_status mixllm_select_top_t_workspace_bytes(int64_t n, size_t *bytes);
+
+/*
+ * Global mixed-precision search, step 2 (Algorithm 1 of the same notes): the
+ * scores of all channels of all layers in one list S (device fp32 [n], no
+ * NaN; the concatenation order is the caller's); is8[i] = 1 for the T
+ * largest, 0 for the rest (device uint8 [n], written).  Equal scores are
+ * taken in list order (the lower index first), so the result is unique; -0
+ * and +0 are equal.  0 <= T <= n.  workspace: device, at least
+ * mixllm_select_top_t_workspace_bytes(n) bytes, 16-byte aligned, no
+ * initialisation needed; not shared by calls that run at the same time.
+ * Asynchronous on `stream` (a radix select on the device, no host round trip).
+ */
+MIXLLM_API mixllm_status mixllm_select_top_t(const float *S, int64_t n, int64_t T, uint8_t *is8, void *workspace,
+                                             size_t workspace_bytes, void *stream);
+
+/*
  * Waits for `stream`, then reads and clears the device status word of the
  * current device.  Returns MIXLLM_ERR_TIMEOUT if a kernel of this library
  * gave up a wait since the last call, MIXLLM_ERR_CUDA if the stream reports

@@ -12,6 +12,7 @@ from ._lib import (  # noqa: F401
     empty_packed,
     gemm_debug_partials,
     gemm_w4w8a8,
+    channel_salience,
     gemm_w4w8a8_into,
     gemm_w4w8a8_small_m,
     gemm_w4w8a8_small_m_noalloc_into,
@@ -22,6 +23,7 @@ from ._lib import (  # noqa: F401
     packed_sizes,
     quantize_act,
     quantize_act_into,
+    select_top_t,
     selftest_wait_timeout,
     small_m_kernel,
     small_m_workspace,

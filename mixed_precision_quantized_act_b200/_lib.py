@@ -35,6 +35,9 @@ SIGNATURES = {
                                                   _vp, _vp, _vp, _i64, _vp, _vp]),
     "mixllm_small_m_workspace_bytes": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(ctypes.c_size_t)]),
     "mixllm_small_m_kernel": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(ctypes.c_int32)]),
+    "mixllm_channel_salience": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i64, _vp, _vp]),
+    "mixllm_select_top_t_workspace_bytes": (ctypes.c_int, [_i64, ctypes.POINTER(ctypes.c_size_t)]),
+    "mixllm_select_top_t": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, ctypes.c_size_t, _vp]),
     "mixllm_gemm_w4w8a8_small_m": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64,
                                                   _vp, _vp, _vp, _i64, _vp, _vp, ctypes.c_size_t, _vp]),
     "mixllm_gemm_w4w8a8_small_m_noalloc": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64,
@@ -282,3 +285,59 @@ def sync_status(stream=None):
 
 def selftest_wait_timeout(limit_us: int, stream=None):
     _check(load().mixllm_selftest_wait_timeout(limit_us, _stream(stream)), "mixllm_selftest_wait_timeout")
+
+
+# ---------------------------------------------------------------- global search
+
+def channel_salience(W: torch.Tensor, G: torch.Tensor, stream=None) -> torch.Tensor:
+    """Salience of every output channel of one layer (mixllm_channel_salience):
+    W fp32 [N, K], G fp32 [D, N, K] per-sample gradients, both on the device."""
+    _need_cuda(W, G)
+    W = W.contiguous()
+    G = G.contiguous()
+    N, K = W.shape
+    D = G.shape[0]
+    if G.dtype != torch.float32 or W.dtype != torch.float32 or tuple(G.shape) != (D, N, K):
+        raise ValueError("W must be fp32 [N, K] and G fp32 [D, N, K]")
+    S = torch.empty(N, dtype=torch.float32, device=W.device)
+    _check(load().mixllm_channel_salience(_ptr(W), N, K, _ptr(G), D, _ptr(S), _stream(stream)),
+           "mixllm_channel_salience")
+    return S
+
+
+def channel_salience_into(W: torch.Tensor, G: torch.Tensor, S: torch.Tensor, stream=None):
+    """mixllm_channel_salience into a caller's fp32 [N] tensor (e.g. a slice
+    of one list of all layers' scores)."""
+    N, K = W.shape
+    D = G.shape[0]
+    if not (W.is_contiguous() and G.is_contiguous() and S.is_contiguous()) or S.numel() != N:
+        raise ValueError("contiguous W [N, K], G [D, N, K] and S [N] expected")
+    _check(load().mixllm_channel_salience(_ptr(W), N, K, _ptr(G), D, _ptr(S), _stream(stream)),
+           "mixllm_channel_salience")
+
+
+def select_top_t_workspace(n: int, device) -> torch.Tensor:
+    out = ctypes.c_size_t(0)
+    _check(load().mixllm_select_top_t_workspace_bytes(n, ctypes.byref(out)), "mixllm_select_top_t_workspace_bytes")
+    return torch.empty(max(16, out.value), dtype=torch.uint8, device=device)
+
+
+def select_top_t_into(S: torch.Tensor, T: int, is8: torch.Tensor, workspace: torch.Tensor, stream=None):
+    """mixllm_select_top_t with the caller's bit map and workspace."""
+    _check(load().mixllm_select_top_t(_ptr(S), S.numel(), int(T), _ptr(is8), _ptr(workspace), workspace.numel(),
+                                      _stream(stream)), "mixllm_select_top_t")
+
+
+def select_top_t(S: torch.Tensor, T: int, stream=None) -> torch.Tensor:
+    """Bit map of the T largest scores, equal scores in index order
+    (mixllm_select_top_t): S fp32 [n] on the device."""
+    _need_cuda(S)
+    S = S.contiguous()
+    n = S.numel()
+    out = ctypes.c_size_t(0)
+    _check(load().mixllm_select_top_t_workspace_bytes(n, ctypes.byref(out)), "mixllm_select_top_t_workspace_bytes")
+    ws = torch.empty(max(1, out.value), dtype=torch.uint8, device=S.device)
+    is8 = torch.empty(n, dtype=torch.uint8, device=S.device)
+    _check(load().mixllm_select_top_t(_ptr(S), n, int(T), _ptr(is8), _ptr(ws), out.value, _stream(stream)),
+           "mixllm_select_top_t")
+    return is8

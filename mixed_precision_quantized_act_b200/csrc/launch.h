@@ -54,6 +54,13 @@ size_t small_m_scratch_capacity();
 
 cudaError_t launch_selftest_wait_timeout(uint32_t limit_us, cudaStream_t stream);
 
+// Global mixed-precision search (search.cuh).
+cudaError_t launch_channel_salience(const float *W, int64_t N, int64_t K, const float *G, int64_t D, float *S,
+                                    cudaStream_t stream, const char **msg);
+size_t select_top_t_workspace_bytes(int64_t n);
+cudaError_t launch_select_top_t(const float *S, int64_t n, int64_t T, uint8_t *is8, void *ws, cudaStream_t stream,
+                                const char **msg);
+
 int64_t padded_channels(int64_t n);  // n rounded up to a multiple of 256
 
 }  // namespace mixllm

@@ -12,6 +12,7 @@
 #include "../../include/mixllm.h"
 #include "gemm_w4w8a8.cuh"
 #include "gemm_small_m.cuh"
+#include "search.cuh"
 #include "launch.h"
 #include "quant.cuh"
 
@@ -280,6 +281,50 @@ mixllm_status mixllm_gemm_w4w8a8_small_m_noalloc(const int8_t *A_q, const float 
   const char *msg = "";
   cudaError_t e = mixllm::launch_gemm_small_m_noalloc(a, static_cast<cudaStream_t>(stream), &msg);
   if (e == cudaErrorNotSupported) return fail(MIXLLM_ERR_UNSUPPORTED, "%s", msg);
+  if (e != cudaSuccess) return fail(MIXLLM_ERR_CUDA, "%s: %s", msg, cudaGetErrorString(e));
+  return ok();
+}
+
+mixllm_status mixllm_channel_salience(const float *W, int64_t N, int64_t K, const float *G, int64_t D, float *S,
+                                      void *stream) {
+  mixllm_status st = check_k(K, MIXLLM_GROUP);
+  if (st != MIXLLM_OK) return st;
+  if (K > 56832) return fail(MIXLLM_ERR_UNSUPPORTED, "K = %lld is beyond 56832", static_cast<long long>(K));
+  if (N < 0 || D < 1) return fail(MIXLLM_ERR_INVALID_ARG, "need N >= 0 and D >= 1");
+  if (N > 0x7FFFFFFF) return fail(MIXLLM_ERR_INVALID_ARG, "N beyond the supported 2^31 range");
+  if (N == 0) return ok();
+  if (!W || !G || !S) return fail(MIXLLM_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(W, 16) || !aligned(G, 16) || !aligned(S, 4))
+    return fail(MIXLLM_ERR_INVALID_ARG, "W and G must be 16-byte aligned, S 4-byte aligned");
+  st = check_device();
+  if (st != MIXLLM_OK) return st;
+  const char *msg = "";
+  cudaError_t e = mixllm::launch_channel_salience(W, N, K, G, D, S, static_cast<cudaStream_t>(stream), &msg);
+  if (e != cudaSuccess) return fail(MIXLLM_ERR_CUDA, "%s: %s", msg, cudaGetErrorString(e));
+  return ok();
+}
+
+mixllm_status mixllm_select_top_t_workspace_bytes(int64_t n, size_t *bytes) {
+  if (!bytes) return fail(MIXLLM_ERR_INVALID_ARG, "null bytes");
+  if (n < 0 || n > (1ll << 40)) return fail(MIXLLM_ERR_INVALID_ARG, "bad n");
+  *bytes = mixllm::select_top_t_workspace_bytes(n);
+  return ok();
+}
+
+mixllm_status mixllm_select_top_t(const float *S, int64_t n, int64_t T, uint8_t *is8, void *workspace,
+                                  size_t workspace_bytes, void *stream) {
+  if (n < 0 || n > (1ll << 40)) return fail(MIXLLM_ERR_INVALID_ARG, "bad n");
+  if (T < 0 || T > n) return fail(MIXLLM_ERR_INVALID_ARG, "need 0 <= T <= n");
+  if (n == 0) return ok();
+  if (!S || !is8) return fail(MIXLLM_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(S, 4)) return fail(MIXLLM_ERR_INVALID_ARG, "S must be 4-byte aligned");
+  const size_t need = mixllm::select_top_t_workspace_bytes(n);
+  if (workspace_bytes < need || !workspace || !aligned(workspace, 16))
+    return fail(MIXLLM_ERR_INVALID_ARG, "workspace must be a 16-byte aligned device buffer of %zu bytes", need);
+  mixllm_status st = check_device();
+  if (st != MIXLLM_OK) return st;
+  const char *msg = "";
+  cudaError_t e = mixllm::launch_select_top_t(S, n, T, is8, workspace, static_cast<cudaStream_t>(stream), &msg);
   if (e != cudaSuccess) return fail(MIXLLM_ERR_CUDA, "%s: %s", msg, cudaGetErrorString(e));
   return ok();
 }

@@ -147,6 +147,31 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // ---------------------------------------------------------------------------
+// The 4-bit asymmetric quantizer of one group (MLSys 2026 talk notes on MixLLM,
+// notes.yuuk.io, §設計判断の概要: 4-bit asymmetric, group 128), given the
+// group's range lo = min(0, min w), hi = max(0, max w): scale
+// fp16(min((hi - lo) / 15, 65504)) (IEEE division), zero point
+// clamp(rne(-lo / s), 0, 15), code clamp(rne(w / s) + z, 0, 15); a zero scale
+// gives z = q = 0.  Shared by the packer and the channel-salience search.
+// ---------------------------------------------------------------------------
+struct W4Params {
+  __half sh;  // the scale as stored
+  float sf;   // the same as fp32
+  int z;
+};
+__device__ __forceinline__ W4Params w4_params(float lo, float hi) {
+  W4Params p;
+  const float sc = fminf(__fdiv_rn(__fsub_rn(hi, lo), 15.0f), 65504.0f);
+  p.sh = __float2half_rn(sc);
+  p.sf = __half2float(p.sh);
+  p.z = p.sf != 0.0f ? max(0, min(15, __float2int_rn(__fdiv_rn(-lo, p.sf)))) : 0;
+  return p;
+}
+__device__ __forceinline__ int w4_code(float v, const W4Params &p) {
+  return p.sf != 0.0f ? max(0, min(15, __float2int_rn(__fdiv_rn(v, p.sf)) + p.z)) : 0;
+}
+
+// ---------------------------------------------------------------------------
 // 4-bit asymmetric pack.  One warp per (pair of packed rows, group): the two
 // rows share the zero-point byte.  The codes of row r, group g go to the
 // 64-byte row r % 128 of block (r / 128, g) -- each 128-channel tile's group
@@ -184,16 +209,12 @@ __global__ void __launch_bounds__(256) pack_w4_kernel(const float *__restrict__ 
       }
       lo = warp_min(lo);
       hi = warp_max(hi);
-      const float sc = fminf(__fdiv_rn(__fsub_rn(hi, lo), 15.0f), 65504.0f);
-      const __half sh = __float2half_rn(sc);
-      const float sf = __half2float(sh);
-      int z = 0;
-      uint32_t q[4] = {0u, 0u, 0u, 0u};
-      if (sf != 0.0f) {
-        z = max(0, min(15, __float2int_rn(__fdiv_rn(-lo, sf))));
+      const W4Params wp = w4_params(lo, hi);
+      const __half sh = wp.sh;
+      const int z = wp.z;
+      uint32_t q[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) q[i] = static_cast<uint32_t>(max(0, min(15, __float2int_rn(__fdiv_rn(v[i], sf)) + z)));
-      }
+      for (int i = 0; i < 4; ++i) q[i] = static_cast<uint32_t>(w4_code(v[i], wp));
       const uint32_t two = (q[0] | (q[1] << 4)) | ((q[2] | (q[3] << 4)) << 8);
       *reinterpret_cast<uint16_t *>(W4 + (((r >> 7) * G + g) * 128 + (r & 127)) * 64 + 2 * lane) =
           static_cast<uint16_t>(two);
