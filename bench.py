@@ -509,8 +509,9 @@ def run_layer(args, rank, world, local_rank):
         "config": {"workload": f"{LAYER_WORKLOAD}@M{M}", "M": M, "linears": [l.name.split("_M")[0] for l in layers],
                    "l2": "flushed by a 256 MiB device write before every timed step",
                    "parallelism": f"dp{world} (weights replicated, M tokens per GPU)"},
-        "step": "8 kernels (4 x quantize_act + fused GEMM) replayed as one CUDA graph",
-        "gpu_launches": 8 * K,
+        "step": f"{chain.launches()} kernels (each linear: quantize_act + the GEMM, or for one token the GEMV "
+                "quantizing its own activations) replayed as one CUDA graph",
+        "gpu_launches": chain.launches() * K,
         "clocks": clocks.summary(),
     }
 

@@ -246,6 +246,36 @@ MIXLLM_API mixllm_status mixllm_gemm_w4w8a8_small_m(const int8_t *A_q, const flo
                                          void *stream);
 
 /*
+ * The whole few-token layer from fp16 activations: quantize_act and
+ * mixllm_gemm_w4w8a8_small_m in one call, with the same result (the same
+ * codes, scales and kernel arithmetic, so Y is bit-identical to the two calls).
+ * For one token, where the plan runs the split GEMV and a CTA's slice of X
+ * (groups x 256 bytes) fits one 32 KiB slot of its weight ring, the GEMV
+ * quantizes that slice itself in its prologue (no A_q in HBM, one launch);
+ * otherwise the activations are quantized into the workspace first (two
+ * launches; with more tokens every CTA quantizing its own slice costs more
+ * than the separate pass).
+ * This fuses the activation quantization into the GEMM prologue for decode
+ * (MLSys 2026 talk notes on MixLLM, notes.yuuk.io, §設計判断の概要 and
+ * §二段階逆量子化による int8 Tensor Core 活用: the same two steps, without the
+ * A_q round trip).
+ *   X_f16      device fp16 [M, K] row-major, 16-byte aligned.
+ *   workspace  device, at least mixllm_linear_small_m_workspace_bytes() bytes,
+ *              256-byte aligned, zero-filled before its first use; calls
+ *              leave its counters at zero (the rest is scratch); not shared by
+ *              calls that run at the same time.
+ * Other arguments, the M <= 64 bound and the errors: as
+ * mixllm_gemm_w4w8a8_small_m.  Asynchronous on `stream`.
+ */
+MIXLLM_API mixllm_status mixllm_linear_small_m_workspace_bytes(int64_t M, int64_t K, int64_t N4, int64_t N8,
+                                                               size_t *bytes);
+MIXLLM_API mixllm_status mixllm_linear_small_m(const void *X_f16, int64_t M, int64_t K, const uint8_t *W4,
+                                               const uint8_t *z4, const void *s_w4_f16, const int32_t *idx4,
+                                               int64_t N4, const int8_t *W8, const void *s_w8_f16,
+                                               const int32_t *idx8, int64_t N8, void *Y_f16, void *workspace,
+                                               size_t workspace_bytes, void *stream);
+
+/*
  * mixllm_gemm_w4w8a8_small_m without a workspace argument and without any
  * allocation: the split partial sums and tile counters live in a fixed 8 MiB
  * scratch array in the library's static device memory (one per device,

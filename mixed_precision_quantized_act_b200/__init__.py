@@ -18,6 +18,8 @@ from ._lib import (  # noqa: F401
     gemm_w4w8a8_small_m_noalloc_into,
     gemm_w4w8a8_small_m_into,
     linear,
+    linear_small_m_into,
+    linear_small_m_workspace,
     load,
     pack_weights,
     packed_sizes,

@@ -36,6 +36,9 @@ SIGNATURES = {
     "mixllm_small_m_workspace_bytes": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(ctypes.c_size_t)]),
     "mixllm_small_m_kernel": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(ctypes.c_int32)]),
     "mixllm_channel_salience": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i64, _vp, _vp]),
+    "mixllm_linear_small_m_workspace_bytes": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(ctypes.c_size_t)]),
+    "mixllm_linear_small_m": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64,
+                                             _vp, _vp, ctypes.c_size_t, _vp]),
     "mixllm_select_top_t_workspace_bytes": (ctypes.c_int, [_i64, ctypes.POINTER(ctypes.c_size_t)]),
     "mixllm_select_top_t": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, ctypes.c_size_t, _vp]),
     "mixllm_gemm_w4w8a8_small_m": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64,
@@ -219,6 +222,24 @@ def small_m_workspace_bytes(M: int, K: int, N4: int, N8: int) -> int:
     out = ctypes.c_size_t(0)
     _check(load().mixllm_small_m_workspace_bytes(M, K, N4, N8, ctypes.byref(out)), "mixllm_small_m_workspace_bytes")
     return out.value
+
+
+def linear_small_m_workspace(M: int, p: PackedLinear, device) -> torch.Tensor:
+    """A zero-filled workspace for mixllm_linear_small_m (every call leaves
+    its counters at zero, so it can be reused)."""
+    out = ctypes.c_size_t(0)
+    _check(load().mixllm_linear_small_m_workspace_bytes(M, p.K, p.N4, p.N8, ctypes.byref(out)),
+           "mixllm_linear_small_m_workspace_bytes")
+    return torch.zeros(max(256, out.value), dtype=torch.uint8, device=device)
+
+
+def linear_small_m_into(X, p: PackedLinear, Y, workspace: torch.Tensor, stream=None):
+    """The few-token layer from fp16 X, quantization included (mixllm_linear_small_m)."""
+    _need_cuda(X, Y, workspace)
+    M, K = X.shape
+    _check(load().mixllm_linear_small_m(_ptr(X), M, K, _ptr(p.W4), _ptr(p.z4), _ptr(p.s_w4), _ptr(p.idx4), p.N4,
+                                        _ptr(p.W8), _ptr(p.s_w8), _ptr(p.idx8), p.N8, _ptr(Y), _ptr(workspace),
+                                        workspace.numel(), _stream(stream)), "mixllm_linear_small_m")
 
 
 SMALL_M_KERNELS = ("tensor-core split-K", "GEMV split-K", "GEMV persistent")

@@ -626,7 +626,7 @@ static bool encode_w8_groups_3d(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorM
   return true;
 }
 
-template <int MT>
+template <int MT, bool FUSE = false>
 static cudaError_t launch_gemv_mt(const GemmArgs &a, const SmallMPlan &p, void *ws, cudaStream_t stream,
                                   const char **msg) {
   static_assert(gemv_min_blocks(MT) * (gemv_smem_bytes<MT>() + 1024) <= 228 * 1024, "resident CTAs per SM");
@@ -649,7 +649,7 @@ static cudaError_t launch_gemv_mt(const GemmArgs &a, const SmallMPlan &p, void *
     *msg = "too many tiles";
     return cudaErrorInvalidValue;
   }
-  auto kern = gemv_w4w8a8_kernel<MT>;
+  auto kern = gemv_w4w8a8_kernel<MT, FUSE>;
   int dev = 0;
   cudaGetDevice(&dev);
   static unsigned long long configured = 0;  // one bit per device ordinal
@@ -674,7 +674,8 @@ static cudaError_t launch_gemv_mt(const GemmArgs &a, const SmallMPlan &p, void *
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(
-      &cfg, kern, tmW8, a.A_q, a.s_a, a.W4, a.z4, static_cast<const __half *>(a.s_w4), a.idx4,
+      &cfg, kern, tmW8, static_cast<const __half *>(a.X), a.A_q, a.s_a, a.W4, a.z4,
+      static_cast<const __half *>(a.s_w4), a.idx4,
       static_cast<const __half *>(a.s_w8), a.idx8, static_cast<int>(a.M), static_cast<int>(a.K),
       static_cast<int>(a.N4), static_cast<int>(a.N8), static_cast<int>(padded_channels(a.N4)),
       static_cast<int>(padded_channels(a.N8)), p.nt4, tiles, p.splits, p.splits8, static_cast<__half *>(a.Y), ws_part,
@@ -738,6 +739,58 @@ static cudaError_t launch_gemv_persistent_mt(const GemmArgs &a, const SmallMPlan
 
 size_t small_m_workspace_bytes(int64_t M, int64_t N4, int64_t N8, int64_t K) {
   return plan_small_m(M, N4, N8, K).bytes();
+}
+
+// The split GEMV's fused form needs a CTA's slice of X (tokens x groups x
+// 256 bytes) to fit the second 32 KiB ring slot; 4-bit CTAs hold the most
+// groups.  Measured on B200 (the 8B decoder layer's four linears, rotating
+// weights): one token 50.8 -> 46.9 us fused; four and eight tokens 2-3 %
+// slower, each CTA quantizing its slice on the critical path -- so one token only.
+static bool plan_fuses(const SmallMPlan &p) {
+  if (!p.gemv || p.persistent || p.mp != 1) return false;
+  const int ng_max = (p.groups + p.splits - 1) / p.splits;
+  return static_cast<int64_t>(p.mp) * ng_max * 256 <= kGvSlotBytesSplit;
+}
+
+bool linear_small_m_fused(int64_t M, int64_t N4, int64_t N8, int64_t K) {
+  return plan_fuses(plan_small_m(M, N4, N8, K));
+}
+
+static size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+size_t linear_small_m_workspace_bytes(int64_t M, int64_t N4, int64_t N8, int64_t K) {
+  const SmallMPlan p = plan_small_m(M, N4, N8, K);
+  if (plan_fuses(p)) return p.bytes();
+  return round256(p.bytes()) + round256(static_cast<size_t>(M * K)) + static_cast<size_t>(M * (K / 128)) * 4;
+}
+
+cudaError_t launch_linear_small_m(const GemmArgs &a, void *ws, size_t ws_bytes, cudaStream_t stream,
+                                  const char **msg) {
+  const SmallMPlan p = plan_small_m(a.M, a.N4, a.N8, a.K);
+  if (ws_bytes < linear_small_m_workspace_bytes(a.M, a.N4, a.N8, a.K) || (ws_bytes > 0 && !ws)) {
+    *msg = "workspace too small for this shape";
+    return cudaErrorInvalidValue;
+  }
+  if (plan_fuses(p)) {
+    if (p.mp == 1) return launch_gemv_mt<1, true>(a, p, ws, stream, msg);
+    if (p.mp == 2) return launch_gemv_mt<2, true>(a, p, ws, stream, msg);
+    if (p.mp == 4) return launch_gemv_mt<4, true>(a, p, ws, stream, msg);
+    return launch_gemv_mt<8, true>(a, p, ws, stream, msg);
+  }
+  // quantize into the workspace, then the planned kernel
+  GemmArgs q = a;
+  unsigned char *base = static_cast<unsigned char *>(ws);
+  int8_t *A_q = reinterpret_cast<int8_t *>(base + round256(p.bytes()));
+  float *s_a = reinterpret_cast<float *>(base + round256(p.bytes()) + round256(static_cast<size_t>(a.M * a.K)));
+  cudaError_t e = launch_quantize_act(a.X, a.M, a.K, A_q, s_a, stream);
+  if (e != cudaSuccess) {
+    *msg = "launch of the activation quantizer failed";
+    return e;
+  }
+  q.A_q = A_q;
+  q.s_a = s_a;
+  q.X = nullptr;
+  return launch_gemm_small_m(q, ws, p.bytes(), stream, msg);
 }
 
 int small_m_kernel_kind(int64_t M, int64_t N4, int64_t N8, int64_t K) {

@@ -48,10 +48,12 @@
 #include "gemm_w4w8a8.cuh"  // kI2FBias, kI2FBiasBits
 #include "launch.h"
 #include "ptx_sm100.cuh"
+#include "quant.cuh"  // quant_act_8x16
 
 namespace mixllm {
 
 constexpr int kGvThreads = 256;  // 128 channel rows x 2 (even / odd groups)
+constexpr int kGvSlotBytesSplit = 32768;  // the split kernel's slot (its fused form stages X in one)
 
 // Per token bound: the ring (slots x bytes per copy) and the groups a CTA may
 // take (bounds the staged tables), sized so that two CTAs fit on an SM.
@@ -61,7 +63,7 @@ constexpr int kGvThreads = 256;  // 128 channel rows x 2 (even / odd groups)
 template <int MT>
 struct GvCfg {
   static constexpr int kSlots = 2;
-  static constexpr int kSlotBytes = 32768;
+  static constexpr int kSlotBytes = kGvSlotBytesSplit;
   static constexpr int kGroupsMax = 32;
   static constexpr int kChunk4 = kSlotBytes / 8192;   // 4-bit groups per copy (8 KiB each)
   static constexpr int kChunk8 = kSlotBytes / 16384;  // 8-bit groups per copy (16 KiB each)
@@ -187,11 +189,17 @@ __device__ __forceinline__ void gv_group8(const uint8_t *wrow, int r, const int8
 // MT: the token bound of this instantiation (1, 2, 4 or 8), M <= MT.
 // Grid: nt4 4-bit tiles x S4 splits, then nt8 8-bit tiles x S8 splits; split
 // s of S takes groups [s*G/S, (s+1)*G/S), 1 to GvCfg<MT>::kGroupsMax of them.
+// FUSE: the activations come in as fp16 X [M, K] and each CTA quantizes the
+// slice it needs itself (the same quantizer as quantize_act_kernel, so the
+// same codes): its slice of X is bulk-copied into the second ring slot while
+// the first weight chunk streams into the first (the host launches this form
+// only when the slice fits in a slot), then the slot is refilled with weights.
 // tmW8: the 8-bit weights as a 3-D tensor (k within a group, row, group)
 // with boxes of GvCfg<MT>::kChunk8 groups.
-template <int MT>
+template <int MT, bool FUSE>
 __global__ void __launch_bounds__(kGvThreads, gemv_min_blocks(MT))
-    gemv_w4w8a8_kernel(const __grid_constant__ CUtensorMap tmW8, const int8_t *__restrict__ A_q,
+    gemv_w4w8a8_kernel(const __grid_constant__ CUtensorMap tmW8, const __half *__restrict__ X,
+                       const int8_t *__restrict__ A_q,
                        const float *__restrict__ s_a, const uint8_t *__restrict__ W4, const uint8_t *__restrict__ z4,
                        const __half *__restrict__ s_w4, const int32_t *__restrict__ idx4,
                        const __half *__restrict__ s_w8, const int32_t *__restrict__ idx8, int M, int K, int N4,
@@ -253,9 +261,18 @@ __global__ void __launch_bounds__(kGvThreads, gemv_min_blocks(MT))
   const int mt = M < MT ? M : MT;
   // s_a rows as bulk copies too when they are 16-byte pieces (the CTAs of a
   // split read the same few lines: one request per token instead of a warp's loads)
-  const bool sa_bulk = ((g0 | ng | G) & 3) == 0 && (reinterpret_cast<uintptr_t>(s_a) & 15) == 0;
+  const bool sa_bulk = !FUSE && ((g0 | ng | G) & 3) == 0 && (reinterpret_cast<uintptr_t>(s_a) & 15) == 0;
   int issued = 0;
-  if (threadIdx.x == 0) {
+  if (FUSE && threadIdx.x == 0) {
+    // the tokens' fp16 activations of groups [g0, g1) into the second slot, one
+    // bulk copy per token, and the first weight chunk into the first
+    mbar_arrive_expect_tx(&S.a_full, static_cast<uint32_t>(mt * ng * 256));
+    for (int m = 0; m < mt; ++m)
+      bulk_load(ring + kGvSlotBytes + m * ng * 256, X + static_cast<int64_t>(m) * K + g0 * 128,
+                static_cast<uint32_t>(ng * 256), &S.a_full);
+    issue(issued++);
+  }
+  if (!FUSE && threadIdx.x == 0) {
     // the tokens' codes (and scales) of groups [g0, g1): one bulk copy per token, first
     mbar_arrive_expect_tx(&S.a_full, static_cast<uint32_t>(mt * ng * (128 + (sa_bulk ? 4 : 0))));
     for (int m = 0; m < mt; ++m) {
@@ -273,7 +290,12 @@ __global__ void __launch_bounds__(kGvThreads, gemv_min_blocks(MT))
       *reinterpret_cast<int4 *>(&S.a[mt + e / (ng * 8)][(e % (ng * 8)) * 16]) = make_int4(0, 0, 0, 0);
     for (int e = threadIdx.x; e < MT * ng; e += kGvThreads) {
       const int m = e / ng, i = e - m * ng;
-      if (m >= mt || !sa_bulk) S.sa[m][i] = m < M ? s_a[static_cast<int64_t>(m) * G + g0 + i] : 0.0f;
+      if (m >= mt) {
+        S.sa[m][i] = 0.0f;
+        if (FUSE) S.asum[m][i] = 0;
+      } else if (!FUSE && !sa_bulk) {
+        S.sa[m][i] = s_a[static_cast<int64_t>(m) * G + g0 + i];
+      }
     }
     const __half *swp = is4 ? s_w4 + static_cast<int64_t>(g0) * N4p + n0 : s_w8 + static_cast<int64_t>(g0) * N8p + n0;
     const int64_t sws = is4 ? N4p : N8p;
@@ -288,26 +310,48 @@ __global__ void __launch_bounds__(kGvThreads, gemv_min_blocks(MT))
             *reinterpret_cast<const uint4 *>(z4 + static_cast<int64_t>(g0 + i) * (N4p >> 1) + (n0 >> 1) + q * 16);
       }
     }
-    // the sum of each (token, group)'s 128 codes, once they have landed:
-    // 8 threads per (token, group), one 16-byte piece each
-    (void)warp_wait(&S.a_full, 0, &S.abort_flag);
-    const int pieces = MT * ng * 8;
-    for (int e0 = 0; e0 < pieces; e0 += kGvThreads) {  // the same trip count in every thread
-      const int e = e0 + static_cast<int>(threadIdx.x);
-      const bool ok = e < pieces;
-      const int m = ok ? (e >> 3) / ng : 0, i = ok ? (e >> 3) - m * ng : 0;
-      const int4 v = ok ? lds_i4(&S.a[m][i * 128 + (e & 7) * 16]) : make_int4(0, 0, 0, 0);
-      int sum = __dp4a(v.x, 0x01010101, 0);
-      sum = __dp4a(v.y, 0x01010101, sum);
-      sum = __dp4a(v.z, 0x01010101, sum);
-      sum = __dp4a(v.w, 0x01010101, sum);
-      sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
-      sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
-      sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 4);
-      if (ok && (e & 7) == 0) S.asum[m][i] = sum;
+    if (FUSE) {
+      // quantize: a half warp per (token, group), eight activations per lane
+      (void)warp_wait(&S.a_full, 0, &S.abort_flag);
+      const int lane16 = threadIdx.x & 15, hw = threadIdx.x >> 4;
+      const unsigned mask = 0xFFFFu << (threadIdx.x & 16);
+      for (int pr = hw; pr < mt * ng; pr += kGvThreads / 16) {  // uniform within a half warp (its shuffle mask)
+        const int m = pr / ng, i = pr - m * ng;
+        const uint4 raw = lds_u4(ring + kGvSlotBytes + pr * 256 + lane16 * 16);
+        uint32_t packed[2];
+        const float sa = quant_act_8x16(raw, mask, packed);
+        *reinterpret_cast<uint2 *>(&S.a[m][i * 128 + lane16 * 8]) = make_uint2(packed[0], packed[1]);
+        int sum = __dp4a(static_cast<int>(packed[0]), 0x01010101, __dp4a(static_cast<int>(packed[1]), 0x01010101, 0));
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(mask, sum, o);
+        if (lane16 == 0) {
+          S.sa[m][i] = sa;
+          S.asum[m][i] = sum;
+        }
+      }
+    } else {
+      // the sum of each (token, group)'s 128 codes, once they have landed:
+      // 8 threads per (token, group), one 16-byte piece each
+      (void)warp_wait(&S.a_full, 0, &S.abort_flag);
+      const int pieces = MT * ng * 8;
+      for (int e0 = 0; e0 < pieces; e0 += kGvThreads) {  // the same trip count in every thread
+        const int e = e0 + static_cast<int>(threadIdx.x);
+        const bool ok = e < pieces;
+        const int m = ok ? (e >> 3) / ng : 0, i = ok ? (e >> 3) - m * ng : 0;
+        const int4 v = ok ? lds_i4(&S.a[m][i * 128 + (e & 7) * 16]) : make_int4(0, 0, 0, 0);
+        int sum = __dp4a(v.x, 0x01010101, 0);
+        sum = __dp4a(v.y, 0x01010101, sum);
+        sum = __dp4a(v.z, 0x01010101, sum);
+        sum = __dp4a(v.w, 0x01010101, sum);
+        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
+        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
+        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 4);
+        if (ok && (e & 7) == 0) S.asum[m][i] = sum;
+      }
     }
   }
   __syncthreads();
+  if (FUSE && threadIdx.x == 0 && issued < nch) issue(issued++);  // the second slot is free again
 
   // 4-bit: rows rp and rp + 64, group j4 of every chunk; 8-bit: row r8, group j8
   const int rp = threadIdx.x & 63, j4 = threadIdx.x >> 6;

@@ -33,6 +33,7 @@ struct GemmArgs {
   int64_t N8;
   void *Y;     // fp16 [M, N4 + N8]
   int32_t *P;  // debug partials [M, N, G] or null
+  const void *X = nullptr;  // fp16 [M, K] activations: the fused few-token path quantizes them itself
 };
 
 // Returns a CUDA error, or cudaErrorNotSupported when the tensor-map encoder
@@ -47,6 +48,14 @@ cudaError_t launch_gemm_small_m(const GemmArgs &a, void *ws, size_t ws_bytes, cu
 size_t small_m_workspace_bytes(int64_t M, int64_t N4, int64_t N8, int64_t K);
 // 0: tensor-core kernel, 1: split GEMV, 2: persistent GEMV (mixllm_small_m_kind)
 int small_m_kernel_kind(int64_t M, int64_t N4, int64_t N8, int64_t K);
+// The few-token layer from fp16 X (quantization included): the split GEMV
+// quantizes in its prologue when its slice of X fits a ring slot; otherwise
+// the quantizer writes A_q / s_a into the workspace first.  a.X is required,
+// a.A_q / a.s_a are ignored.  Workspace: linear_small_m_workspace_bytes().
+size_t linear_small_m_workspace_bytes(int64_t M, int64_t N4, int64_t N8, int64_t K);
+bool linear_small_m_fused(int64_t M, int64_t N4, int64_t N8, int64_t K);
+cudaError_t launch_linear_small_m(const GemmArgs &a, void *ws, size_t ws_bytes, cudaStream_t stream,
+                                  const char **msg);
 // The same with a static device scratch instead of a workspace (no allocation);
 // fails with cudaErrorInvalidValue when the shape needs more than it holds.
 cudaError_t launch_gemm_small_m_noalloc(const GemmArgs &a, cudaStream_t stream, const char **msg);

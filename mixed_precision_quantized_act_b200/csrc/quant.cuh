@@ -39,6 +39,48 @@ namespace mixllm {
 //     operands' last places, below 2^13 of them): |e| < s/2 keeps q0, |e| >
 //     s/2 moves q0 one step toward e, |e| = s/2 is a tie and picks the even one.
 // ---------------------------------------------------------------------------
+// One group of 128 activations held eight per lane by the 16 lanes of `mask`
+// (MLSys 2026 talk notes on MixLLM, notes.yuuk.io, §設計判断の概要: 8-bit
+// symmetric, group-wise RTN): s_a = bf16(amax / 127) (IEEE division), codes
+// rne(x / s_a) clamped to +-127 (an all-zero group gives s_a = 0 and zero
+// codes).  x / s_a is rounded exactly: q0 = rint(x * (1/s)), e = fma(-q0, s, x)
+// is exact (x fp16, s bf16), and q0 moves by one when |e| > s/2 (or = s/2
+// with q0 odd), which is rne(fl(x / s)) for these operands.  `raw`: the
+// lane's eight fp16 values; the codes are returned packed, lowest k first;
+// returns s_a.  Shared by quantize_act_kernel and the fused decode GEMV.
+__device__ __forceinline__ float quant_act_8x16(const uint4 raw, unsigned mask, uint32_t (&packed)[2]) {
+  const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw);
+  float x[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(h2[i]);
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(mask, amax, o));
+  const float s = __bfloat162float(__float2bfloat16_rn(__fdiv_rn(amax, 127.0f)));
+  packed[0] = packed[1] = 0u;
+  if (s != 0.0f) {
+    const float r = __frcp_rn(s);
+    const float half_s = 0.5f * s;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int q0 = __float2int_rn(x[i] * r);
+      const float e = __fmaf_rn(-static_cast<float>(q0), s, x[i]);  // exact remainder x - q0*s
+      const float ae = fabsf(e);
+      int qi = q0;
+      if (ae > half_s || (ae == half_s && (q0 & 1))) qi += e > 0.0f ? 1 : -1;
+      qi = max(-127, min(127, qi));
+      packed[i >> 2] |= (static_cast<uint32_t>(qi) & 0xFFu) << ((i & 3) * 8);
+    }
+  }
+  return s;
+}
+
 __global__ void __launch_bounds__(256) quantize_act_kernel(const __half *__restrict__ X, int64_t M, int64_t K,
                                                            int8_t *__restrict__ A_q, float *__restrict__ s_a) {
   // the GEMM that consumes A_q and s_a may start its prologue now; it reads
@@ -53,35 +95,8 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const __half *__restr
     const int64_t m = hw / G, g = hw - m * G;
     const int64_t off = m * K + (g << 7) + lane16 * 8;
     const uint4 raw = *reinterpret_cast<const uint4 *>(X + off);
-    const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw);
-    float x[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __half22float2(h2[i]);
-      x[2 * i] = f.x;
-      x[2 * i + 1] = f.y;
-    }
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(mask, amax, o));
-    const float s = __bfloat162float(__float2bfloat16_rn(__fdiv_rn(amax, 127.0f)));
-    uint32_t packed[2] = {0u, 0u};
-    if (s != 0.0f) {
-      const float r = __frcp_rn(s);
-      const float half_s = 0.5f * s;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int q0 = __float2int_rn(x[i] * r);
-        const float e = __fmaf_rn(-static_cast<float>(q0), s, x[i]);  // exact remainder x - q0*s
-        const float ae = fabsf(e);
-        int qi = q0;
-        if (ae > half_s || (ae == half_s && (q0 & 1))) qi += e > 0.0f ? 1 : -1;
-        qi = max(-127, min(127, qi));
-        packed[i >> 2] |= (static_cast<uint32_t>(qi) & 0xFFu) << ((i & 3) * 8);
-      }
-    }
+    uint32_t packed[2];
+    const float s = quant_act_8x16(raw, mask, packed);
     *reinterpret_cast<uint2 *>(A_q + off) = make_uint2(packed[0], packed[1]);
     if (lane16 == 0) s_a[m * G + g] = s;
   }

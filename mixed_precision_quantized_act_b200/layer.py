@@ -9,9 +9,11 @@ linear reads its own input buffer.
 
 `LinearChain` holds the packed weights and every intermediate buffer of such
 a chain, runs it eagerly, and captures it once into a CUDA graph so that a
-replay issues all eight kernels with one launch from the host (the few-token
-path is used for M <= 64).  Buffers are allocated once, at construction; a
-replay allocates nothing.
+replay issues all of its kernels with one launch from the host.  For M <= 64
+each linear is one mixllm_linear_small_m call (by default; fused=False keeps
+quantize_act and the few-token GEMM as two calls): where the plan allows, the
+GEMV quantizes its own slice of X and the layer is a single kernel.  Buffers
+are allocated once, at construction; a replay allocates nothing.
 """
 from dataclasses import dataclass
 from typing import List, Optional
@@ -29,13 +31,15 @@ class _Stage:
     s_a: torch.Tensor    # fp32 [M, K/128]
     Y: torch.Tensor      # fp16 [M, N] output
     ws: Optional[torch.Tensor]  # few-token workspace, or None
+    lws: Optional[torch.Tensor]  # workspace of the fused few-token layer, or None
 
 
 class LinearChain:
     """A fixed sequence of W4.4A8 linears over one batch of M tokens."""
 
-    def __init__(self, packed: List[_lib.PackedLinear], M: int, device):
+    def __init__(self, packed: List[_lib.PackedLinear], M: int, device, fused: bool = True):
         self.M = M
+        self.fused = fused
         self.device = torch.device(device)
         self.stages: List[_Stage] = []
         for p in packed:
@@ -43,8 +47,10 @@ class LinearChain:
             A_q = torch.empty((M, p.K), dtype=torch.int8, device=self.device)
             s_a = torch.empty((M, p.K // _lib.GROUP), dtype=torch.float32, device=self.device)
             Y = torch.empty((M, p.N), dtype=torch.float16, device=self.device)
-            ws = _lib.small_m_workspace(M, p, self.device) if 0 < M <= _lib.SMALL_M_MAX else None
-            self.stages.append(_Stage(p, X, A_q, s_a, Y, ws))
+            small = 0 < M <= _lib.SMALL_M_MAX
+            ws = _lib.small_m_workspace(M, p, self.device) if small else None
+            lws = _lib.linear_small_m_workspace(M, p, self.device) if small and fused else None
+            self.stages.append(_Stage(p, X, A_q, s_a, Y, ws, lws))
         self.graph: Optional[torch.cuda.CUDAGraph] = None
 
     @property
@@ -55,12 +61,26 @@ class LinearChain:
     def outputs(self) -> List[torch.Tensor]:
         return [s.Y for s in self.stages]
 
+    def launches(self) -> int:
+        """Kernels one run issues: one per linear whose GEMV quantizes its own
+        activations (the fused workspace is no larger than the GEMM's alone),
+        two otherwise."""
+        n = 0
+        for s in self.stages:
+            fused = s.lws is not None and s.lws.numel() == max(
+                256, _lib.small_m_workspace_bytes(self.M, s.p.K, s.p.N4, s.p.N8))
+            n += 1 if fused else 2
+        return n
+
     def ops(self) -> int:
         return sum(2 * self.M * s.p.N * s.p.K for s in self.stages)
 
     def run(self, stream=None):
         """Every stage, eagerly, on `stream` (default: the current stream)."""
         for s in self.stages:
+            if s.lws is not None:
+                _lib.linear_small_m_into(s.X, s.p, s.Y, s.lws, stream)
+                continue
             _lib.quantize_act_into(s.X, s.A_q, s.s_a, stream)
             if s.ws is not None:
                 _lib.gemm_w4w8a8_small_m_into(s.A_q, s.s_a, s.p, s.Y, s.ws, stream)
