@@ -459,8 +459,10 @@ LAYER_WORKLOAD = "llama3.1-8b_layer"  # the four linears of one decoder layer, "
 
 def run_layer(args, rank, world, local_rank):
     """The decoder layer's four linears (qkv, o_proj, gate_up, down), each as
-    quantize + GEMM, replayed as one CUDA graph per step; L2 flushed before
-    each step, outside the graph.  Reports TOPS over the four GEMMs."""
+    quantize + GEMM (or, for one token, the GEMV quantizing its own input).
+    M > 64: one CUDA graph per step, L2 flushed before each step outside the
+    graph.  M <= 64: the K steps as one CUDA graph over weight sets larger
+    than L2 together.  Reports TOPS over the four GEMMs."""
     import torch
     import mixed_precision_quantized_act_b200 as mx
     from mixed_precision_quantized_act_b200.layer import LinearChain
@@ -472,30 +474,69 @@ def run_layer(args, rank, world, local_rank):
     layers = [l.with_m(M) for l in wl.LLAMA8B_LAYER]
     packed = [mx.pack_weights(torch.from_numpy(wl.make_w(l, args.seed)).to(dev),
                               torch.from_numpy(wl.make_bitmap(l, args.seed)).to(dev)) for l in layers]
-    chain = LinearChain(packed, M, dev)
-    for l, x in zip(layers, chain.inputs):
-        x.copy_(torch.from_numpy(wl.make_x(l, dp.batch_seed(args.seed, rank))))
-    chain.capture()
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-    for _ in range(max(args.warmup, 3)):
-        flush.fill_(1)
-        chain.replay()
-    mx.sync_status(stream)
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clocks:
-        for i in range(K):
-            flush.fill_(i & 0xFF)
-            ev[i][0].record(stream)
-            chain.replay()
-            ev[i][1].record(stream)
+    if M <= mx.SMALL_M_MAX:
+        # decode: rotate over weight sets larger than L2 together, K steps as one CUDA graph
+        wbytes = sum(p.nbytes() for p in packed)
+        ncopy = max(2, -(-ROTATE_BYTES // wbytes))
+        sets = [packed] + [[mx.PackedLinear(**{k: (v.clone() if isinstance(v, torch.Tensor) else v)
+                                               for k, v in vars(p).items()}) for p in packed]
+                           for _ in range(ncopy - 1)]
+        chains = [LinearChain(ps, M, dev) for ps in sets]
+        for c in chains:
+            for l, x in zip(layers, c.inputs):
+                x.copy_(torch.from_numpy(wl.make_x(l, dp.batch_seed(args.seed, rank))))
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            for i in range(max(args.warmup, 3)):
+                chains[i % ncopy].run()
+        stream.wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            for i in range(K):
+                chains[i % ncopy].run()
+        g.replay()
+        mx.sync_status(stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
         torch.cuda.synchronize()
-    barrier(world)
-    mx.sync_status(stream)
-    t_step = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / K, world)
+        with ClockSampler(local_rank) as clocks:
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+        barrier(world)
+        mx.sync_status(stream)
+        t_step = max_over_ranks(e0.elapsed_time(e1) / K, world)
+        del g
+        chain = chains[0]
+        l2 = f"inputs larger than L2: {ncopy} sets of the layer's packed weights, step i uses set i mod {ncopy}"
+    else:
+        chain = LinearChain(packed, M, dev)
+        for l, x in zip(layers, chain.inputs):
+            x.copy_(torch.from_numpy(wl.make_x(l, dp.batch_seed(args.seed, rank))))
+        chain.capture()
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        for _ in range(max(args.warmup, 3)):
+            flush.fill_(1)
+            chain.replay()
+        mx.sync_status(stream)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        barrier(world)
+        torch.cuda.synchronize()
+        with ClockSampler(local_rank) as clocks:
+            for i in range(K):
+                flush.fill_(i & 0xFF)
+                ev[i][0].record(stream)
+                chain.replay()
+                ev[i][1].record(stream)
+            torch.cuda.synchronize()
+        barrier(world)
+        mx.sync_status(stream)
+        t_step = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / K, world)
+        l2 = "flushed by a 256 MiB device write before every timed step"
     chain.release()
     ops = chain.ops()
     if rank != 0:
@@ -507,7 +548,7 @@ def run_layer(args, rank, world, local_rank):
         "vs_baseline": None, "dtype": "int8",
         "data": "synthetic (seeded N(0,1) X with x20 outlier columns, N(0,0.02) W, random 8-bit channel sets)",
         "config": {"workload": f"{LAYER_WORKLOAD}@M{M}", "M": M, "linears": [l.name.split("_M")[0] for l in layers],
-                   "l2": "flushed by a 256 MiB device write before every timed step",
+                   "l2": l2,
                    "parallelism": f"dp{world} (weights replicated, M tokens per GPU)"},
         "step": f"{chain.launches()} kernels (each linear: quantize_act + the GEMM, or for one token the GEMV "
                 "quantizing its own activations) replayed as one CUDA graph",
