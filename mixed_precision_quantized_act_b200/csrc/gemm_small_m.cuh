@@ -54,10 +54,14 @@ constexpr int kSmGroupsMax = 32;  // groups per CTA (bounds the scale tables)
 template <int MP>
 struct SmallMCfg {
   static_assert(MP == 16 || MP == 32 || MP == 64, "token tile");
-  // The ring holds as many stages as fit (all of a CTA's groups when they
-  // fit, so one round of loads covers the whole K range): a stage is the
-  // weight tile (int8 16 KB, or packed 4-bit 8 KB) followed by the token tile.
+  // The ring holds stages of several groups each (four 4-bit groups, or two
+  // 8-bit ones: 32 KiB of weights), loaded with one copy per operand: a CTA's
+  // copy rate grows with the bytes per copy, so per-group copies of 8 KiB
+  // would bound it far below HBM speed.  A stage is the chunk's weights, then
+  // its token tiles (one 3-D box, group after group).
   static constexpr int kRingBytes = 128 * 1024;
+  static constexpr int kGpc4 = 4, kGpc8 = 2;                // groups per chunk
+  static constexpr int kChunkWBytes = 32768;
   static constexpr int kMaxStages = 16;
   // Unpacked 4-bit tiles: buffer i % kTBufs is free again only when the MMAs
   // of group i - kTBufs have completed (~800 cycles after their commit), so
@@ -74,7 +78,7 @@ struct SmallMCfg {
   static constexpr int kOffStages = 0;
   static constexpr int kOffTBuf = kOffStages + kRingBytes;
   static constexpr int kOffZ = kOffTBuf + kTBufs * kWBytes;
-  static constexpr int kOffSw = kOffZ + kMaxStages * 64;               // fp16 s_w [groups][128]
+  static constexpr int kOffSw = kOffZ + kMaxStages * kGpc4 * 64;      // fp16 s_w [groups][128]
   static constexpr int kOffSa = kOffSw + kSmGroupsMax * 128 * 4;       // fp32 s_a [groups][MP]
   static constexpr int kOffBar = kOffSa + kSmGroupsMax * MP * 4;
   static constexpr int kNumBars = kMaxStages + kDone + kTBufs + kAccBufs + 3;  // + table ready, 2 drains
@@ -86,7 +90,7 @@ struct SmallMCfg {
   static constexpr int kSmemBytes = kOffMisc + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;
   static_assert(kXBytes % 1024 == 0 && kRingBytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
-  static_assert(kWBytes + kXBytes <= kRingBytes, "one stage must fit");
+  static_assert(2 * (kChunkWBytes + kGpc4 * kXBytes) <= kRingBytes, "two stages must fit");
   static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
 };
 
@@ -151,7 +155,8 @@ __device__ __forceinline__ void sm_reg_fence(uint32_t (&r)[MP]) {
 template <int MP>
 __global__ void __launch_bounds__(kSmThreads, 1)
     gemm_small_m_kernel(const __grid_constant__ CUtensorMap tmX, const uint8_t *__restrict__ W4,
-                        const __grid_constant__ CUtensorMap tmW8, const float *__restrict__ s_a,
+                        const __grid_constant__ CUtensorMap tmW8, const __grid_constant__ CUtensorMap tmZ,
+                        const float *__restrict__ s_a,
                         const uint8_t *__restrict__ z4, const __half *__restrict__ s_w4,
                         const int32_t *__restrict__ idx4, const __half *__restrict__ s_w8,
                         const int32_t *__restrict__ idx8, int M, int K, int N4, int N8, int N4p, int N8p, int nt4,
@@ -187,32 +192,41 @@ __global__ void __launch_bounds__(kSmThreads, 1)
   const __half *s_w = is4 ? s_w4 : s_w8;
   const int32_t *idx = is4 ? idx4 : idx8;
 
-  // stage = weight tile (packed 4-bit or int8) + token tile; as many as fit
-  const int wbytes = is4 ? C::kW4Bytes : C::kWBytes;
-  const int stage_sz = wbytes + C::kXBytes;  // a multiple of 1024
+  // stage = one chunk: its weights (32 KiB), then the token tiles of four
+  // groups (one box of the token tensor map serves both sets; an 8-bit chunk
+  // of two groups leaves two of them unread); as many stages as fit, even
+  const int gpc = is4 ? C::kGpc4 : C::kGpc8;
+  const int nch = (ng + gpc - 1) / gpc;
+  const int stage_sz = C::kChunkWBytes + C::kGpc4 * C::kXBytes;  // a multiple of 1024
   int nst = C::kRingBytes / stage_sz < C::kMaxStages ? C::kRingBytes / stage_sz : C::kMaxStages;
-  nst &= ~1;  // even: every stage belongs to one MMA issuer
+  nst &= ~1;  // even
   auto stage_w = [&](int s) { return smem + C::kOffStages + s * stage_sz; };
-  auto stage_x = [&](int s) { return smem + C::kOffStages + s * stage_sz + wbytes; };
+  auto stage_x = [&](int s) { return smem + C::kOffStages + s * stage_sz + C::kChunkWBytes; };
   auto tbuf = [&](int b) { return smem + C::kOffTBuf + b * C::kWBytes; };
-  auto zmeta = [&](int s) { return smem + C::kOffZ + s * 64; };
-  const uint32_t stage_bytes = static_cast<uint32_t>(C::kXBytes + (is4 ? C::kW4Bytes + 64 : C::kWBytes));
-  auto load = [&](int i) {  // local group i of this CTA into stage i % nst
-    const int s = i % nst, g = g0 + i;
-    mbar_arrive_expect_tx(&full[s], stage_bytes);
-    tma_load_2d(stage_x(s), &tmX, &full[s], g * 128, 0);
+  auto zmeta = [&](int s) { return smem + C::kOffZ + s * C::kGpc4 * 64; };
+  // where local group i lives: its chunk's stage, its offset in the chunk, the phase of the stage
+  auto gstage = [&](int i) { return (i / gpc) % nst; };
+  auto gphase = [&](int i) { return static_cast<uint32_t>(((i / gpc) / nst) & 1); };
+  auto load = [&](int c) {  // chunk c (local groups c*gpc ..) into stage c % nst
+    const int s = c % nst, i0 = c * gpc, g = g0 + i0;
+    const int n = min(gpc, ng - i0);
+    // boxes always land whole (groups past the CTA's last come from the next
+    // split or are zero past K; tokens past M are zero) and are never read
+    const uint32_t wb = is4 ? static_cast<uint32_t>(n) * C::kW4Bytes : static_cast<uint32_t>(C::kChunkWBytes);
+    mbar_arrive_expect_tx(&full[s], wb + static_cast<uint32_t>(C::kGpc4 * C::kXBytes) + (is4 ? C::kGpc4 * 64u : 0u));
+    tma_load_3d(stage_x(s), &tmX, &full[s], 0, 0, g);
     if (is4) {
-      // the tile's packed group is one contiguous 8 KB block: one bulk copy
-      bulk_load(stage_w(s), W4 + (static_cast<int64_t>(n0 >> 7) * G + g) * C::kW4Bytes, C::kW4Bytes, &full[s]);
-      bulk_load(zmeta(s), z4 + static_cast<int64_t>(g) * (N4p >> 1) + (n0 >> 1), 64, &full[s]);
+      // the tile's packed groups are contiguous 8 KB blocks: one bulk copy
+      bulk_load(stage_w(s), W4 + (static_cast<int64_t>(n0 >> 7) * G + g) * C::kW4Bytes, wb, &full[s]);
+      tma_load_2d(zmeta(s), &tmZ, &full[s], n0 >> 1, g);
     } else {
-      tma_load_2d(stage_w(s), &tmW8, &full[s], g * 128, n0);
+      tma_load_3d(stage_w(s), &tmW8, &full[s], 0, n0, g);
     }
   };
 
   if (threadIdx.x == 0) {
     prefetch_tmap(&tmX);
-    if (!is4) prefetch_tmap(&tmW8);
+    prefetch_tmap(is4 ? &tmZ : &tmW8);
     for (int s = 0; s < C::kMaxStages; ++s) mbar_init(&full[s], 1);
     for (int i = 0; i < C::kDone; ++i) mbar_init(&done[i], 1);
     for (int b = 0; b < C::kTBufs; ++b) mbar_init(&tfull[b], kSmUnpackWarps);
@@ -241,16 +255,21 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       // every global read of this grid comes after this wait (here, in the
       // scale warp, or in roles ordered after these loads by barriers)
       pdl_wait();
-      int issued = ng < nst ? ng : nst;
-      for (int i = 0; i < issued; ++i) load(i);
-      for (int i = nst; i < ng; ++i) {
-        const int ip = i - nst;  // the stage last held local group ip
-        if (!mbar_wait(&done[ip % C::kDone], (ip / C::kDone) & 1, abort_flag)) break;
-        load(i);
-        issued = i + 1;
+      int issued = nch < nst ? nch : nst;
+      for (int c = 0; c < issued; ++c) load(c);
+      for (int c = nst; c < nch; ++c) {
+        // the stage last held chunk c - nst: free once both issuers' MMAs of it are done
+        // (each issuer commits in its own order; there is none between the two)
+        const int cp = c - nst;
+        const int last = cp * gpc + gpc - 1;  // a full chunk: its last even and last odd group
+        bool ok = mbar_wait(&done[last % C::kDone], (last / C::kDone) & 1, abort_flag);
+        ok = ok && mbar_wait(&done[(last - 1) % C::kDone], ((last - 1) / C::kDone) & 1, abort_flag);
+        if (!ok) break;
+        load(c);
+        issued = c + 1;
       }
-      for (int i = (issued > nst ? issued - nst : 0); i < issued; ++i)
-        (void)mbar_wait_drain(&full[i % nst], (i / nst) & 1, 1ll << 26);
+      for (int c = (issued > nst ? issued - nst : 0); c < issued; ++c)
+        (void)mbar_wait_drain(&full[c % nst], (c / nst) & 1, 1ll << 26);
     }
   } else if (warp == 1 || warp == 3) {
     // ------------------------------------------------------------ MMA issuers
@@ -260,14 +279,14 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       constexpr uint32_t idesc = idesc_i8(128, MP);
       const int who = warp == 1 ? 0 : 1;
       for (int i = who; i < ng; i += 2) {
-        const int s = i % nst, b = i % C::kTBufs, a = i % C::kAccBufs;
-        if (!mbar_wait(&full[s], (i / nst) & 1, abort_flag)) break;
+        const int s = gstage(i), j = i % gpc, b = i % C::kTBufs, a = i % C::kAccBufs;
+        if (!mbar_wait(&full[s], gphase(i), abort_flag)) break;
         if (is4 && !mbar_wait(&tfull[b], (i / C::kTBufs) & 1, abort_flag)) break;
         // phase 0 of accempty[a] is the epilogue's bias fill, phase u+1 its drain of use u
         if (!mbar_wait(&accempty[a], (i / C::kAccBufs) & 1, abort_flag)) break;
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(is4 ? tbuf(b) : stage_w(s));  // weights: 128 channels x 128 k
-        const uint32_t b_addr = smem_u32(stage_x(s));                   // tokens: MP rows x 128 k
+        const uint32_t a_addr = smem_u32(is4 ? tbuf(b) : stage_w(s) + j * C::kWBytes);  // weights: 128 channels x 128 k
+        const uint32_t b_addr = smem_u32(stage_x(s) + j * C::kXBytes);                   // tokens: MP rows x 128 k
         const uint32_t d = tmem_base + static_cast<uint32_t>(a * MP);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
@@ -307,14 +326,14 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       const int zshift = (r0 & 1) * 4;
       const int sw = r0 & 7;
       for (int i = 0; i < ng; ++i) {
-        const int s = i % nst, b = i % C::kTBufs;
-        if (!warp_wait(&full[s], (i / nst) & 1, abort_flag)) break;
+        const int s = gstage(i), j = i % gpc, b = i % C::kTBufs;
+        if (!warp_wait(&full[s], gphase(i), abort_flag)) break;
         if (i >= C::kTBufs) {  // buffer b last held local group i - kTBufs
           const int ip = i - C::kTBufs;
           if (!warp_wait(&done[ip % C::kDone], (ip / C::kDone) & 1, abort_flag)) break;
         }
-        const uint8_t *raw = stage_w(s);
-        const uint8_t *zb = zmeta(s);
+        const uint8_t *raw = stage_w(s) + j * C::kW4Bytes;
+        const uint8_t *zb = zmeta(s) + j * 64;
         uint8_t *dst = tbuf(b);
         uint4 x[2];
         uint32_t zz[2];
@@ -532,6 +551,9 @@ SmallMPlan plan_small_m(int64_t M, int64_t N4, int64_t N8, int64_t K) {
   return p;
 }
 
+static bool encode_groups_3d(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *map, const void *W8, int64_t K,
+                             int64_t N8, int box_rows, int groups_per_box);
+
 template <int MP>
 static cudaError_t launch_small_m_mp(const GemmArgs &a, const SmallMPlan &p, void *ws, cudaStream_t stream,
                                      const char **msg) {
@@ -541,15 +563,21 @@ static cudaError_t launch_small_m_mp(const GemmArgs &a, const SmallMPlan &p, voi
     *msg = "cuTensorMapEncodeTiled is not available from the driver";
     return cudaErrorNotSupported;
   }
-  CUtensorMap tmX, tmW8;
+  CUtensorMap tmX, tmW8, tmZ;
   memset(&tmX, 0, sizeof(tmX));
   memset(&tmW8, 0, sizeof(tmW8));
-  if (!encode_2d_u8(enc, &tmX, a.A_q, a.K, a.M, 128, MP, true)) {
+  memset(&tmZ, 0, sizeof(tmZ));
+  // token tiles of four groups, 8-bit weights of two, zero points of four groups (one box each)
+  if (!encode_groups_3d(enc, &tmX, a.A_q, a.K, a.M, MP, C::kGpc4)) {
     *msg = "tensor map encoding of A_q failed";
     return cudaErrorInvalidValue;
   }
-  if (a.N8 > 0 && !encode_2d_u8(enc, &tmW8, a.W8, a.K, a.N8, 128, 128, true)) {
+  if (a.N8 > 0 && !encode_groups_3d(enc, &tmW8, a.W8, a.K, a.N8, 128, C::kGpc8)) {
     *msg = "tensor map encoding of W8 failed";
+    return cudaErrorInvalidValue;
+  }
+  if (a.N4 > 0 && !encode_2d_u8(enc, &tmZ, a.z4, padded_channels(a.N4) / 2, a.K / 128, 64, C::kGpc4, false)) {
+    *msg = "tensor map encoding of z4 failed";
     return cudaErrorInvalidValue;
   }
   const int tiles = p.nt4 + p.nt8;
@@ -583,7 +611,7 @@ static cudaError_t launch_small_m_mp(const GemmArgs &a, const SmallMPlan &p, voi
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(
-      &cfg, kern, tmX, a.W4, tmW8, a.s_a, a.z4, static_cast<const __half *>(a.s_w4), a.idx4,
+      &cfg, kern, tmX, a.W4, tmW8, tmZ, a.s_a, a.z4, static_cast<const __half *>(a.s_w4), a.idx4,
       static_cast<const __half *>(a.s_w8), a.idx8, static_cast<int>(a.M), static_cast<int>(a.K),
       static_cast<int>(a.N4), static_cast<int>(a.N8), static_cast<int>(padded_channels(a.N4)),
       static_cast<int>(padded_channels(a.N8)), p.nt4, tiles, p.splits, static_cast<__half *>(a.Y), ws_part, ws_cnt);
@@ -592,15 +620,16 @@ static cudaError_t launch_small_m_mp(const GemmArgs &a, const SmallMPlan &p, voi
   return e;
 }
 
-// W8 [N8, K] int8 as a 3-D tensor (k within a group, row, group) with
-// 128 x 128 x groups_per_box boxes: whole groups of a 128-row tile, each
-// 128-byte row swizzled.  Encodings are cached by (base, K, N8, box).
-static bool encode_w8_groups_3d(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *map, const void *W8, int64_t K,
-                                int64_t N8, int groups_per_box) {
+// An int8 [rows, K] matrix (W8 [N8, K], or A_q [M, K]) as a 3-D tensor (k
+// within a group, row, group) with 128 x box_rows x groups_per_box boxes:
+// whole groups of a block of rows, each 128-byte row swizzled.  Encodings are
+// cached by (base, K, rows, box).
+static bool encode_groups_3d(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *map, const void *W8, int64_t K,
+                             int64_t N8, int box_rows, int groups_per_box) {
   struct Entry {
     const void *base;
     int64_t K, N8;
-    int gpb;
+    int rows, gpb;
     bool valid;
     CUtensorMap map;
   };
@@ -609,19 +638,19 @@ static bool encode_w8_groups_3d(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorM
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
   for (const Entry &e : table)
-    if (e.valid && e.base == W8 && e.K == K && e.N8 == N8 && e.gpb == groups_per_box) {
+    if (e.valid && e.base == W8 && e.K == K && e.N8 == N8 && e.rows == box_rows && e.gpb == groups_per_box) {
       *map = e.map;
       return true;
     }
   const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(N8), static_cast<cuuint64_t>(K / 128)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K), 128};  // bytes, dims 1 and 2
-  const cuuint32_t box[3] = {128, 128, static_cast<cuuint32_t>(groups_per_box)};
+  const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(groups_per_box)};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(W8), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return false;
-  table[next] = Entry{W8, K, N8, groups_per_box, true, *map};
+  table[next] = Entry{W8, K, N8, box_rows, groups_per_box, true, *map};
   next = (next + 1) % 32;
   return true;
 }
@@ -638,7 +667,7 @@ static cudaError_t launch_gemv_mt(const GemmArgs &a, const SmallMPlan &p, void *
       *msg = "cuTensorMapEncodeTiled is not available from the driver";
       return cudaErrorNotSupported;
     }
-    if (!encode_w8_groups_3d(enc, &tmW8, a.W8, a.K, a.N8, GvCfg<MT>::kChunk8)) {
+    if (!encode_groups_3d(enc, &tmW8, a.W8, a.K, a.N8, 128, GvCfg<MT>::kChunk8)) {
       *msg = "tensor map encoding of W8 failed";
       return cudaErrorInvalidValue;
     }
@@ -697,7 +726,7 @@ static cudaError_t launch_gemv_persistent_mt(const GemmArgs &a, const SmallMPlan
       *msg = "cuTensorMapEncodeTiled is not available from the driver";
       return cudaErrorNotSupported;
     }
-    if (!encode_w8_groups_3d(enc, &tmW8, a.W8, a.K, a.N8, 2)) {
+    if (!encode_groups_3d(enc, &tmW8, a.W8, a.K, a.N8, 128, 2)) {
       *msg = "tensor map encoding of W8 failed";
       return cudaErrorInvalidValue;
     }
