@@ -11,6 +11,9 @@
 // How it runs on B200 (one CTA of 16 warps per 128 x BN output tile, both
 // channel sets in the same launch, warp-specialized, registers rebalanced
 // with setmaxnreg toward the epilogue):
+// The weights are the MMA's A operand (the tile's BN channels are the TMEM
+// lanes of the accumulator) and the activations its B operand (kBM tokens are
+// the accumulator's columns).
 //   warp 0      TMA producer: the A_q tile [128 x 128] (128-byte swizzle) of
 //               every group -- together with the int8 weight tile [BN x 128]
 //               on 8-bit tiles -- into a ring of stages, and on 4-bit tiles
@@ -20,27 +23,30 @@
 //   warps 1, 3  one thread each issues the MMAs of alternate groups: 4 x
 //               tcgen05.mma.kind::i8 (K = 32 each) into one of kAccBufs int32
 //               accumulators in tensor memory (TMEM), then one commit to the
-//               group's `done` barrier, which frees the A stage and unpacked
+//               group's `done` barrier, which frees the A_q stage and unpacked
 //               buffer it read and hands the accumulator to the epilogue.  The
 //               MMA of later groups overlaps the SIMT work on earlier ones.
-//   warp 2      stages, per group, the column scales s_w (fp32) and the row
+//   warp 2      stages, per group, the channel scales s_w (fp32) and the token
 //               scales s_a of the tile in a small ring the epilogue reads.
 //   warps 12-15 4-bit set only: unpack nibbles and subtract the zero point in
 //               SWAR form (four bytes per 32-bit op, no borrow between bytes)
-//               into an int8 tile in the 128-byte swizzled K-major layout the
-//               tensor core reads -- the B200 counterpart of the pages' vsub4
-//               pre-dequantization step (§ソフトウェアパイプライン).
+//               -- the B200 counterpart of the pages' vsub4 pre-dequantization
+//               step (§ソフトウェアパイプライン) -- and store the int8 rows
+//               with tcgen05.st into a TMEM buffer, from which the MMA reads
+//               its A operand: the unpacked tile never touches shared memory,
+//               so the tensor core's shared-memory reads per group halve.
 //   warps 4-11  epilogue: tcgen05.ld a group's int32 partials, which the
 //               accumulator already holds biased by 0x4b400000 (TMEM is preset
 //               to the bias), so their bits read as float are 1.5*2^23 + P
 //               exactly for |P| <= 2^22 -- the bias trick with no integer add.
-//               The bias is folded into an exact FMA with the row scale:
-//               u = fma(v, s_a, -1.5*2^23*s_a) = fl(P*s_a), exact because s_a
-//               is bf16-valued; then acc = fma(u, s_w, acc): two f32x2 FMAs
-//               per pair of elements, one shared-memory load per four.  After the last
-//               group, fp16 results are staged in shared memory and scattered
-//               row-wise to Y[:, idx] so each warp store covers a short run of
-//               one output row.
+//               The bias is folded into one FMA with the channel scale:
+//               u = fma(v, s_w, -1.5*2^23*s_w) = fl(P*s_w), one rounding,
+//               because 1.5*2^23*s_w is exact for an fp16-valued s_w; then
+//               acc = fma(u, s_a, acc): two f32x2 FMAs per pair of elements,
+//               one shared-memory load per four.  After the last group, fp16
+//               results are staged in shared memory and scattered row-wise to
+//               Y[:, idx] so each warp store covers a short run of one output
+//               row.
 // Every ring slot is refilled as soon as its own consumer is done with it (the
 // A stages and unpacked buffers through the group's `done` barrier, the packed
 // tiles through the unpack warps), and the rings are deep enough to cover the
@@ -79,16 +85,17 @@ struct GemmCfg {
   static constexpr int kABytes = kBM * kKG;        // 16 KB A_q tile of one group
   static constexpr int kW8Bytes = BN * kKG;        // 16 KB int8 weight tile
   static constexpr int kW4Bytes = BN * kKG / 2;    //  8 KB packed uint4 weight tile
-  static constexpr int kTBufBytes = BN * kKG;      // 16 KB unpacked 4-bit tile
   static constexpr int kZBytes = BN / 2;           // zero points of one group, two per byte
   // The ring region is laid out one of two ways, chosen per CTA:
   //   8-bit tile: kStages8 stages of [A | W8]                      (32 KB each)
-  //   4-bit tile: kStagesA4 A stages, kTBufs unpacked buffers and kRaw packed
-  //               tiles                                            (16/16/8 KB)
+  //   4-bit tile: kStagesA4 A stages and kRaw packed tiles          (16/8 KB)
+  // The unpacked 4-bit tiles live in tensor memory (kTBufs buffers of 32
+  // columns), where the MMA reads its weight operand: they take no shared
+  // memory and no shared-memory bandwidth.
   static constexpr int kStages8 = 6;
-  static constexpr int kStagesA4 = 6;
-  static constexpr int kTBufs = 4;
-  static constexpr int kRaw = 4;
+  static constexpr int kStagesA4 = 8;
+  static constexpr int kTBufs = 8;
+  static constexpr int kRaw = 8;
   static constexpr int kMaxStages = kStages8 > kStagesA4 ? kStages8 : kStagesA4;
   // Two threads issue the MMAs of alternate groups.  Every barrier an issuer
   // waits on must belong to one issuer only, or a parity wait could see a
@@ -96,15 +103,20 @@ struct GemmCfg {
   static_assert(kStages8 % 2 == 0 && kStagesA4 % 2 == 0 && kTBufs % 2 == 0, "rings the issuers wait on");
   // One commit per group, to done[g % kDone]; a waiter never falls a full ring
   // behind as long as kDone covers every ring that is released through it.
-  static constexpr int kDone = kMaxStages;
+  static constexpr int kDone = kMaxStages > kTBufs ? kMaxStages : kTBufs;
   static constexpr int kRing8 = kStages8 * (kABytes + kW8Bytes);
-  static constexpr int kRing4 = kStagesA4 * kABytes + kTBufs * kTBufBytes + kRaw * kW4Bytes;
+  static constexpr int kRing4 = kStagesA4 * kABytes + kRaw * kW4Bytes;
   static constexpr int kRingBytes = kRing8 > kRing4 ? kRing8 : kRing4;
-  static constexpr int kAccBufs = 4;
+  static constexpr int kAccBufs = 2;
   static_assert(kAccBufs % 2 == 0, "accumulators alternate between the issuers");
   static_assert(kDone >= kStages8 && kDone >= kStagesA4 && kDone >= kTBufs && kDone >= kAccBufs, "done ring");
   static constexpr int kTabSlots = 4;
-  static constexpr int kTmemCols = kAccBufs * BN;  // 512
+  // tensor memory: kAccBufs int32 accumulators of kBM (token) columns, then
+  // the unpacked weight tiles, 128 bytes of K per lane = 32 columns each
+  static constexpr int kTmemABase = kAccBufs * kBM;
+  static constexpr int kTmemABufCols = kKG / 4;
+  static constexpr int kTmemCols = 512;
+  static_assert(kTmemABase + kTBufs * kTmemABufCols <= kTmemCols, "tensor memory");
   static constexpr int kColsPerThread = BN * kBM / kEpiThreads;  // 64
   static constexpr int kTabSwBytes = BN * 4;                   // s_w of the tile's columns (fp32)
   static constexpr int kTabBytes = kTabSwBytes + kBM * 4;      // + s_a of the tile's rows
@@ -126,7 +138,7 @@ struct GemmCfg {
   static constexpr int kSmemAlloc = kSmemBytes + 1024;
   static constexpr int kStagingStride = (BN + 2) * 2;  // bytes per staged fp16 row
   static_assert(kBM * kStagingStride <= kRingBytes, "staging must fit in the ring region");
-  static_assert(kABytes % 1024 == 0 && kTBufBytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+  static_assert(kABytes % 1024 == 0 && kW8Bytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
 };
 
@@ -175,16 +187,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int32_t *idx = is4 ? idx4 : idx8;
   const int S = is4 ? C::kStagesA4 : C::kStages8;  // A stages of this tile
 
-  // ring region: 8-bit tiles [A | W8] x kStages8; 4-bit tiles A x kStagesA4, then unpacked, then packed
+  // ring region: 8-bit tiles [A | W8] x kStages8; 4-bit tiles A x kStagesA4, then the packed tiles
   const int stage_bytes = is4 ? C::kABytes : C::kABytes + C::kW8Bytes;
   auto stage_a = [&](int s) { return smem + C::kOffRing + s * stage_bytes; };
   auto stage_w8 = [&](int s) { return smem + C::kOffRing + s * stage_bytes + C::kABytes; };
-  auto tbuf = [&](int b) { return smem + C::kOffRing + C::kStagesA4 * C::kABytes + b * C::kTBufBytes; };
-  auto raw_w4 = [&](int r) {
-    return smem + C::kOffRing + C::kStagesA4 * C::kABytes + C::kTBufs * C::kTBufBytes + r * C::kW4Bytes;
-  };
+  auto raw_w4 = [&](int r) { return smem + C::kOffRing + C::kStagesA4 * C::kABytes + r * C::kW4Bytes; };
   auto zmeta = [&](int r) { return smem + C::kOffZ + r * C::kZBytes; };
   auto table = [&](int slot) { return reinterpret_cast<float4 *>(smem + C::kOffTab + slot * C::kTabBytes); };
+  auto table_sw = [&](int slot) { return reinterpret_cast<const float *>(smem + C::kOffTab + slot * C::kTabBytes); };
   auto table_sa = [&](int slot) {
     return reinterpret_cast<float *>(smem + C::kOffTab + slot * C::kTabBytes + C::kTabSwBytes);
   };
@@ -199,6 +209,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_arrive_expect_tx(&full[s], a_bytes);
     tma_load_2d(stage_a(s), &tmA, &full[s], g * kKG, m0);
     if (!is4) tma_load_2d(stage_w8(s), &tmW8, &full[s], g * kKG, n0);
+  };
+  // Loads of the packed 4-bit tile and zero points of group g into slot g % kRaw.
+  auto load_raw = [&](int g) {
+    const int r = g % C::kRaw;
+    mbar_arrive_expect_tx(&rfull[r], static_cast<uint32_t>(C::kW4Bytes + C::kZBytes));
+    // the tile's packed group is one contiguous block: one bulk copy
+    bulk_load(raw_w4(r), W4 + (static_cast<int64_t>(n0 >> 7) * G + g) * C::kW4Bytes, C::kW4Bytes, &rfull[r]);
+    bulk_load(zmeta(r), z4 + static_cast<int64_t>(g) * (N4p >> 1) + (n0 >> 1), C::kZBytes, &rfull[r]);
   };
 
   if (threadIdx.x == 0) {
@@ -254,11 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // packed slot gw % kRaw last held group gw - kRaw; the unpack warps released it
           if (gw < G &&
               (gw < C::kRaw || mbar_try_wait(smem_u32(&rempty[gw % C::kRaw]), ((gw / C::kRaw) - 1) & 1))) {
-            const int r = gw % C::kRaw;
-            mbar_arrive_expect_tx(&rfull[r], static_cast<uint32_t>(C::kW4Bytes + C::kZBytes));
-            // the tile's packed group is one contiguous block: one bulk copy
-            bulk_load(raw_w4(r), W4 + (static_cast<int64_t>(n0 >> 7) * G + gw) * C::kW4Bytes, C::kW4Bytes, &rfull[r]);
-            bulk_load(zmeta(r), z4 + static_cast<int64_t>(gw) * (N4p >> 1) + (n0 >> 1), C::kZBytes, &rfull[r]);
+            load_raw(gw);
             ++gw;
             progressed = true;
           }
@@ -294,8 +308,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Two threads issue alternate groups (warp 1 the even ones, warp 3 the
       // odd ones): one thread pays for every tcgen05.mma and commit it issues
       // and leaves the tensor pipe idle between groups, two keep it busy.
+      // The weights are the MMA's A operand (BN channels = the TMEM lanes of
+      // the accumulator), the activations its B operand (kBM token columns):
+      // on 4-bit tiles A comes from the unpacked buffer in tensor memory.
       if (lane == 0) {
-        constexpr uint32_t idesc = idesc_i8(kBM, BN);
+        constexpr uint32_t idesc = idesc_i8(BN, kBM);
         const int who = warp == 1 ? 0 : 1;
         for (int g = who; g < G; g += 2) {
           const int s = g % S, b = g % C::kTBufs, a = g % C::kAccBufs;
@@ -304,12 +321,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           // phase 0 of accempty[a] is the epilogue's bias fill; phase u+1 its drain of use u
           if (!mbar_wait(&accempty[a], (g / C::kAccBufs) & 1, abort_flag)) break;
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(stage_a(s));
-          const uint32_t b_addr = smem_u32(is4 ? tbuf(b) : stage_w8(s));
-          const uint32_t d = tmem_base + static_cast<uint32_t>(a * BN);
+          const uint32_t x_addr = smem_u32(stage_a(s));
+          const uint32_t d = tmem_base + static_cast<uint32_t>(a * kBM);
+          if (is4) {
+            const uint32_t wt = tmem_base + static_cast<uint32_t>(C::kTmemABase + b * C::kTmemABufCols);
 #pragma unroll
-          for (int kk = 0; kk < kKG / 32; ++kk)
-            mma_i8(d, sw128_kmajor_desc(a_addr + 32 * kk), sw128_kmajor_desc(b_addr + 32 * kk), idesc, 1u);
+            for (int kk = 0; kk < kKG / 32; ++kk)
+              mma_i8_ts(d, wt + 8 * kk, sw128_kmajor_desc(x_addr + 32 * kk), idesc, 1u);
+          } else {
+            const uint32_t w_addr = smem_u32(stage_w8(s));
+#pragma unroll
+            for (int kk = 0; kk < kKG / 32; ++kk)
+              mma_i8(d, sw128_kmajor_desc(w_addr + 32 * kk), sw128_kmajor_desc(x_addr + 32 * kk), idesc, 1u);
+          }
           mma_commit(&done[g % C::kDone]);
         }
         mma_commit(&drain[who]);
@@ -376,67 +400,79 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_dec<kRegsXform>();
     // ------------------------------------------------------------ 4-bit unpack
     if (is4) {
-      // Thread tt owns the 16-byte column chunk c = tt % 4 (32 nibbles = 32
-      // weights) of rows r0, r0+32, r0+64, r0+96 (r0 = tt / 4): all four loads
-      // are issued before any arithmetic, so one warp per SM sub-partition
-      // keeps several shared-memory loads in flight.
-      const int tt = threadIdx.x - 384;  // 0..127
-      const int c = tt & 3, r0 = tt >> 2;
-      const int zshift = (r0 & 1) * 4;   // rows r0 + 32k share r0's parity and swizzle phase
-      const int sw = r0 & 7;
-      constexpr int kRowsPerThread = BN / 32;
+      // Warp 12 + q writes TMEM lane quadrant q: thread `lane` unpacks weight
+      // row rr = 32q + lane of the tile (64 packed bytes -> 128 int8 values)
+      // and stores it as the 32 columns of its lane in the group's buffer.
+      // The packed rows are 64 bytes apart, so lanes read their four 16-byte
+      // chunks in a rotated order (8 distinct bank groups per load) and the
+      // rotation is undone in registers.
+      const int q = warp & 3;
+      const int rr = q * 32 + lane;
+      const int rot = (lane >> 1) & 3;
+      const int zshift = (rr & 1) * 4;
+      const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + C::kTmemABase;
       for (int g = 0; g < G; ++g) {
         const int r = g % C::kRaw, b = g % C::kTBufs;
         if (!warp_wait(&rfull[r], (g / C::kRaw) & 1, abort_flag)) break;
-        // unpacked buffer b last held group g - kTBufs: free once that group is done
+        // buffer b last held group g - kTBufs: free once that group's MMAs are done
         if (g >= C::kTBufs) {
           const int gp = g - C::kTBufs;
           if (!warp_wait(&done[gp % C::kDone], (gp / C::kDone) & 1, abort_flag)) break;
+          tc_fence_after();
         }
-        const uint8_t *raw = raw_w4(r);
-        const uint8_t *zb = zmeta(r);
-        uint8_t *dst = tbuf(b);
-        uint4 x[kRowsPerThread];
-        uint32_t zz[kRowsPerThread];
+        const uint8_t *src = raw_w4(r) + rr * 64;
+        uint4 x[4];
 #pragma unroll
-        for (int k = 0; k < kRowsPerThread; ++k) {
-          const int rr = r0 + 32 * k;
-          x[k] = *reinterpret_cast<const uint4 *>(raw + rr * 64 + c * 16);
-          zz[k] = ((static_cast<uint32_t>(zb[rr >> 1]) >> zshift) & 0xFu) * 0x01010101u;
+        for (int c = 0; c < 4; ++c) x[c] = *reinterpret_cast<const uint4 *>(src + (((c + rot) & 3) << 4));
+        const uint32_t zz = ((static_cast<uint32_t>(zmeta(r)[rr >> 1]) >> zshift) & 0xFu) * 0x01010101u;
+        // x[c] holds chunk (c + rot) & 3: rotate back by rot = (rot & 1) + (rot & 2)
+        if (rot & 1) {
+          const uint4 t3 = x[3];
+          x[3] = x[2];
+          x[2] = x[1];
+          x[1] = x[0];
+          x[0] = t3;
         }
+        if (rot & 2) {
+          const uint4 t0 = x[0], t1 = x[1];
+          x[0] = x[2];
+          x[1] = x[3];
+          x[2] = t0;
+          x[3] = t1;
+        }
+        // chunk c: low nibbles are k = 32c .. 32c+15 (columns 8c .. 8c+3),
+        // high nibbles k = 32c+16 .. 32c+31 (columns 8c+4 .. 8c+7)
+        uint32_t o[32];
 #pragma unroll
-        for (int k = 0; k < kRowsPerThread; ++k) {
-          const int rr = r0 + 32 * k;
-          uint4 lo, hi;
-          lo.x = sub_zero_bytes(x[k].x & 0x0F0F0F0Fu, zz[k]);
-          lo.y = sub_zero_bytes(x[k].y & 0x0F0F0F0Fu, zz[k]);
-          lo.z = sub_zero_bytes(x[k].z & 0x0F0F0F0Fu, zz[k]);
-          lo.w = sub_zero_bytes(x[k].w & 0x0F0F0F0Fu, zz[k]);
-          hi.x = sub_zero_bytes((x[k].x >> 4) & 0x0F0F0F0Fu, zz[k]);
-          hi.y = sub_zero_bytes((x[k].y >> 4) & 0x0F0F0F0Fu, zz[k]);
-          hi.z = sub_zero_bytes((x[k].z >> 4) & 0x0F0F0F0Fu, zz[k]);
-          hi.w = sub_zero_bytes((x[k].w >> 4) & 0x0F0F0F0Fu, zz[k]);
-          *reinterpret_cast<uint4 *>(dst + rr * 128 + (((2 * c) ^ sw) << 4)) = lo;
-          *reinterpret_cast<uint4 *>(dst + rr * 128 + (((2 * c + 1) ^ sw) << 4)) = hi;
+        for (int c = 0; c < 4; ++c) {
+          o[8 * c + 0] = sub_zero_bytes(x[c].x & 0x0F0F0F0Fu, zz);
+          o[8 * c + 1] = sub_zero_bytes(x[c].y & 0x0F0F0F0Fu, zz);
+          o[8 * c + 2] = sub_zero_bytes(x[c].z & 0x0F0F0F0Fu, zz);
+          o[8 * c + 3] = sub_zero_bytes(x[c].w & 0x0F0F0F0Fu, zz);
+          o[8 * c + 4] = sub_zero_bytes((x[c].x >> 4) & 0x0F0F0F0Fu, zz);
+          o[8 * c + 5] = sub_zero_bytes((x[c].y >> 4) & 0x0F0F0F0Fu, zz);
+          o[8 * c + 6] = sub_zero_bytes((x[c].z >> 4) & 0x0F0F0F0Fu, zz);
+          o[8 * c + 7] = sub_zero_bytes((x[c].w >> 4) & 0x0F0F0F0Fu, zz);
         }
-        fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&rempty[r]);
-          mbar_arrive(&tfull[b]);
-        }
+        if (lane == 0) mbar_arrive(&rempty[r]);  // the packed tile is in registers
+        tmem_st_32x32b_x32(trow + static_cast<uint32_t>(b * C::kTmemABufCols), o);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tfull[b]);
       }
     }
   } else {
     regs_inc<kRegsEpi>();
     // ------------------------------------------------------------ epilogue
-    constexpr int CPT = C::kColsPerThread;  // 64 columns per thread
+    // The accumulator is D[channel, token]: this thread owns channel `ch` of
+    // the tile (its TMEM lane) and the tokens half*CPT .. half*CPT+CPT-1.
+    constexpr int CPT = C::kColsPerThread;  // 64 token columns per thread
     const int e = warp - 4;                 // 0..7
     const int quad = warp & 3;              // TMEM lane quadrant of this warp
     const int half = e >> 2;                // column half
-    const int row = quad * 32 + lane;
-    const int m = m0 + row;
-    const bool row_ok = m < M;
+    const int ch = quad * 32 + lane;
 
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + half * CPT;
     // Every accumulator starts at the bias 0x4b400000 (and is reset to it after
@@ -445,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int a = 0; a < C::kAccBufs; ++a)
 #pragma unroll
-      for (int c = 0; c < CPT; c += 32) tmem_st_32x32b_x32_fill(lane_base + a * BN + c, kI2FBiasBits);
+      for (int c = 0; c < CPT; c += 32) tmem_st_32x32b_x32_fill(lane_base + a * kBM + c, kI2FBiasBits);
     tmem_st_wait();
     tc_fence_before();
     __syncwarp();
@@ -461,20 +497,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     // chunk, or the next group's first) is in flight.
     constexpr int CW = 16, NCH = CPT / CW;
     uint32_t rbuf[2][CW];
-    // v = bits of (1.5*2^23 + P) as float; u = fma(v, s_a, -1.5*2^23*s_a) is
-    // exactly fl(P * s_a) (the bias term is exact for a bf16-valued s_a); then
-    // acc += u * s_w.  tab holds the s_w of 4 consecutive columns per float4.
-    auto convert = [&](uint32_t(&r)[CW], const float4 *tab, float2 sa2, float2 cb2, int c0) {
+    // v = bits of (1.5*2^23 + P) as float; u = fma(v, s_w, -1.5*2^23*s_w) is
+    // exactly fl(P * s_w): the bias term 1.5*2^23*s_w is exact for an
+    // fp16-valued s_w and the fma rounds v*s_w - 1.5*2^23*s_w = P*s_w once.
+    // Then acc += u * s_a.  tab holds the s_a of 4 consecutive tokens per float4.
+    auto convert = [&](uint32_t(&r)[CW], const float4 *tab, float2 sw2, float2 cb2, int c0) {
 #pragma unroll
       for (int j = 0; j < CW / 4; ++j) {
-        const float4 sw = tab[j];
+        const float4 sa = tab[j];
         const float2 v0 = make_float2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]));
         const float2 v1 = make_float2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
-        const float2 u0 = __ffma2_rn(v0, sa2, cb2);
-        const float2 u1 = __ffma2_rn(v1, sa2, cb2);
-        const float2 o0 = __ffma2_rn(u0, make_float2(sw.x, sw.y), make_float2(acc[c0 + 4 * j], acc[c0 + 4 * j + 1]));
+        const float2 u0 = __ffma2_rn(v0, sw2, cb2);
+        const float2 u1 = __ffma2_rn(v1, sw2, cb2);
+        const float2 o0 = __ffma2_rn(u0, make_float2(sa.x, sa.y), make_float2(acc[c0 + 4 * j], acc[c0 + 4 * j + 1]));
         const float2 o1 =
-            __ffma2_rn(u1, make_float2(sw.z, sw.w), make_float2(acc[c0 + 4 * j + 2], acc[c0 + 4 * j + 3]));
+            __ffma2_rn(u1, make_float2(sa.z, sa.w), make_float2(acc[c0 + 4 * j + 2], acc[c0 + 4 * j + 3]));
         acc[c0 + 4 * j] = o0.x;
         acc[c0 + 4 * j + 1] = o0.y;
         acc[c0 + 4 * j + 2] = o1.x;
@@ -482,12 +519,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     auto dump = [&](uint32_t(&r)[CW], int g, int c0) {
-      if (row_ok) {
+      if (n0 + ch < Nset) {
+        const int64_t nout = idx[n0 + ch];
 #pragma unroll 4
         for (int j = 0; j < CW; ++j) {
-          const int col = half * CPT + c0 + j;
-          if (n0 + col < Nset)
-            P[(static_cast<int64_t>(m) * N + idx[n0 + col]) * G + g] = static_cast<int32_t>(r[j] - kI2FBiasBits);
+          const int m = m0 + half * CPT + c0 + j;
+          if (m < M) P[(static_cast<int64_t>(m) * N + nout) * G + g] = static_cast<int32_t>(r[j] - kI2FBiasBits);
         }
       }
     };
@@ -499,12 +536,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int g = 0; live && g < G; ++g) {
       const int a = g % C::kAccBufs, slot = g % C::kTabSlots;
-      const uint32_t col = lane_base + static_cast<uint32_t>(a * BN);
+      const uint32_t col = lane_base + static_cast<uint32_t>(a * kBM);
       if (!warp_wait(&tabfull[slot], (g / C::kTabSlots) & 1, abort_flag)) break;
-      const float sa = table_sa(slot)[row];
-      const float2 sa2 = make_float2(sa, sa);
-      const float2 cb2 = make_float2(-kI2FBias * sa, -kI2FBias * sa);
-      const float4 *tab = table(slot) + half * (CPT / 4);
+      const float sw = table_sw(slot)[ch];
+      const float2 sw2 = make_float2(sw, sw);
+      const float2 cb2 = make_float2(-kI2FBias * sw, -kI2FBias * sw);
+      const float4 *tab = reinterpret_cast<const float4 *>(table_sa(slot)) + half * (CPT / 4);
 #pragma unroll
       for (int c = 0; c < NCH; ++c) {
         tmem_ld_wait();
@@ -524,14 +561,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             live = warp_wait(&done[(g + 1) % C::kDone], ((g + 1) / C::kDone) & 1, abort_flag);
             if (live) {
               tc_fence_after();
-              tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(a1 * BN), rbuf[(c + 1) & 1]);
+              tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(a1 * kBM), rbuf[(c + 1) & 1]);
             }
           }
         }
         if constexpr (kDebugP) {
           dump(rbuf[c & 1], g, CW * c);
         } else {
-          convert(rbuf[c & 1], tab + (CW / 4) * c, sa2, cb2, CW * c);
+          convert(rbuf[c & 1], tab + (CW / 4) * c, sw2, cb2, CW * c);
         }
       }
       __syncwarp();
@@ -540,11 +577,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_ld_wait();
 
     if constexpr (!kDebugP) {
-      // stage fp16 results: row `row`, columns half*CPT .. +CPT
+      // stage fp16 results as [token][channel]: column `ch`, token rows
+      // half*CPT .. +CPT (a warp's stores cover 64 contiguous bytes of a row)
       uint8_t *st = smem + C::kOffRing;
-      __half2 *dst = reinterpret_cast<__half2 *>(st + row * C::kStagingStride + half * CPT * 2);
+      __half *dst = reinterpret_cast<__half *>(st + half * CPT * C::kStagingStride) + ch;
 #pragma unroll
-      for (int j = 0; j < CPT / 2; ++j) dst[j] = __floats2half2_rn(acc[2 * j], acc[2 * j + 1]);
+      for (int j = 0; j < CPT; ++j) dst[j * (C::kStagingStride / 2)] = __float2half_rn(acc[j]);
       named_bar_sync(1, kEpiThreads);
       if (!*abort_flag) {
         constexpr int CPL = BN / 32;  // columns per lane
