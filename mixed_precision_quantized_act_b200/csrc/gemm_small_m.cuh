@@ -59,13 +59,18 @@ struct SmallMCfg {
   // copy rate grows with the bytes per copy, so per-group copies of 8 KiB
   // would bound it far below HBM speed.  A stage is the chunk's weights, then
   // its token tiles (one 3-D box, group after group).
-  static constexpr int kRingBytes = 128 * 1024;
+  // Where the unpacked 4-bit tiles live: tensor memory for 16 and 32 tokens
+  // (the MMA reads its weight operand there, and the 64 KiB of shared memory
+  // they would take doubles the ring: 4 stages instead of 2); shared memory
+  // for 64 tokens, whose stages are too large for a third one to fit.
+  static constexpr bool kTmemW = MP <= 32;
+  static constexpr int kRingBytes = kTmemW ? 192 * 1024 : 128 * 1024;
   static constexpr int kGpc4 = 4, kGpc8 = 2;                // groups per chunk
   static constexpr int kChunkWBytes = 32768;
   static constexpr int kMaxStages = 16;
-  // Unpacked 4-bit tiles: buffer i % kTBufs is free again only when the MMAs
-  // of group i - kTBufs have completed (~800 cycles after their commit), so
-  // the unpack needs several in flight.
+  // Unpacked 4-bit tiles (32 TMEM columns or 16 KiB of shared memory each):
+  // buffer i % kTBufs is free again only when the MMAs of group i - kTBufs
+  // have completed, so the unpack needs several in flight.
   static constexpr int kTBufs = 4;
   static constexpr int kAccBufs = 4;
   static constexpr int kDone = kMaxStages;              // >= every ring released through it
@@ -73,11 +78,16 @@ struct SmallMCfg {
   static constexpr int kWBytes = 128 * 128;             // int8 weight tile (W8), or the unpacked 4-bit tile
   static constexpr int kW4Bytes = 128 * 64;             // packed 4-bit tile
   static constexpr int kXBytes = MP * 128;              // token tile of one group
-  static constexpr int kTmemCols = kAccBufs * MP < 32 ? 32 : kAccBufs * MP;
+  // tensor memory: kAccBufs accumulators of MP columns, then the unpacked
+  // weight buffers; the allocation is a power of two
+  static constexpr int kTmemABase = kAccBufs * MP;
+  static constexpr int kTmemUsed = kTmemABase + (kTmemW ? kTBufs * 32 : 0);
+  static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128 : kTmemUsed <= 256 ? 256 : 512;
+  static_assert(kTmemUsed <= 512, "tensor memory");
   // shared-memory layout (offsets from a 1024-byte aligned base)
   static constexpr int kOffStages = 0;
   static constexpr int kOffTBuf = kOffStages + kRingBytes;
-  static constexpr int kOffZ = kOffTBuf + kTBufs * kWBytes;
+  static constexpr int kOffZ = kOffTBuf + (kTmemW ? 0 : kTBufs * kWBytes);
   static constexpr int kOffSw = kOffZ + kMaxStages * kGpc4 * 64;      // fp16 s_w [groups][128]
   static constexpr int kOffSa = kOffSw + kSmGroupsMax * 128 * 4;       // fp32 s_a [groups][MP]
   static constexpr int kOffBar = kOffSa + kSmGroupsMax * MP * 4;
@@ -202,7 +212,7 @@ __global__ void __launch_bounds__(kSmThreads, 1)
   nst &= ~1;  // even
   auto stage_w = [&](int s) { return smem + C::kOffStages + s * stage_sz; };
   auto stage_x = [&](int s) { return smem + C::kOffStages + s * stage_sz + C::kChunkWBytes; };
-  auto tbuf = [&](int b) { return smem + C::kOffTBuf + b * C::kWBytes; };
+  auto tbuf = [&](int b) { return smem + C::kOffTBuf + b * C::kWBytes; };  // shared-memory unpacked tiles
   auto zmeta = [&](int s) { return smem + C::kOffZ + s * C::kGpc4 * 64; };
   // where local group i lives: its chunk's stage, its offset in the chunk, the phase of the stage
   auto gstage = [&](int i) { return (i / gpc) % nst; };
@@ -229,7 +239,7 @@ __global__ void __launch_bounds__(kSmThreads, 1)
     prefetch_tmap(is4 ? &tmZ : &tmW8);
     for (int s = 0; s < C::kMaxStages; ++s) mbar_init(&full[s], 1);
     for (int i = 0; i < C::kDone; ++i) mbar_init(&done[i], 1);
-    for (int b = 0; b < C::kTBufs; ++b) mbar_init(&tfull[b], kSmUnpackWarps);
+    for (int b = 0; b < C::kTBufs; ++b) mbar_init(&tfull[b], C::kTmemW ? kSmUnpackWarps / 2 : kSmUnpackWarps);
     for (int a = 0; a < C::kAccBufs; ++a) mbar_init(&accempty[a], 4);
     mbar_init(tabready, 1);
     mbar_init(&drain[0], 1);
@@ -285,12 +295,18 @@ __global__ void __launch_bounds__(kSmThreads, 1)
         // phase 0 of accempty[a] is the epilogue's bias fill, phase u+1 its drain of use u
         if (!mbar_wait(&accempty[a], (i / C::kAccBufs) & 1, abort_flag)) break;
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(is4 ? tbuf(b) : stage_w(s) + j * C::kWBytes);  // weights: 128 channels x 128 k
-        const uint32_t b_addr = smem_u32(stage_x(s) + j * C::kXBytes);                   // tokens: MP rows x 128 k
+        const uint32_t b_addr = smem_u32(stage_x(s) + j * C::kXBytes);  // tokens: MP rows x 128 k
         const uint32_t d = tmem_base + static_cast<uint32_t>(a * MP);
+        if (is4 && C::kTmemW) {  // weights: 128 channels x 128 k, unpacked into tensor memory
+          const uint32_t wt = tmem_base + static_cast<uint32_t>(C::kTmemABase + b * 32);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_i8(d, sw128_kmajor_desc(a_addr + 32 * kk), sw128_kmajor_desc(b_addr + 32 * kk), idesc, 1u);
+          for (int kk = 0; kk < 4; ++kk) mma_i8_ts(d, wt + 8 * kk, sw128_kmajor_desc(b_addr + 32 * kk), idesc, 1u);
+        } else {  // weights in shared memory: the unpacked tile, or the int8 tile of the stage
+          const uint32_t a_addr = smem_u32(is4 ? tbuf(b) : stage_w(s) + j * C::kWBytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_i8(d, sw128_kmajor_desc(a_addr + 32 * kk), sw128_kmajor_desc(b_addr + 32 * kk), idesc, 1u);
+        }
         mma_commit(&done[i % C::kDone]);
       }
       mma_commit(&drain[who]);
@@ -318,9 +334,72 @@ __global__ void __launch_bounds__(kSmThreads, 1)
   } else if (warp < 12) {
     regs_dec<kSmRegsUnpack>();
     // ------------------------------------------------------------ 4-bit unpack
+    // Warps 4 + q and 8 + q both write TMEM lane quadrant q and take alternate
+    // groups.  Thread `lane` unpacks weight row rr = 32q + lane of the tile
+    // (64 packed bytes -> 128 int8 values) and stores it as the 32 columns of
+    // its lane in the group's buffer.  The packed rows are 64 bytes apart, so
+    // lanes read their four 16-byte chunks in a rotated order (8 distinct bank
+    // groups per load) and the rotation is undone in registers.
+    if (C::kTmemW && is4) {
+      const int q = warp & 3, h = (warp - 4) >> 2;
+      const int rr = q * 32 + lane;
+      const int rot = (lane >> 1) & 3;
+      const int zshift = (rr & 1) * 4;
+      const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + C::kTmemABase;
+      for (int i = h; i < ng; i += 2) {
+        const int s = gstage(i), j = i % gpc, b = i % C::kTBufs;
+        if (!warp_wait(&full[s], gphase(i), abort_flag)) break;
+        if (i >= C::kTBufs) {  // buffer b last held local group i - kTBufs
+          const int ip = i - C::kTBufs;
+          if (!warp_wait(&done[ip % C::kDone], (ip / C::kDone) & 1, abort_flag)) break;
+          tc_fence_after();
+        }
+        const uint8_t *src = stage_w(s) + j * C::kW4Bytes + rr * 64;
+        uint4 x[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) x[k] = *reinterpret_cast<const uint4 *>(src + (((k + rot) & 3) << 4));
+        const uint32_t zz = ((static_cast<uint32_t>(zmeta(s)[j * 64 + (rr >> 1)]) >> zshift) & 0xFu) * 0x01010101u;
+        // x[k] holds chunk (k + rot) & 3: rotate back by rot = (rot & 1) + (rot & 2)
+        if (rot & 1) {
+          const uint4 t3 = x[3];
+          x[3] = x[2];
+          x[2] = x[1];
+          x[1] = x[0];
+          x[0] = t3;
+        }
+        if (rot & 2) {
+          const uint4 t0 = x[0], t1 = x[1];
+          x[0] = x[2];
+          x[1] = x[3];
+          x[2] = t0;
+          x[3] = t1;
+        }
+        // chunk k: low nibbles are k-slice 32k .. 32k+15 (columns 8k .. 8k+3),
+        // high nibbles 32k+16 .. 32k+31 (columns 8k+4 .. 8k+7)
+        uint32_t o[32];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          o[8 * k + 0] = sm_sub_zero_bytes(x[k].x & 0x0F0F0F0Fu, zz);
+          o[8 * k + 1] = sm_sub_zero_bytes(x[k].y & 0x0F0F0F0Fu, zz);
+          o[8 * k + 2] = sm_sub_zero_bytes(x[k].z & 0x0F0F0F0Fu, zz);
+          o[8 * k + 3] = sm_sub_zero_bytes(x[k].w & 0x0F0F0F0Fu, zz);
+          o[8 * k + 4] = sm_sub_zero_bytes((x[k].x >> 4) & 0x0F0F0F0Fu, zz);
+          o[8 * k + 5] = sm_sub_zero_bytes((x[k].y >> 4) & 0x0F0F0F0Fu, zz);
+          o[8 * k + 6] = sm_sub_zero_bytes((x[k].z >> 4) & 0x0F0F0F0Fu, zz);
+          o[8 * k + 7] = sm_sub_zero_bytes((x[k].w >> 4) & 0x0F0F0F0Fu, zz);
+        }
+        tmem_st_32x32b_x32(trow + static_cast<uint32_t>(b * 32), o);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tfull[b]);
+      }
+    }
+    // 64 tokens: the unpacked tile goes to shared memory in the 128-byte
+    // swizzled K-major layout.
     // Thread tt owns the 16-byte column chunk c = tt % 4 (32 weights) of rows
     // r0 and r0 + 64 (r0 = tt / 4).
-    if (is4) {
+    if (!C::kTmemW && is4) {
       const int tt = threadIdx.x - 128;  // 0..255
       const int c = tt & 3, r0 = tt >> 2;
       const int zshift = (r0 & 1) * 4;
