@@ -24,9 +24,11 @@
 // group into a ring of stages), warps 1 and 3 MMA issuers (alternate groups,
 // one commit per group),
 // warp 2 scale tables (this CTA's groups, loaded once), warps 4-11 4-bit
-// unpack into the swizzled int8 operand (with few tokens it is the longest
-// per-group step), warps 12-15 epilogue (one TMEM lane quadrant each).  Every
-// wait is bounded as in the tiled kernel.
+// unpack (with few tokens it is the longest per-group step) -- for 16 and 32
+// tokens into tensor memory, where the MMA reads its weight operand, for 64
+// tokens into the swizzled int8 operand in shared memory -- warps 12-15
+// epilogue (one TMEM lane quadrant each).  Every wait is bounded as in the
+// tiled kernel.
 // Up to kGemvMaxM tokens the entry points below run the GEMV kernel instead
 // (gemv_w4w8a8.cuh): the same plan, workspace layout and split reduction.
 #pragma once
