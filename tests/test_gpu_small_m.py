@@ -44,8 +44,9 @@ def _layer(name, M, N, K, n8, outliers=4):
 
 
 # GEMV (M <= 8: token bounds 1 / 2 / 4 / 8) and tensor-core kernel (token
-# tiles 16 / 32 / 64) on either side of M = 8, ragged N, one set empty, one
-# 8-bit channel, split counts from 1 (wide N) to the group cap (long K)
+# tiles 16 / 32 / 64) on either side of M = 8, ragged N, one set empty (on
+# both kernels), one 8-bit channel, split counts from 1 (wide N) to the
+# group cap (long K)
 CASES = [
     wl.Q_PROJ_P10.with_m(1),
     wl.Q_PROJ_P10.with_m(2),
@@ -58,6 +59,8 @@ CASES = [
     _layer("sm_m33", 33, 640, 1024, 64),
     _layer("sm_m7_p0", 7, 512, 512, 0),
     _layer("sm_m7_p100", 7, 512, 512, 512),
+    _layer("sm_m16_p0", 16, 384, 640, 0),
+    _layer("sm_m40_p100", 40, 384, 512, 384),
     _layer("sm_m2_one_8bit", 2, 260, 256, 1),
     _layer("sm_m3_k128", 3, 384, 128, 40),
     _layer("sm_m1_k8960", 1, 200, 8960, 30),
