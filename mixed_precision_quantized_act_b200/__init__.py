@@ -13,6 +13,7 @@ from ._lib import (  # noqa: F401
     gemm_debug_partials,
     gemm_w4w8a8,
     channel_salience,
+    channel_salience_into,
     gemm_w4w8a8_into,
     gemm_w4w8a8_small_m,
     gemm_w4w8a8_small_m_noalloc_into,
@@ -26,6 +27,8 @@ from ._lib import (  # noqa: F401
     quantize_act,
     quantize_act_into,
     select_top_t,
+    select_top_t_into,
+    select_top_t_workspace,
     selftest_wait_timeout,
     small_m_kernel,
     small_m_workspace,

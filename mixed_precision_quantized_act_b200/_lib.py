@@ -95,6 +95,12 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+def _require(ok: bool, what: str):
+    """Argument check that stays on under ``python -O`` (unlike assert)."""
+    if not ok:
+        raise ValueError(what)
+
+
 def _need_cuda(*ts):
     for t in ts:
         if t is not None and t.numel() > 0 and not t.is_cuda:
@@ -115,8 +121,9 @@ def packed_sizes(N: int, K: int, N8: int, group: int = GROUP):
 
 def quantize_act_into(X: torch.Tensor, A_q: torch.Tensor, s_a: torch.Tensor, stream=None):
     _need_cuda(X, A_q, s_a)
-    assert X.dtype == torch.float16 and A_q.dtype == torch.int8 and s_a.dtype == torch.float32
-    assert X.is_contiguous() and A_q.is_contiguous() and s_a.is_contiguous()
+    _require(X.dtype == torch.float16 and A_q.dtype == torch.int8 and s_a.dtype == torch.float32,
+             "X must be fp16, A_q int8 and s_a fp32")
+    _require(X.is_contiguous() and A_q.is_contiguous() and s_a.is_contiguous(), "X, A_q and s_a must be contiguous")
     M, K = X.shape
     _check(load().mixllm_quantize_act(_ptr(X), M, K, GROUP, _ptr(A_q), _ptr(s_a), _stream(stream)),
            "mixllm_quantize_act")
@@ -174,14 +181,15 @@ def pack_weights(W: torch.Tensor, is8: torch.Tensor, stream=None) -> PackedLinea
     """W fp32 [N, K] and the channel bit map uint8 [N] (CUDA) -> PackedLinear.
     Synchronous (offline step)."""
     _need_cuda(W, is8)
-    assert W.dtype == torch.float32 and W.is_contiguous()
-    assert is8.dtype == torch.uint8 and is8.is_contiguous()
+    _require(W.dtype == torch.float32 and W.is_contiguous() and W.dim() == 2, "W must be a contiguous fp32 [N, K]")
+    _require(is8.dtype == torch.uint8 and is8.is_contiguous() and is8.numel() == W.shape[0],
+             "is8 must be a contiguous uint8 [N]")
     N, K = W.shape
     N8 = int((is8 != 0).sum().item())
     p = empty_packed(N, K, N8, W.device)
     sizes = packed_sizes(N, K, N8)
     got = [t.numel() * t.element_size() for t in (p.W4, p.z4, p.s_w4, p.idx4, p.W8, p.s_w8, p.idx8)]
-    assert got == sizes, (got, sizes)
+    _require(got == sizes, f"packed buffer sizes {got} differ from the library's {sizes}")
     _check(load().mixllm_pack_weights(_ptr(W), N, K, _ptr(is8), N8, GROUP, _ptr(p.W4), _ptr(p.z4),
                                       _ptr(p.s_w4), _ptr(p.idx4), _ptr(p.W8), _ptr(p.s_w8),
                                       _ptr(p.idx8), _stream(stream)), "mixllm_pack_weights")
@@ -191,7 +199,8 @@ def pack_weights(W: torch.Tensor, is8: torch.Tensor, stream=None) -> PackedLinea
 def gemm_w4w8a8_into(A_q, s_a, p: PackedLinear, Y, stream=None):
     _need_cuda(A_q, s_a, Y)
     M, K = A_q.shape
-    assert K == p.K and Y.shape == (M, p.N) and Y.dtype == torch.float16 and Y.is_contiguous()
+    _require(K == p.K and tuple(Y.shape) == (M, p.N) and Y.dtype == torch.float16 and Y.is_contiguous(),
+             "Y must be a contiguous fp16 [M, N] and A_q must have the layer's K")
     _check(load().mixllm_gemm_w4w8a8(_ptr(A_q), _ptr(s_a), M, K, _ptr(p.W4), _ptr(p.z4), _ptr(p.s_w4),
                                      _ptr(p.idx4), p.N4, _ptr(p.W8), _ptr(p.s_w8), _ptr(p.idx8), p.N8,
                                      _ptr(Y), _stream(stream)), "mixllm_gemm_w4w8a8")
@@ -262,8 +271,9 @@ def small_m_workspace(M: int, p: PackedLinear, device) -> torch.Tensor:
 def gemm_w4w8a8_small_m_into(A_q, s_a, p: PackedLinear, Y, workspace: torch.Tensor, stream=None):
     _need_cuda(A_q, s_a, Y, workspace)
     M, K = A_q.shape
-    assert K == p.K and Y.shape == (M, p.N) and Y.dtype == torch.float16 and Y.is_contiguous()
-    assert workspace.is_contiguous()
+    _require(K == p.K and tuple(Y.shape) == (M, p.N) and Y.dtype == torch.float16 and Y.is_contiguous(),
+             "Y must be a contiguous fp16 [M, N] and A_q must have the layer's K")
+    _require(workspace.is_contiguous(), "the workspace must be contiguous")
     _check(load().mixllm_gemm_w4w8a8_small_m(_ptr(A_q), _ptr(s_a), M, K, _ptr(p.W4), _ptr(p.z4), _ptr(p.s_w4),
                                              _ptr(p.idx4), p.N4, _ptr(p.W8), _ptr(p.s_w8), _ptr(p.idx8), p.N8,
                                              _ptr(Y), _ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -284,7 +294,8 @@ def gemm_w4w8a8_small_m_noalloc_into(A_q, s_a, p: PackedLinear, Y, stream=None):
     no allocation); calls must not overlap in time on one device."""
     _need_cuda(A_q, s_a, Y)
     M, K = A_q.shape
-    assert K == p.K and Y.shape == (M, p.N) and Y.dtype == torch.float16 and Y.is_contiguous()
+    _require(K == p.K and tuple(Y.shape) == (M, p.N) and Y.dtype == torch.float16 and Y.is_contiguous(),
+             "Y must be a contiguous fp16 [M, N] and A_q must have the layer's K")
     _check(load().mixllm_gemm_w4w8a8_small_m_noalloc(_ptr(A_q), _ptr(s_a), M, K, _ptr(p.W4), _ptr(p.z4),
                                                      _ptr(p.s_w4), _ptr(p.idx4), p.N4, _ptr(p.W8), _ptr(p.s_w8),
                                                      _ptr(p.idx8), p.N8, _ptr(Y), _stream(stream)),
