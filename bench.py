@@ -210,7 +210,7 @@ def run_reference(args, layer, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic", "config": config_of(layer, world),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "host_cores": os.cpu_count(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -417,7 +417,7 @@ def run_ours(args, layer, rank, world, local_rank):
         cpu = None
         if world == 1:
             rate, secs, rows = oracle_rate(layer, X, W, is8, args.cpu_seconds)
-            cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
+            cpu = {"value": rate, "unit": UNIT, "cores": 1, "host_cores": os.cpu_count(), "kind": "oracle",
                    "sample": f"{rows} token rows (cycling over the {layer.M}-row batch) x all {layer.N} "
                              f"channels x K={layer.K}, quantize + two-step GEMM, {secs:.1f} s single-threaded"}
         line = {
@@ -659,7 +659,7 @@ def run_search(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "achieved": sal_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": sal_gbs / peaks["hbm_gbs"], "traffic": None,
                      "peak_source": f"{peak_src} HBM copy {peaks['hbm_gbs']} GB/s", "algorithmic_bytes": sal_bytes},
-        "cpu_baseline": {"value": cpu_gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": cpu_gbs, "unit": "GB/s", "cores": 1, "host_cores": os.cpu_count(), "kind": "oracle",
                          "sample": f"{rows} channels of the 4096 x 4096 layer x {D} samples, fp64, {secs:.2f} s"},
         "e2e": {"value": step_bytes / (t_e2e * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": sum(G.numel() * 4 for G in Gs), "d2h_bytes_per_step": n_all},

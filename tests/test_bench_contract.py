@@ -39,6 +39,7 @@ def test_reference_arm_prints_one_contract_line():
     assert d["config"]["workload"] == "llama3.1-8b_q_proj_p10_M512_N4096_K4096"
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert cb["host_cores"] >= cb["cores"]
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
