@@ -36,3 +36,4 @@ from ._lib import (  # noqa: F401
     sync_status,
     version,
 )
+from .packfile import load_packed, save_packed  # noqa: F401
