@@ -28,12 +28,15 @@ from . import _lib
 MAGIC = b"MIXLLMW1"
 FIELDS = ("W4", "z4", "s_w4", "idx4", "W8", "s_w8", "idx8")
 
-if sys.byteorder != "little":  # the buffers are written in host order
-    raise ImportError("the packed-weight file format assumes a little-endian host")
+def _little_endian_host():
+    # the buffers are written and read in host order
+    if sys.byteorder != "little":
+        raise RuntimeError("the packed-weight file format needs a little-endian host")
 
 
 def save_packed(p: _lib.PackedLinear, path: str) -> None:
     """Write `p` (device or host tensors) to `path`."""
+    _little_endian_host()
     with open(path, "wb") as f:
         f.write(MAGIC)
         f.write(struct.pack("<5q", p.N, p.K, p.N4, p.N8, _lib.GROUP))
@@ -46,6 +49,7 @@ def save_packed(p: _lib.PackedLinear, path: str) -> None:
 
 def load_packed(path: str, device="cuda") -> _lib.PackedLinear:
     """Read a file written by save_packed into tensors on `device`."""
+    _little_endian_host()
     with open(path, "rb") as f:
         if f.read(len(MAGIC)) != MAGIC:
             raise ValueError(f"{path}: not a packed W4.4A8 weight file")
