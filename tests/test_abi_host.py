@@ -189,3 +189,36 @@ def test_small_m_workspace_plan(L):
     assert ws(8, 100, 100, 10)[0] == _lib.ERR_UNSUPPORTED
     null = L.mixllm_small_m_workspace_bytes(8, 4096, 100, 10, None)
     assert null == _lib.ERR_INVALID_ARG
+
+
+def test_header_is_plain_c_and_links_from_c(tmp_path):
+    """The boundary is a C ABI: a strict C99 program includes the header,
+    links against the library and calls its host-only entry points."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    src = tmp_path / "use_abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "mixllm.h"
+int main(void) {
+  size_t sizes[7];
+  if (mixllm_version() <= 0) return 1;
+  if (mixllm_packed_sizes(4096, 4096, 410, 128, sizes) != MIXLLM_OK) return 2;
+  if (mixllm_packed_sizes(4096, 4096, 410, 64, sizes) != MIXLLM_ERR_UNSUPPORTED) return 3;
+  if (mixllm_last_error()[0] == '\0') return 4;
+  printf("%zu\n", sizes[0]);
+  return 0;
+}
+''')
+    exe = tmp_path / "use_abi"
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", inc, str(src), "-o", str(exe),
+                        _lib.LIB_PATH, "-Wl,-rpath," + libdir], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, (r.returncode, r.stderr)
+    assert int(r.stdout) == _lib.packed_sizes(4096, 4096, 410)[0]
