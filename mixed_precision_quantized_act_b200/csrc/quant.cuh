@@ -7,7 +7,6 @@
 // (weights packed and interleaved offline so no permutation runs at run time).
 #pragma once
 
-#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cstdint>
 
@@ -19,35 +18,32 @@ namespace mixllm {
 // ---------------------------------------------------------------------------
 // Activation quantization.  One half-warp per (token m, group g): 16 lanes x
 // 8 fp16 = the 128 values of the group, loaded as one 16-byte vector per lane.
-// amax over the group, s_a = bf16(amax / 127) (IEEE division in fp32, then
-// rounded to bfloat16 precision and kept as fp32), q = clamp(round_half_even(
-// x / s_a), -127, 127); amax == 0 gives s_a = q = 0.  The bf16 scale keeps the
-// RTN error within s_a/2 and makes 1.5*2^23*s_a exact for the GEMM epilogue.
+// amax over the group, s_a = amax / 127 (IEEE division in fp32, kept as fp32),
+// q = clamp(round_half_even(x / s_a), -127, 127) with x / s_a the IEEE fp32
+// quotient; amax == 0 gives s_a = q = 0.
 //
-// The codes are those of rint(fl(x / s_a)), the plain CPU evaluation of the
-// definition, without a division per element:
-//   * fl(x/s) never crosses or lands on a half-integer k + 1/2 unless x/s is
-//     exactly k + 1/2: with x = mx 2^a (fp16, |mx| < 2^11) and s = ms 2^b
-//     (bf16, 2^7 <= ms < 2^8), x/s - (k + 1/2) = (mx 2^(a+1) - (2k+1) ms 2^b)
-//     / (2 ms 2^b) is, when non-zero, at least 2^-12 in magnitude for every
-//     |x/s| >= 1/2 (smaller quotients round to 0 either way), far above the
-//     2^-17 that fl() can move a quotient below 128.  So rint(fl(x/s)) is
-//     round_half_even of the exact quotient.
-//   * That is computed from q0 = rint(x * (1/s)), which is off by at most one,
-//     and the remainder e = x - q0*s, which one FMA gives exactly (q0*s has at
-//     most 15 significant bits and e is a multiple of the smaller of the two
-//     operands' last places, below 2^13 of them): |e| < s/2 keeps q0, |e| >
-//     s/2 moves q0 one step toward e, |e| = s/2 is a tie and picks the even one.
+// The codes are those of rint(fl(x / s)), the plain CPU evaluation of the
+// definition, with an IEEE division only for the rare element that needs it:
+//   * q0 = rint(x * (1/s)) is within one of rint(x/s): the product is off
+//     from the quotient by at most ~2^-23 of it (below 2^-16 for |x/s| < 128);
+//   * e = fma(-q0, s, x) = x - q0*s exactly: x is an fp16 value and q0*s has
+//     at most 8 + 24 significant bits; when q0 != 0, |x| >= s/2 puts x's last
+//     place above s's, so e is a multiple of s's last place and below s in
+//     magnitude -- 24 bits suffice;
+//   * the exact quotient is q0 + e/s.  fl(x/s) differs from it by at most half
+//     an ulp, 2^-18 for quotients below 128, so rint(fl(x/s)) = rint(x/s)
+//     unless the quotient lies within 2^-18 of a half-integer.  Away from
+//     those (| |e| - s/2 | > 2^-14 s, a wide margin) the code is q0, or q0
+//     moved one step toward e when |e| > s/2; within the margin (rare for real
+//     data, every tie case of the tests) the element takes the IEEE division.
 // ---------------------------------------------------------------------------
 // One group of 128 activations held eight per lane by the 16 lanes of `mask`
 // (MLSys 2026 talk notes on MixLLM, notes.yuuk.io, §設計判断の概要: 8-bit
-// symmetric, group-wise RTN): s_a = bf16(amax / 127) (IEEE division), codes
+// symmetric, group-wise RTN): s_a = amax / 127 (IEEE division), codes
 // rne(x / s_a) clamped to +-127 (an all-zero group gives s_a = 0 and zero
-// codes).  x / s_a is rounded exactly: q0 = rint(x * (1/s)), e = fma(-q0, s, x)
-// is exact (x fp16, s bf16), and q0 moves by one when |e| > s/2 (or = s/2
-// with q0 odd), which is rne(fl(x / s)) for these operands.  `raw`: the
-// lane's eight fp16 values; the codes are returned packed, lowest k first;
-// returns s_a.  Shared by quantize_act_kernel and the fused decode GEMV.
+// codes), computed as described above.  `raw`: the lane's eight fp16 values;
+// the codes are returned packed, lowest k first; returns s_a.  Shared by
+// quantize_act_kernel and the fused decode GEMV.
 __device__ __forceinline__ float quant_act_8x16(const uint4 raw, unsigned mask, uint32_t (&packed)[2]) {
   const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw);
   float x[8];
@@ -62,18 +58,23 @@ __device__ __forceinline__ float quant_act_8x16(const uint4 raw, unsigned mask, 
   for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(mask, amax, o));
-  const float s = __bfloat162float(__float2bfloat16_rn(__fdiv_rn(amax, 127.0f)));
+  const float s = __fdiv_rn(amax, 127.0f);
   packed[0] = packed[1] = 0u;
   if (s != 0.0f) {
     const float r = __frcp_rn(s);
     const float half_s = 0.5f * s;
+    const float margin = s * 0x1p-14f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int q0 = __float2int_rn(x[i] * r);
       const float e = __fmaf_rn(-static_cast<float>(q0), s, x[i]);  // exact remainder x - q0*s
-      const float ae = fabsf(e);
-      int qi = q0;
-      if (ae > half_s || (ae == half_s && (q0 & 1))) qi += e > 0.0f ? 1 : -1;
+      const float d = fabsf(e) - half_s;
+      int qi;
+      if (fabsf(d) > margin) {
+        qi = d > 0.0f ? q0 + (e > 0.0f ? 1 : -1) : q0;
+      } else {
+        qi = __float2int_rn(__fdiv_rn(x[i], s));  // near a half-integer: the IEEE quotient, rounded
+      }
       qi = max(-127, min(127, qi));
       packed[i >> 2] |= (static_cast<uint32_t>(qi) & 0xFFu) << ((i & 3) * 8);
     }

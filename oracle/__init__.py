@@ -51,9 +51,6 @@ def configure(L):
     L.oracle_f32_to_f16.argtypes = [ctypes.c_float]
     L.oracle_f32_to_f16_array.argtypes = [vp, i64, vp]
     L.oracle_f16_to_f32_array.argtypes = [vp, i64, vp]
-    L.oracle_round_bf16.restype = ctypes.c_float
-    L.oracle_round_bf16.argtypes = [ctypes.c_float]
-    L.oracle_round_bf16_array.argtypes = [vp, i64, vp]
     L.oracle_i2f_bias.restype = ctypes.c_float
     L.oracle_i2f_bias.argtypes = [ctypes.c_int32]
     L.oracle_i2f_mismatches.restype = i64
@@ -102,14 +99,6 @@ def f16_to_f32(h) -> np.ndarray:
     return out
 
 
-def round_bf16(x) -> np.ndarray:
-    """fp32 values rounded (RNE) to bfloat16 precision, returned as fp32."""
-    x = _c(x, np.float32)
-    out = np.empty(x.shape, np.float32)
-    lib().oracle_round_bf16_array(_p(x), x.size, _p(out))
-    return out
-
-
 def i2f_bias(p: int) -> float:
     return lib().oracle_i2f_bias(int(p))
 
@@ -121,7 +110,7 @@ def i2f_mismatches(lo: int, hi: int) -> int:
 # ---------------------------------------------------------------- quantizers
 
 def quantize_act(X: np.ndarray):
-    """X fp16 [M, K] -> (A_q int8 [M, K], s_a fp32 [M, K/128], bf16-valued)."""
+    """X fp16 [M, K] -> (A_q int8 [M, K], s_a fp32 [M, K/128])."""
     X = _c(X, np.float16)
     M, K = X.shape
     assert K % GROUP == 0

@@ -24,11 +24,10 @@
  *     and converted with f32_to_f16_rne / f16_to_f32 below.
  *
  * Readings of points the pages leave open (each one is also a test pin):
- *   R1 activation scale s_a = bf16(amax/127): the quotient in fp32, rounded
- *      to bfloat16 precision (8 significant bits, fp32 range) and carried as
- *      an fp32 value; q = clamp(rne(x/s_a), -127, 127); an all-zero group gets
- *      s_a = 0 and q = 0.  The pages give no dtype for this scale; bf16 keeps
- *      the rounding error of RTN within s_a/2 and makes 1.5*2^23*s_a exact.
+ *   R1 activation scale s_a = amax/127, the IEEE fp32 quotient, kept as fp32;
+ *      q = clamp(rne(x/s_a), -127, 127) with x/s_a the IEEE fp32 quotient; an
+ *      all-zero group gets s_a = 0 and q = 0.  The pages give no dtype for this
+ *      scale; fp32 is the plainest reading of "8-bit symmetric RTN".
  *   R2 4-bit asymmetric: lo = min(0, min w), hi = max(0, max w);
  *      s = fp16(min((hi-lo)/15, 65504)); if s == 0 the group is all zero
  *      (q = z = 0); else z = clamp(rne(-lo/s), 0, 15),
@@ -110,26 +109,7 @@ uint16_t oracle_f32_to_f16(float f)
     return (uint16_t)(sign | (uint16_t)n);
 }
 
-/* binary32 -> bfloat16 precision, round to nearest, ties to even, returned
- * as a binary32 value (the upper 16 bits of the result are the bf16 bits).
- * Written from the format: keep the sign, the 8 exponent bits and the top 7
- * fraction bits; round on the 16 bits dropped. */
-float oracle_round_bf16(float f)
-{
-    if (isnan(f) || isinf(f) || f == 0.0f) return f;
-    uint32_t u = f32_bits(f);
-    uint32_t keep = u >> 16;             /* sign, exponent, 7 fraction bits */
-    uint32_t dropped = u & 0xFFFFu;
-    if (dropped > 0x8000u || (dropped == 0x8000u && (keep & 1u))) keep += 1u;  /* may carry into exponent */
-    return bits_f32(keep << 16);
-}
-
-/* Array forms of the conversions (for the tests). */
-void oracle_round_bf16_array(const float *x, int64_t n, float *out)
-{
-    for (int64_t i = 0; i < n; ++i) out[i] = oracle_round_bf16(x[i]);
-}
-
+/* Array form of the conversion (for the tests). */
 void oracle_f32_to_f16_array(const float *x, int64_t n, uint16_t *out)
 {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_f32_to_f16(x[i]);
@@ -183,7 +163,7 @@ void oracle_quantize_act(const uint16_t *X, int64_t M, int64_t K,
                 float v = fabsf(oracle_f16_to_f32(x[i]));
                 if (v > amax) amax = v;
             }
-            float s = oracle_round_bf16(amax / 127.0f);
+            float s = amax / 127.0f;
             s_a[m * G + g] = s;
             for (int i = 0; i < ORACLE_GROUP; ++i) {
                 int q = 0;

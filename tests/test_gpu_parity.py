@@ -92,8 +92,8 @@ def test_quantize_act_special_values(dev):
 
 
 def _tie_groups():
-    """Groups whose scale is known exactly (amax = 127 * s0, s0 bf16-valued and
-    127 * s0 fp16-valued), filled with the exact half-integer multiples
+    """Groups whose scale is known exactly (amax = 127 * s0 with 127 * s0
+    fp16-valued, so s_a = s0), filled with the exact half-integer multiples
     (k + 1/2) * s0 that fp16 holds and with their fp16 neighbours on both sides:
     rounding ties and the values that must not be taken for ties."""
     rows = []

@@ -22,9 +22,9 @@ MUTATIONS = {
         "float scale = oracle_f16_to_f32(s4[n * G + g]) * s_a[m * G];"),
     "truncate_instead_of_round": ("float r = nearbyintf(oracle_f16_to_f32(x[i]) / s);",
                                   "float r = truncf(oracle_f16_to_f32(x[i]) / s);"),
-    "scale_divisor_128": ("oracle_round_bf16(amax / 127.0f)", "oracle_round_bf16(amax / 128.0f)"),
-    "scale_not_rounded_to_bf16": ("float s = oracle_round_bf16(amax / 127.0f);", "float s = amax / 127.0f;"),
-    "bf16_truncates": ("if (dropped > 0x8000u || (dropped == 0x8000u && (keep & 1u))) keep += 1u;", ""),
+    "scale_divisor_128": ("float s = amax / 127.0f;", "float s = amax / 128.0f;"),
+    "scale_rounded_to_fp16": ("float s = amax / 127.0f;", "float s = oracle_f16_to_f32(oracle_f32_to_f16(amax / 127.0f));"),
+    "scale_as_reciprocal_product": ("float s = amax / 127.0f;", "float s = amax * (1.0f / 127.0f);"),
     "f16_ties_away": ("float r = nearbyintf(units); /* ties to even */",
                       "float r = floorf(units + 0.5f);"),
     "w8_operand_shift": ("p += (int32_t)q[i] * (int32_t)a[i];",
@@ -47,9 +47,10 @@ MUTATIONS = {
 
 def _pins():
     yield pins.test_f32_to_f16_matches_ieee_rne, ()
-    yield pins.test_round_bf16_matches_torch, ()
     yield pins.test_act_quant_invariants, ()
     yield pins.test_act_quant_ties_half_even_and_zero_group, ()
+    yield pins.test_act_quant_scale_keeps_full_precision, ()
+    yield pins.test_act_quant_scale_is_correctly_rounded, ()
     yield pins.test_act_quant_lossless_grid, ()
     yield pins.test_w4_invariants, ()
     yield pins.test_w4_lossless_grid_and_special_groups, ()

@@ -56,25 +56,6 @@ def test_f32_to_f16_matches_ieee_rne(oracle_mod):
     assert np.array_equal(got, ref)
 
 
-def test_round_bf16_matches_torch(oracle_mod):
-    """The bf16 rounding of the activation scale: RNE to 8 significant bits,
-    checked against torch's float32 -> bfloat16 conversion."""
-    import torch
-    rng = np.random.default_rng(11)
-    parts = [rng.standard_normal(200000).astype(np.float32) * np.float32(50.0),
-             (rng.standard_normal(50000) * 1e-30).astype(np.float32),
-             np.array([0.0, -0.0, 1.0, 3.4e38, -3.4e38, np.inf, -np.inf, 1e-45, 2.0 ** -126], np.float32)]
-    # exact ties between adjacent bf16 values
-    b = (np.arange(0x3F00, 0x4100, dtype=np.uint32) << 16)
-    lo = b.view(np.float32).astype(np.float64)
-    hi = ((b + 0x10000).view(np.float32)).astype(np.float64)
-    parts.append(((lo + hi) / 2).astype(np.float32))
-    x = np.concatenate(parts)
-    got = oracle_mod.round_bf16(x)
-    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float32).numpy()
-    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
-
-
 # ------------------------------------------------------------ fast I2F
 
 def test_i2f_bias_exhaustive_window(oracle_mod, golden):
@@ -107,11 +88,11 @@ def test_act_quant_invariants(oracle_mod):
     assert np.all(np.abs(a).max(axis=2) == 127)  # amax maps to +-127
     err = np.abs(x - s[:, :, None].astype(np.float64) * a)
     assert np.all(err <= s[:, :, None] * 0.5 * (1 + 1e-5))  # + rounding of x/s
-    # the scale is amax/127 (fp32 quotient) rounded to bfloat16 precision
-    import torch
-    amax = np.abs(x).max(axis=2)
-    q = torch.from_numpy((amax / np.float32(127.0)).astype(np.float32))
-    assert np.array_equal(s, q.to(torch.bfloat16).to(torch.float32).numpy())
+    # the scale carries amax at fp32 precision: 127 * s_a gives back amax to
+    # within the rounding of the quotient and of the product (a scale rounded
+    # to bf16 or fp16, or a divisor other than 127, misses by far more)
+    amax = np.abs(x).max(axis=2).astype(np.float64)
+    assert np.all(np.abs(127.0 * s.astype(np.float64) - amax) <= amax * 2.0 ** -23)
 
 
 def test_act_quant_ties_half_even_and_zero_group(oracle_mod):
@@ -119,10 +100,68 @@ def test_act_quant_ties_half_even_and_zero_group(oracle_mod):
     x[0, 0] = 127.0        # amax = 127 -> s_a = 1 exactly
     x[0, 1:9] = [2.5, 3.5, -2.5, 0.5, 1.5, -1.5, 126.5, -0.5]
     A, s = oracle_mod.quantize_act(x)
-    assert s[0, 0] == 1.0  # 127/127, exact in bf16
+    assert s[0, 0] == 1.0  # 127/127
     assert list(A[0, 1:9]) == [2, 4, -2, 0, 2, -2, 126, 0]
     assert s[0, 1] == 0.0 and np.all(A[0, 128:] == 0)   # all-zero group
     assert s[1, 0] == 0.0 and np.all(A[1] == 0)
+
+
+def test_act_quant_scale_keeps_full_precision(oracle_mod):
+    """amax = 100 gives s_a = 100/127 = 0.78740157..., which needs all 24 bits
+    of an fp32 significand.  The codes of the values k * (100/127) (their fp16
+    roundings) must come back as k for every k: the fp16 rounding moves each
+    value by at most 2^-11 of itself, far less than half a step, so the
+    quantizer must return k exactly whatever the precision of its arithmetic,
+    and s_a itself must be the fp32 quotient to the bit (checked against a
+    decimal expansion of 100/127 computed here)."""
+    from fractions import Fraction
+    ks = np.arange(-127, 128)
+    vals = np.array([float(Fraction(100, 127) * int(k)) for k in ks])
+    x = np.zeros((1, 256), np.float16)
+    x[0, 0] = 100.0
+    x[0, 1:1 + len(ks) - 1] = vals[np.arange(len(ks)) != 227].astype(np.float16)  # 227 -> k = 100: amax itself
+    A, s = oracle_mod.quantize_act(x[:, :256].reshape(1, 256)[:, :256])
+    s0 = s[0, 0]
+    # the correctly rounded fp32 value of 100/127, from exact rationals
+    exact = Fraction(100, 127)
+    cand = [np.float32(float(exact)), np.nextafter(np.float32(float(exact)), np.float32(0)),
+            np.nextafter(np.float32(float(exact)), np.float32(2))]
+    best = min(cand, key=lambda c: abs(Fraction(float(c)) - exact))
+    assert s0 == best
+    assert A[0, 0] == 127
+    got = A[0, 1:len(ks)].astype(np.int64)
+    want = ks[np.arange(len(ks)) != 227]
+    assert np.array_equal(got, want)
+
+
+def _rn_f32(fr):
+    """The fp32 value nearest to the rational fr (ties to even), by exact arithmetic."""
+    from fractions import Fraction
+    f = np.float32(float(fr))  # within one ulp of fr
+    cands = [np.nextafter(f, np.float32(-np.inf)), f, np.nextafter(f, np.float32(np.inf))]
+    errs = [abs(Fraction(float(c)) - fr) for c in cands]
+    m = min(errs)
+    best = [c for c, e in zip(cands, errs) if e == m]
+    if len(best) > 1:  # a tie: the even significand
+        best = [c for c in best if (np.array(c, np.float32).view(np.uint32) & 1) == 0]
+    return best[0]
+
+
+def test_act_quant_scale_is_correctly_rounded(oracle_mod):
+    """s_a is amax/127 correctly rounded to fp32 for every group: checked
+    against exact rational arithmetic over 3000 fp16 values of amax (random
+    bit patterns plus the extremes of the fp16 range)."""
+    from fractions import Fraction
+    rng = np.random.default_rng(21)
+    bits = rng.integers(0x0001, 0x7C00, size=3000).astype(np.uint16)
+    bits[:4] = [0x0001, 0x03FF, 0x0400, 0x7BFF]  # smallest subnormal, largest subnormal, smallest normal, 65504
+    amax = bits.view(np.float16)
+    X = np.zeros((len(amax), 128), np.float16)
+    X[:, 5] = amax
+    X[:, 9] = -amax / np.float16(3)
+    _, s = oracle_mod.quantize_act(X)
+    want = np.array([_rn_f32(Fraction(float(a)) / 127) for a in amax], np.float32)
+    assert np.array_equal(s[:, 0].view(np.uint32), want.view(np.uint32))
 
 
 def test_act_quant_lossless_grid(oracle_mod):
