@@ -88,13 +88,12 @@ MIXLLM_API mixllm_status mixllm_packed_sizes(int64_t N, int64_t K, int64_t N8, i
 
 /*
  * Activation quantization (one kernel): for every token m and group g of
- * 128 columns, amax = max |x|, s_a = amax / 127 (fp32, IEEE division)
- * rounded to bfloat16 precision (8 significant bits, kept as an fp32 value),
- * A_q = clamp(round_half_even(x / s_a), -127, 127); a group whose amax is 0
- * gets s_a = 0 and A_q = 0.  (Talk notes §設計判断の概要: activations 8-bit
- * symmetric, group-wise RTN; the rounding mode and the scale precision are
- * this library's reading -- the pages give neither.  With a bf16 scale the
- * RTN error stays within s_a/2 and the GEMM's bias term 1.5*2^23*s_a is exact.)
+ * 128 columns, amax = max |x|, s_a = amax / 127 (fp32, IEEE division),
+ * A_q = clamp(round_half_even(x / s_a), -127, 127) with x / s_a the IEEE fp32
+ * quotient; a group whose amax is 0 gets s_a = 0 and A_q = 0.  (Talk notes
+ * §設計判断の概要: activations 8-bit symmetric, group-wise RTN; the rounding
+ * mode and the fp32 scale are this library's reading -- the pages give
+ * neither.)
  *   X_f16  device, fp16 [M, K] row-major, 16-byte aligned, read only
  *   A_q    device, int8 [M, K] row-major, 16-byte aligned, written
  *   s_a    device, fp32 [M, K/128] row-major, 4-byte aligned, written
@@ -143,9 +142,10 @@ MIXLLM_API mixllm_status mixllm_pack_weights(const float *W, int64_t N, int64_t 
  * output channel n of a set and token m,
  *   P_g = sum_{k in group g} (W_q[n,k] - z[n,g]) * A_q[m,k]   (int32 exact,
  *         z = 0 for the 8-bit set; int8 tensor cores, tcgen05 kind::i8),
- *   acc = sum_g float(P_g) * s_a[m,g] * s_w[n,g]  (fp32; float(P_g) by the
- *         0x4b400000 bias trick, exact for |P_g| <= 2^22; the product with
- *         s_a is correctly rounded, then accumulated with an FMA by s_w),
+ *   acc = sum_g float(P_g) * s_w[n,g] * s_a[m,g]  (fp32, groups in K order;
+ *         float(P_g) by the 0x4b400000 bias trick, exact for |P_g| <= 2^22,
+ *         and folded into one FMA that rounds P_g * s_w once; that product
+ *         is then accumulated with an FMA by s_a),
  *   Y[m, idx[n]] = fp16_rn(acc).
  * Arguments:
  *   A_q, s_a   device, as written by mixllm_quantize_act (A_q 16-byte
@@ -181,6 +181,23 @@ MIXLLM_API mixllm_status mixllm_gemm_debug_partials(const int8_t *A_q, const flo
                                          const int8_t *W8, const void *s_w8_f16,
                                          const int32_t *idx8, int64_t N8,
                                          int32_t *P, void *stream);
+
+/*
+ * The same GEMM as mixllm_gemm_w4w8a8 with one step done the plain way: the
+ * int32 partials are converted to float by the int -> float convert
+ * instruction, and the tensor-memory accumulator is not preset to the
+ * 0x4b400000 bias.  MLSys 2026 talk notes on MixLLM, §高速 I2F 変換, measure
+ * what the bias trick gains over this (on A100); this entry point exists to
+ * measure the same on B200.  The converted value is exact (|P_g| < 2^24), so
+ * fl(float(P_g) * s_w) equals the bias-trick FMA and Y is bit-identical to
+ * mixllm_gemm_w4w8a8's.  Same arguments, rules and errors.
+ */
+MIXLLM_API mixllm_status mixllm_gemm_w4w8a8_plain_i2f(const int8_t *A_q, const float *s_a, int64_t M, int64_t K,
+                                 const uint8_t *W4, const uint8_t *z4, const void *s_w4_f16,
+                                 const int32_t *idx4, int64_t N4,
+                                 const int8_t *W8, const void *s_w8_f16,
+                                 const int32_t *idx8, int64_t N8,
+                                 void *Y_f16, void *stream);
 
 /*
  * Bytes of workspace mixllm_gemm_w4w8a8_small_m needs for this shape (0 when

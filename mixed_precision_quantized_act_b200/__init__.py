@@ -15,6 +15,7 @@ from ._lib import (  # noqa: F401
     channel_salience,
     channel_salience_into,
     gemm_w4w8a8_into,
+    gemm_w4w8a8_plain_i2f_into,
     gemm_w4w8a8_small_m,
     gemm_w4w8a8_small_m_noalloc_into,
     gemm_w4w8a8_small_m_into,

@@ -33,6 +33,8 @@ SIGNATURES = {
                                           _vp, _vp, _vp, _i64, _vp, _vp]),
     "mixllm_gemm_debug_partials": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64,
                                                   _vp, _vp, _vp, _i64, _vp, _vp]),
+    "mixllm_gemm_w4w8a8_plain_i2f": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64,
+                                                    _vp, _vp, _vp, _i64, _vp, _vp]),
     "mixllm_small_m_workspace_bytes": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(ctypes.c_size_t)]),
     "mixllm_small_m_kernel": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(ctypes.c_int32)]),
     "mixllm_channel_salience": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i64, _vp, _vp]),
@@ -204,6 +206,18 @@ def gemm_w4w8a8_into(A_q, s_a, p: PackedLinear, Y, stream=None):
     _check(load().mixllm_gemm_w4w8a8(_ptr(A_q), _ptr(s_a), M, K, _ptr(p.W4), _ptr(p.z4), _ptr(p.s_w4),
                                      _ptr(p.idx4), p.N4, _ptr(p.W8), _ptr(p.s_w8), _ptr(p.idx8), p.N8,
                                      _ptr(Y), _stream(stream)), "mixllm_gemm_w4w8a8")
+
+
+def gemm_w4w8a8_plain_i2f_into(A_q, s_a, p: PackedLinear, Y, stream=None):
+    """The fused GEMM with a plain int -> float convert instead of the bias
+    trick (the ablation the talk notes' fast-I2F section measures); same Y."""
+    _need_cuda(A_q, s_a, Y)
+    M, K = A_q.shape
+    _require(K == p.K and tuple(Y.shape) == (M, p.N) and Y.dtype == torch.float16 and Y.is_contiguous(),
+             "Y must be a contiguous fp16 [M, N] and A_q must have the layer's K")
+    _check(load().mixllm_gemm_w4w8a8_plain_i2f(_ptr(A_q), _ptr(s_a), M, K, _ptr(p.W4), _ptr(p.z4), _ptr(p.s_w4),
+                                               _ptr(p.idx4), p.N4, _ptr(p.W8), _ptr(p.s_w8), _ptr(p.idx8), p.N8,
+                                               _ptr(Y), _stream(stream)), "mixllm_gemm_w4w8a8_plain_i2f")
 
 
 def gemm_w4w8a8(A_q, s_a, p: PackedLinear, stream=None) -> torch.Tensor:

@@ -632,9 +632,6 @@ SmallMPlan plan_small_m(int64_t M, int64_t N4, int64_t N8, int64_t K) {
   return p;
 }
 
-static bool encode_groups_3d(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *map, const void *W8, int64_t K,
-                             int64_t N8, int box_rows, int groups_per_box);
-
 template <int MP>
 static cudaError_t launch_small_m_mp(const GemmArgs &a, const SmallMPlan &p, void *ws, cudaStream_t stream,
                                      const char **msg) {
@@ -699,41 +696,6 @@ static cudaError_t launch_small_m_mp(const GemmArgs &a, const SmallMPlan &p, voi
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) *msg = "launch of the small-M GEMM failed";
   return e;
-}
-
-// An int8 [rows, K] matrix (W8 [N8, K], or A_q [M, K]) as a 3-D tensor (k
-// within a group, row, group) with 128 x box_rows x groups_per_box boxes:
-// whole groups of a block of rows, each 128-byte row swizzled.  Encodings are
-// cached by (base, K, rows, box).
-static bool encode_groups_3d(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *map, const void *W8, int64_t K,
-                             int64_t N8, int box_rows, int groups_per_box) {
-  struct Entry {
-    const void *base;
-    int64_t K, N8;
-    int rows, gpb;
-    bool valid;
-    CUtensorMap map;
-  };
-  static Entry table[32];
-  static int next = 0;
-  static std::mutex mu;
-  std::lock_guard<std::mutex> lock(mu);
-  for (const Entry &e : table)
-    if (e.valid && e.base == W8 && e.K == K && e.N8 == N8 && e.rows == box_rows && e.gpb == groups_per_box) {
-      *map = e.map;
-      return true;
-    }
-  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(N8), static_cast<cuuint64_t>(K / 128)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K), 128};  // bytes, dims 1 and 2
-  const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(groups_per_box)};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(W8), dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return false;
-  table[next] = Entry{W8, K, N8, box_rows, groups_per_box, true, *map};
-  next = (next + 1) % 32;
-  return true;
 }
 
 template <int MT, bool FUSE = false>

@@ -8,56 +8,66 @@
 //     acc += float(P_g) * s_w[n,g] * s_a[m,g]      fp32
 //   then Y[m, idx[n]] = fp16(acc).
 //
-// How it runs on B200 (one CTA of 16 warps per 128 x BN output tile, both
-// channel sets in the same launch, warp-specialized, registers rebalanced
-// with setmaxnreg toward the epilogue):
-// The weights are the MMA's A operand (the tile's BN channels are the TMEM
-// lanes of the accumulator) and the activations its B operand (kBM tokens are
-// the accumulator's columns).
+// How it runs on B200.  A tile is 128 output channels x 128 tokens.  The
+// weights are the MMA's A operand (the tile's channels are the TMEM lanes of
+// the accumulator) and the activations its B operand (the tokens are the
+// accumulator's columns).  The grid is persistent: CTA c of a channel set
+// takes that set's tiles c, c + C, c + 2C, ... (C = the set's CTA count), and
+// every role walks one running group index gi = (tile of this CTA) * G + g,
+// so the rings run on across tile boundaries and the next tile's first
+// groups are loaded and multiplied while the epilogue still drains the last
+// tile.  Both channel sets share the launch: the first CTAs take the 4-bit
+// tiles, the others the 8-bit ones (the rings are laid out per set).
+// 24 warps, warp-specialized, registers rebalanced with setmaxnreg toward the
+// epilogue:
 //   warp 0      TMA producer: the A_q tile [128 x 128] (128-byte swizzle) of
-//               every group -- together with the int8 weight tile [BN x 128]
-//               on 8-bit tiles -- into a ring of stages, and on 4-bit tiles
-//               the packed uint4 weight tile [BN x 64 B] (one contiguous 8 KB
-//               block per tile and group: a single bulk copy) and the group's
-//               zero points into a ring of their own.
+//               every group -- with the int8 weight tile on 8-bit tiles --
+//               into a ring of stages; on 4-bit tiles the packed uint4 weight
+//               tile (one contiguous 8 KiB block per tile and group) and the
+//               group's zero points into a ring of their own.
 //   warps 1, 3  one thread each issues the MMAs of alternate groups: 4 x
-//               tcgen05.mma.kind::i8 (K = 32 each) into one of kAccBufs int32
+//               tcgen05.mma.kind::i8 (K = 32 each) into one of two int32
 //               accumulators in tensor memory (TMEM), then one commit to the
-//               group's `done` barrier, which frees the A_q stage and unpacked
-//               buffer it read and hands the accumulator to the epilogue.  The
-//               MMA of later groups overlaps the SIMT work on earlier ones.
-//   warp 2      stages, per group, the channel scales s_w (fp32) and the token
-//               scales s_a of the tile in a small ring the epilogue reads.
-//   warps 12-15 4-bit set only: unpack nibbles and subtract the zero point in
-//               SWAR form (four bytes per 32-bit op, no borrow between bytes)
-//               -- the B200 counterpart of the pages' vsub4 pre-dequantization
-//               step (§ソフトウェアパイプライン) -- and store the int8 rows
-//               with tcgen05.st into a TMEM buffer, from which the MMA reads
-//               its A operand: the unpacked tile never touches shared memory,
-//               so the tensor core's shared-memory reads per group halve.
-//   warps 4-11  epilogue: tcgen05.ld a group's int32 partials, which the
-//               accumulator already holds biased by 0x4b400000 (TMEM is preset
-//               to the bias), so their bits read as float are 1.5*2^23 + P
-//               exactly for |P| <= 2^22 -- the bias trick with no integer add.
-//               The bias is folded into one FMA with the channel scale:
-//               u = fma(v, s_w, -1.5*2^23*s_w) = fl(P*s_w), one rounding,
-//               because 1.5*2^23*s_w is exact for an fp16-valued s_w; then
-//               acc = fma(u, s_a, acc): two f32x2 FMAs per pair of elements,
-//               one shared-memory load per four.  After the last group, fp16
-//               results are staged in shared memory and scattered row-wise to
-//               Y[:, idx] so each warp store covers a short run of one output
-//               row.
-// Every ring slot is refilled as soon as its own consumer is done with it (the
-// A stages and unpacked buffers through the group's `done` barrier, the packed
-// tiles through the unpack warps), and the rings are deep enough to cover the
-// load latency of HBM.  Every wait is bounded; on a timeout the CTA records
-// an error in the status word, drains its own copies and MMAs, frees TMEM and
-// exits.
+//               group's `done` barrier, which frees the A_q stage and the
+//               unpacked weight buffer and hands the accumulator over.
+//   warp 2      stages per group the channel scales ({s_w, s_w, -1.5*2^23*s_w,
+//               same} per channel, fp32) and the token scales s_a of the tile
+//               in a small ring the epilogue reads.
+//   warps 4-19  epilogue, four warps per TMEM lane quadrant (so four per SM
+//               sub-partition: while one waits on a TMEM load the others keep
+//               the FMA pipe busy), 32 token columns each: tcgen05.ld of the
+//               group's int32 partials, which the accumulator holds biased by
+//               0x4b400000 (TMEM is preset to the bias and refilled with it
+//               after every drain), so their bits read as float are
+//               1.5*2^23 + P exactly for |P| <= 2^22 -- the bias trick with no
+//               integer add.  The bias is folded into one FMA with the channel
+//               scale: u = fma(v, s_w, -1.5*2^23*s_w) = fl(P*s_w), one
+//               rounding, since 1.5*2^23*s_w is exact for an fp16-valued s_w;
+//               then acc = fma(u, s_a, acc); both as f32x2 FMAs.  The running
+//               sums stay in registers; after the tile's last group each
+//               thread writes its 32 fp16 outputs straight to Y[m, idx[n]]
+//               (a warp store covers 32 channels of one token row).
+//   warps 20-23 4-bit set only: unpack the nibbles and subtract the zero
+//               point in SWAR form (four bytes per 32-bit op, no borrow
+//               between bytes) -- the B200 counterpart of the pages' vsub4
+//               pre-dequantization (§ソフトウェアパイプライン) -- and store the
+//               int8 rows with tcgen05.st into a TMEM buffer, from which the
+//               MMA reads its A operand.
+// Every ring slot is refilled as soon as its own consumer is done with it.
+// Every wait is bounded; on a timeout the CTA records an error in the status
+// word, drains its own copies and MMAs, frees TMEM and exits.
+//
+// kCvtI2F (measurement only): the same kernel with the int32 partials
+// converted by the plain int -> float instruction: the accumulator is preset
+// to 0 instead of the bias (the same refill after every drain), so the two
+// variants differ in the conversion alone; fl(float(P)*s_w) is the same
+// value as the bias-trick FMA, so both give identical Y.
 #pragma once
 
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
+#include <atomic>
 #include <cstdint>
 #include <mutex>
 
@@ -66,79 +76,102 @@
 
 namespace mixllm {
 
-constexpr int kBM = 128;         // tile rows (tokens) = TMEM lanes
-constexpr int kKG = 128;         // K per group = K per pipeline stage
-constexpr int kThreads = 512;    // 16 warps = 4 warpgroups
-constexpr int kEpiWarps = 8;     // warps 4..11
+constexpr int kBM = 128;          // tile tokens = accumulator columns
+constexpr int kKG = 128;          // K per group = K per pipeline stage
+// Epilogue warps: 16 (32 token columns each, 24 warps in all) or, with
+// MIXLLM_EPI_WARPS=8, 8 (64 columns each, 16 warps, twice the registers).
+#ifndef MIXLLM_EPI_WARPS
+#define MIXLLM_EPI_WARPS 8
+#endif
+constexpr int kEpiWarps = MIXLLM_EPI_WARPS;  // warps 4 .. 3 + kEpiWarps
+static_assert(kEpiWarps == 8 || kEpiWarps == 16, "epilogue warps");
+constexpr int kThreads = 32 * (8 + kEpiWarps);
 constexpr int kEpiThreads = kEpiWarps * 32;
-constexpr int kXformWarps = 4;   // warps 12..15
+constexpr int kXformWarp0 = 4 + kEpiWarps;  // the four unpack warps
+constexpr int kXformWarps = 4;
 constexpr float kI2FBias = 12582912.0f;     // 1.5 * 2^23, the float with bits 0x4b400000
 constexpr uint32_t kI2FBiasBits = 0x4B400000u;
-// register split (all four warpgroups together must stay within 65536):
-// 128 * (kRegsCtl + kRegsXform) + 256 * kRegsEpi <= 512 * 128 (the launch's registers)
-constexpr int kRegsCtl = 88, kRegsXform = 72, kRegsEpi = 176;
-static_assert(128 * (kRegsCtl + kRegsXform) + 256 * kRegsEpi <= 65536, "register split");
+// Registers: the launch gets kRegsLaunch per thread (768 x 80 = 61440); the
+// warpgroups then rebalance with setmaxnreg within that pool.
+constexpr int kRegsLaunch = kEpiWarps == 16 ? 80 : 128;
+constexpr int kRegsCtl = kEpiWarps == 16 ? 40 : 56, kRegsXform = kEpiWarps == 16 ? 56 : 80;
+constexpr int kRegsEpi = kEpiWarps == 16 ? 96 : 184;
+static_assert(128 * (kRegsCtl + kRegsXform) + kEpiThreads * kRegsEpi <= kThreads * kRegsLaunch, "register split");
+static_assert(kThreads * kRegsLaunch <= 65536, "register file");
 
 template <int BN>
 struct GemmCfg {
   static_assert(BN == 128, "the warp roles below are laid out for BN = 128");
   static constexpr int kABytes = kBM * kKG;        // 16 KB A_q tile of one group
-  static constexpr int kW8Bytes = BN * kKG;        // 16 KB int8 weight tile
-  static constexpr int kW4Bytes = BN * kKG / 2;    //  8 KB packed uint4 weight tile
+  static constexpr int kW8Bytes = BN * kKG;        // 16 KB int8 weight tile of one group
+  static constexpr int kW4Bytes = BN * kKG / 2;    //  8 KB packed uint4 weight tile of one group
   static constexpr int kZBytes = BN / 2;           // zero points of one group, two per byte
-  // The ring region is laid out one of two ways, chosen per CTA:
-  //   8-bit tile: kStages8 stages of [A | W8]                      (32 KB each)
-  //   4-bit tile: kStagesA4 A stages and kRaw packed tiles          (16/8 KB)
-  // The unpacked 4-bit tiles live in tensor memory (kTBufs buffers of 32
-  // columns), where the MMA reads its weight operand: they take no shared
-  // memory and no shared-memory bandwidth.
-  static constexpr int kStages8 = 6;
-  static constexpr int kStagesA4 = 8;
-  static constexpr int kTBufs = 8;
-  static constexpr int kRaw = 8;
-  static constexpr int kMaxStages = kStages8 > kStagesA4 ? kStages8 : kStagesA4;
-  // Two threads issue the MMAs of alternate groups.  Every barrier an issuer
-  // waits on must belong to one issuer only, or a parity wait could see a
-  // phase meant for the other one: the slot counts of those rings are even.
-  static_assert(kStages8 % 2 == 0 && kStagesA4 % 2 == 0 && kTBufs % 2 == 0, "rings the issuers wait on");
-  // One commit per group, to done[g % kDone]; a waiter never falls a full ring
-  // behind as long as kDone covers every ring that is released through it.
-  static constexpr int kDone = kMaxStages > kTBufs ? kMaxStages : kTBufs;
-  static constexpr int kRing8 = kStages8 * (kABytes + kW8Bytes);
-  static constexpr int kRing4 = kStagesA4 * kABytes + kRaw * kW4Bytes;
-  static constexpr int kRingBytes = kRing8 > kRing4 ? kRing8 : kRing4;
+  // Operands arrive in chunks of several groups: a stage holds a chunk's
+  // A_q tiles (one 3-D box: k, token, group) and its weights (4-bit: the
+  // packed tiles of consecutive groups, contiguous, one bulk copy, and their
+  // zero points, one 2-D box; 8-bit: one 3-D box), all on one barrier.  On
+  // B200 a thread that issues copies completes about one such round every
+  // ~350-450 ns whatever its size, and stalls meanwhile, so one dedicated
+  // thread issues one round per chunk: per-group rounds of 8-16 KiB would
+  // bound a group at that time.
+  static constexpr int kC4 = 4, kC8 = 3;  // groups per chunk: 4-bit, 8-bit tiles
+  static constexpr int kStages = 2;
+  static constexpr int kStage4 = kC4 * (kABytes + kW4Bytes);  // 96 KiB
+  static constexpr int kStage8 = kC8 * (kABytes + kW8Bytes);  // 96 KiB
+  static constexpr int kRingBytes = kStages * (kStage4 > kStage8 ? kStage4 : kStage8);
+  static constexpr int kTBufs = 8;   // unpacked 4-bit tiles in TMEM, 32 columns each
+  // Two threads issue the MMAs of alternate groups.  A barrier waited by one
+  // issuer only must have an even slot count (the unpacked buffers, the
+  // accumulators); the chunk barriers are waited by both, which is safe
+  // because a chunk's slot is refilled only after the MMAs of all its groups,
+  // by both issuers, have completed.
+  static_assert(kTBufs % 2 == 0, "rings one issuer waits on");
+  // One commit per group, to done[gi % kDone]: no waiter can fall a whole
+  // ring behind as long as kDone covers every ring released through it.
+  static constexpr int kDone = 8;
+  static_assert(kDone >= kStages * kC4 && kDone >= kStages * kC8 && kDone >= kTBufs, "done ring");
   static constexpr int kAccBufs = 2;
-  static_assert(kAccBufs % 2 == 0, "accumulators alternate between the issuers");
-  static_assert(kDone >= kStages8 && kDone >= kStagesA4 && kDone >= kTBufs && kDone >= kAccBufs, "done ring");
-  static constexpr int kTabSlots = 4;
+  // The scale table: a slot holds kTabG consecutive groups, so the epilogue
+  // waits for it, and releases it, once per kTabG groups.
+  static constexpr int kTabG = 4, kTabSlots = 2;
   // tensor memory: kAccBufs int32 accumulators of kBM (token) columns, then
   // the unpacked weight tiles, 128 bytes of K per lane = 32 columns each
   static constexpr int kTmemABase = kAccBufs * kBM;
   static constexpr int kTmemABufCols = kKG / 4;
   static constexpr int kTmemCols = 512;
   static_assert(kTmemABase + kTBufs * kTmemABufCols <= kTmemCols, "tensor memory");
-  static constexpr int kColsPerThread = BN * kBM / kEpiThreads;  // 64
-  static constexpr int kTabSwBytes = BN * 4;                   // s_w of the tile's columns (fp32)
-  static constexpr int kTabBytes = kTabSwBytes + kBM * 4;      // + s_a of the tile's rows
-  static constexpr int kStgSlots = 12;                         // raw scale staging ring
-  static constexpr int kStgDist = 10;                          // groups prefetched ahead
-  static constexpr int kStgBytes = BN * 2 + kBM * 4;           // raw fp16 s_w + fp32 s_a
+  static constexpr int kColsPerThread = BN * kBM / kEpiThreads;  // token columns per epilogue thread
+  static_assert(kColsPerThread % 32 == 0, "the preset fills 32 columns at a time, the drain loads 16");
+  static constexpr int kTabWBytes = BN * 16;                      // {s_w, s_w, cb, cb} per channel
+  static constexpr int kTabBytes = kTabWBytes + kBM * 4;          // + s_a of the tile's tokens (one group)
+  static constexpr int kTabSlotBytes = kTabG * kTabBytes;
+  // Raw scales.  Vector path (G % 4 == 0, s_a 16-byte aligned): per chunk of
+  // kScG groups one 2-D box of s_w [kScG][BN] fp16 and one of s_a [kBM][kScG]
+  // fp32, into kScStages stages.  Fallback: a staging ring of kStgSlots
+  // single groups filled with cp.async, kStgDist groups ahead.
+  static constexpr int kScG = 4, kScStages = 3;
+  static constexpr int kScSwBytes = kScG * BN * 2, kScBytes = kScSwBytes + kBM * kScG * 4;
+  static constexpr int kStgSlots = 12;                            // raw scale staging ring
+  static constexpr int kStgDist = 10;                             // groups prefetched ahead
+  static constexpr int kStgBytes = BN * 2 + kBM * 4;              // raw fp16 s_w + fp32 s_a
+  static constexpr int kStgArea = kScStages * kScBytes > kStgSlots * kStgBytes ? kScStages * kScBytes
+                                                                                : kStgSlots * kStgBytes;
   // shared-memory layout (offsets from a 1024-byte aligned base)
   static constexpr int kOffRing = 0;
   static constexpr int kOffZ = kOffRing + kRingBytes;
-  static constexpr int kOffTab = kOffZ + kRaw * kZBytes;
-  static constexpr int kOffStg = kOffTab + kTabSlots * kTabBytes;
-  static constexpr int kOffIdx = kOffStg + kStgSlots * kStgBytes;  // output channel of each tile column
-  static constexpr int kOffBar = kOffIdx + BN * 4;
-  // full per stage, done per group ring, full/empty per packed tile, full per unpacked buffer,
-  // empty per accumulator, full/empty per table slot, one drain per issuer
-  static constexpr int kNumBars = kMaxStages + kDone + 2 * kRaw + kTBufs + kAccBufs + 2 * kTabSlots + 2;
+  static constexpr int kOffTab = kOffZ + kStages * kC4 * kZBytes;
+  static constexpr int kOffStg = kOffTab + kTabSlots * kTabSlotBytes;
+  static constexpr int kOffBar = kOffStg + kStgArea;
+  // full per stage, done per group ring, full per unpacked buffer, empty
+  // per accumulator, full/empty per table slot, one drain per issuer, full
+  // per raw scale stage
+  static constexpr int kNumBars = kStages + kDone + kTBufs + kAccBufs + 2 * kTabSlots + 2 + kScStages;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;
-  static constexpr int kStagingStride = (BN + 2) * 2;  // bytes per staged fp16 row
-  static_assert(kBM * kStagingStride <= kRingBytes, "staging must fit in the ring region");
-  static_assert(kABytes % 1024 == 0 && kW8Bytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+  static_assert(kABytes % 1024 == 0 && kW8Bytes % 1024 == 0 && kW4Bytes % 1024 == 0, "1024-byte aligned tiles");
+  static_assert(kTabBytes % 16 == 0 && kStgBytes % 16 == 0 && kOffTab % 16 == 0 && kOffStg % 128 == 0, "alignment");
+  static_assert(kScBytes % 128 == 0 && kScSwBytes % 128 == 0, "TMA destinations");
   static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
 };
 
@@ -148,86 +181,176 @@ __device__ __forceinline__ uint32_t sub_zero_bytes(uint32_t w, uint32_t zz) {
   return ((w | 0x80808080u) - zz) ^ 0x80808080u;
 }
 
-template <int BN, bool kDebugP>
+// The persistent schedule of one CTA: which channel set, and which tiles.
+struct TileSched {
+  bool is4;
+  int first, stride, count;  // tiles first, first + stride, ... of the set (count of them)
+  __device__ __forceinline__ TileSched(int cta, int c4, int c8, int T4, int T8) {
+    is4 = cta < c4;
+    first = is4 ? cta : cta - c4;
+    stride = is4 ? c4 : c8;
+    const int T = is4 ? T4 : T8;
+    count = first < T ? (T - first + stride - 1) / stride : 0;
+  }
+  __device__ __forceinline__ int tile(int tl) const { return first + tl * stride; }
+};
+
+// Walks a CTA's chunks in order without dividing per step (a runtime
+// division compiles to a dozen instructions, several on the XU pipe; every
+// role advances its cursors once per group or chunk).  Chunk: up to CH
+// consecutive groups of one tile, starting at group g0 of the tile and at
+// running group index gi0.
+struct ChunkCursor {
+  int tl, c, g0, ng, gi0, m0, n0;
+  __device__ __forceinline__ void start(const TileSched &sc, int G, int CH, int mt, int BN) {
+    tl = c = g0 = gi0 = 0;
+    ng = G < CH ? G : CH;
+    tile(sc, mt, BN);
+  }
+  __device__ __forceinline__ void tile(const TileSched &sc, int mt, int BN) {
+    if (tl < sc.count) {
+      const int t = sc.tile(tl);
+      m0 = (t % mt) * kBM;
+      n0 = (t / mt) * BN;
+    }
+  }
+  __device__ __forceinline__ void next(const TileSched &sc, int G, int CH, int nch, int mt, int BN) {
+    gi0 += ng;
+    g0 += CH;
+    if (++c == nch) {
+      c = 0;
+      g0 = 0;
+      ++tl;
+      tile(sc, mt, BN);
+    }
+    ng = G - g0 < CH ? G - g0 : CH;
+  }
+};
+
+// Walks groups: running index gi, group g of tile tl, chunk ci (running) and
+// position j inside the chunk.
+struct GroupCursor {
+  int gi, g, tl, ci, j;
+  __device__ __forceinline__ void start() { gi = g = tl = ci = j = 0; }
+  __device__ __forceinline__ void next(int G, int CH) {
+    ++gi;
+    ++j;
+    if (++g == G) {
+      g = 0;
+      j = 0;
+      ++tl;
+      ++ci;
+    } else if (j == CH) {
+      j = 0;
+      ++ci;
+    }
+  }
+};
+
+template <int BN, bool kDebugP, bool kCvtI2F>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_w4w8a8_kernel(const __grid_constant__ CUtensorMap tmA, const uint8_t *__restrict__ W4,
-                       const __grid_constant__ CUtensorMap tmW8, const float *__restrict__ s_a,
-                       const uint8_t *__restrict__ z4, const __half *__restrict__ s_w4,
+    gemm_w4w8a8_kernel(const __grid_constant__ CUtensorMap tmA4, const __grid_constant__ CUtensorMap tmA8,
+                       const uint8_t *__restrict__ W4, const __grid_constant__ CUtensorMap tmW8,
+                       const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmSa,
+                       const __grid_constant__ CUtensorMap tmSw4, const __grid_constant__ CUtensorMap tmSw8, int vec_scales,
+                       const float *__restrict__ s_a, const __half *__restrict__ s_w4,
                        const int32_t *__restrict__ idx4, const __half *__restrict__ s_w8,
                        const int32_t *__restrict__ idx8, int M, int K, int N4, int N8, int N4p, int N8p, int mt,
-                       int nt4, __half *__restrict__ Y, int32_t *__restrict__ P) {
+                       int T4, int T8, int c4, int c8, __half *__restrict__ Y, int32_t *__restrict__ P) {
   using C = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
-  uint64_t *full = bars;                          // TMA -> MMA              (per stage)
-  uint64_t *done = full + C::kMaxStages;          // MMA commit of group g   (ring of kDone): frees the
-                                                  // group's A stage and unpacked buffer, fills its accumulator
-  uint64_t *rfull = done + C::kDone;              // TMA -> unpack           (per packed tile)
-  uint64_t *rempty = rfull + C::kRaw;             // unpack -> TMA           (per packed tile)
-  uint64_t *tfull = rempty + C::kRaw;             // unpack -> MMA           (per unpacked buffer)
-  uint64_t *accempty = tfull + C::kTBufs;         // epilogue -> MMA         (per TMEM accumulator)
-  uint64_t *tabfull = accempty + C::kAccBufs;     // scale warp -> epilogue  (per table slot)
+  uint64_t *full = bars;                          // chunk landed                (per stage)
+  uint64_t *done = full + C::kStages;             // MMA commit of group gi      (ring of kDone): frees the
+                                                  // group's stages and unpacked buffer, fills its accumulator
+  uint64_t *tfull = done + C::kDone;              // unpack -> MMA               (per unpacked buffer)
+  uint64_t *accempty = tfull + C::kTBufs;         // epilogue -> MMA             (per TMEM accumulator)
+  uint64_t *tabfull = accempty + C::kAccBufs;     // scale warp -> epilogue      (per table slot)
   uint64_t *tabempty = tabfull + C::kTabSlots;    // epilogue -> scale warp
   uint64_t *drain = tabempty + C::kTabSlots;      // [2]: each MMA issuer's final commit
+  uint64_t *scfull = drain + 2;                   // raw scale chunk landed  (per raw scale stage)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x;
-  const bool is4 = tile < mt * nt4;
-  const int t = is4 ? tile : tile - mt * nt4;
-  const int m0 = (t % mt) * kBM;
-  const int n0 = (t / mt) * BN;
+  const TileSched sched(static_cast<int>(blockIdx.x), c4, c8, T4, T8);
+  const bool is4 = sched.is4;
   const int G = K >> 7;
+  const int total = sched.count * G;  // groups this CTA runs
   const int Nset = is4 ? N4 : N8;
   const int Np = is4 ? N4p : N8p;
   const int N = N4 + N8;
   const __half *s_w = is4 ? s_w4 : s_w8;
   const int32_t *idx = is4 ? idx4 : idx8;
-  const int S = is4 ? C::kStagesA4 : C::kStages8;  // A stages of this tile
-
-  // ring region: 8-bit tiles [A | W8] x kStages8; 4-bit tiles A x kStagesA4, then the packed tiles
-  const int stage_bytes = is4 ? C::kABytes : C::kABytes + C::kW8Bytes;
+  // chunking of this CTA's set: CH groups per chunk, kStages stages of [A_q tiles | weights]
+  const int CH = is4 ? C::kC4 : C::kC8;
+  constexpr int S = C::kStages;
+  const int nch = (G + CH - 1) / CH;       // chunks per tile (the last may hold fewer groups)
+  const int nchunks = sched.count * nch;   // chunks this CTA loads
+  const int a_bytes = CH * C::kABytes;
+  const int stage_bytes = is4 ? C::kStage4 : C::kStage8;
   auto stage_a = [&](int s) { return smem + C::kOffRing + s * stage_bytes; };
-  auto stage_w8 = [&](int s) { return smem + C::kOffRing + s * stage_bytes + C::kABytes; };
-  auto raw_w4 = [&](int r) { return smem + C::kOffRing + C::kStagesA4 * C::kABytes + r * C::kW4Bytes; };
-  auto zmeta = [&](int r) { return smem + C::kOffZ + r * C::kZBytes; };
-  auto table = [&](int slot) { return reinterpret_cast<float4 *>(smem + C::kOffTab + slot * C::kTabBytes); };
-  auto table_sw = [&](int slot) { return reinterpret_cast<const float *>(smem + C::kOffTab + slot * C::kTabBytes); };
-  auto table_sa = [&](int slot) {
-    return reinterpret_cast<float *>(smem + C::kOffTab + slot * C::kTabBytes + C::kTabSwBytes);
+  auto stage_w = [&](int s) { return smem + C::kOffRing + s * stage_bytes + a_bytes; };
+  auto zmeta = [&](int s) { return smem + C::kOffZ + s * C::kC4 * C::kZBytes; };
+  // table entry of running group gi: slot (gi / kTabG) % kTabSlots, place gi % kTabG
+  auto table_w = [&](int gi) {
+    return reinterpret_cast<float4 *>(smem + C::kOffTab + ((gi / C::kTabG) % C::kTabSlots) * C::kTabSlotBytes +
+                                      (gi % C::kTabG) * C::kTabBytes);
   };
+  auto table_sa = [&](int gi) { return reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(table_w(gi)) + C::kTabWBytes); };
   auto stg_sw = [&](int i) { return smem + C::kOffStg + i * C::kStgBytes; };
   auto stg_sa = [&](int i) { return reinterpret_cast<float *>(smem + C::kOffStg + i * C::kStgBytes + BN * 2); };
-  int32_t *col_idx = reinterpret_cast<int32_t *>(smem + C::kOffIdx);
-
-  // Loads of the A ring (and of W8 on 8-bit tiles) for group g into stage g % S.
-  const uint32_t a_bytes = static_cast<uint32_t>(is4 ? C::kABytes : C::kABytes + C::kW8Bytes);
-  auto load_a = [&](int g) {
-    const int s = g % S;
-    mbar_arrive_expect_tx(&full[s], a_bytes);
-    tma_load_2d(stage_a(s), &tmA, &full[s], g * kKG, m0);
-    if (!is4) tma_load_2d(stage_w8(s), &tmW8, &full[s], g * kKG, n0);
+  // Chunk `k` (a cursor) into stage k.c_run % S, one round on full[]: the
+  // A_q tiles (one 3-D box: 128 k x 128 tokens x CH groups; groups past G
+  // read as zeros and are never multiplied), then the packed 4-bit tiles of
+  // its ng groups (one contiguous bulk copy) and their zero points (one 2-D
+  // box), or the 8-bit tiles (one 3-D box).
+  const CUtensorMap *tmA = is4 ? &tmA4 : &tmA8;
+  auto load_chunk = [&](const ChunkCursor &k, int ci) {
+    const int s = ci % S;
+    if (is4) {
+      const uint32_t wb = static_cast<uint32_t>(k.ng * C::kW4Bytes);
+      mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(a_bytes) + wb + static_cast<uint32_t>(C::kC4 * C::kZBytes));
+      tma_load_3d(stage_a(s), tmA, &full[s], 0, k.m0, k.g0);
+      bulk_load(stage_w(s), W4 + (static_cast<int64_t>(k.n0 >> 7) * G + k.g0) * C::kW4Bytes, wb, &full[s]);
+      tma_load_2d(zmeta(s), &tmZ, &full[s], k.n0 >> 1, k.g0);
+    } else {
+      mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(2 * a_bytes));
+      tma_load_3d(stage_a(s), tmA, &full[s], 0, k.m0, k.g0);
+      tma_load_3d(stage_w(s), &tmW8, &full[s], 0, k.n0, k.g0);
+    }
   };
-  // Loads of the packed 4-bit tile and zero points of group g into slot g % kRaw.
-  auto load_raw = [&](int g) {
-    const int r = g % C::kRaw;
-    mbar_arrive_expect_tx(&rfull[r], static_cast<uint32_t>(C::kW4Bytes + C::kZBytes));
-    // the tile's packed group is one contiguous block: one bulk copy
-    bulk_load(raw_w4(r), W4 + (static_cast<int64_t>(n0 >> 7) * G + g) * C::kW4Bytes, C::kW4Bytes, &rfull[r]);
-    bulk_load(zmeta(r), z4 + static_cast<int64_t>(g) * (N4p >> 1) + (n0 >> 1), C::kZBytes, &rfull[r]);
+  // The producer: stage ci % S is refilled with chunk ci once the MMAs of
+  // chunk ci - S are done -- the commits of its last two groups (one per
+  // issuer) cover all of them.  Blocking (suspending) waits, so the thread
+  // takes no issue slots from the warps of its SM sub-partition meanwhile.
+  auto produce = [&](ChunkCursor &k, int first) {
+    ChunkCursor rel;
+    rel.start(sched, G, CH, mt, BN);
+    int ci = first;
+    for (; ci < nchunks; ++ci) {
+      const int gl = rel.gi0 + rel.ng - 1;
+      if (!mbar_wait(&done[gl % C::kDone], (gl / C::kDone) & 1, abort_flag)) break;
+      if (rel.ng > 1 && !mbar_wait(&done[(gl - 1) % C::kDone], ((gl - 1) / C::kDone) & 1, abort_flag)) break;
+      load_chunk(k, ci);
+      k.next(sched, G, CH, nch, mt, BN);
+      rel.next(sched, G, CH, nch, mt, BN);
+    }
+    return ci;
   };
+  // let the copies of the last stages land before the CTA can exit
+  auto drain_ring = [&](int issued) {
+    for (int ci = (issued > S ? issued - S : 0); ci < issued; ++ci)
+      (void)mbar_wait_drain(&full[ci % S], (ci / S) & 1, 1ll << 26);
+  };
+  ChunkCursor pk;  // the producer's next chunk (thread 0)
 
   if (threadIdx.x == 0) {
-    prefetch_tmap(&tmA);
-    if (!is4) prefetch_tmap(&tmW8);
-    for (int s = 0; s < C::kMaxStages; ++s) mbar_init(&full[s], 1);
+    prefetch_tmap(tmA);
+    prefetch_tmap(is4 ? &tmZ : &tmW8);
+    for (int s = 0; s < C::kStages; ++s) mbar_init(&full[s], 1);
     for (int i = 0; i < C::kDone; ++i) mbar_init(&done[i], 1);
-    for (int r = 0; r < C::kRaw; ++r) {
-      mbar_init(&rfull[r], 1);
-      mbar_init(&rempty[r], kXformWarps);
-    }
     for (int b = 0; b < C::kTBufs; ++b) mbar_init(&tfull[b], kXformWarps);
     for (int a = 0; a < C::kAccBufs; ++a) mbar_init(&accempty[a], kEpiWarps);
     for (int i = 0; i < C::kTabSlots; ++i) {
@@ -236,13 +359,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
+    for (int s = 0; s < C::kScStages; ++s) mbar_init(&scfull[s], 1);
     *abort_flag = 0;
     fence_mbar_init();
-    // Every global read of this grid comes after this wait: here, in the
-    // table warp, and in the roles ordered after these loads by barriers.
+    // Every global read of this grid comes after a pdl_wait: here, in the
+    // scale warp and the epilogue, and in the roles ordered after these
+    // loads by barriers.
     pdl_wait();
     // the first stages need nothing but their barriers: start them before the CTA-wide sync
-    for (int g = 0; g < S && g < G; ++g) load_a(g);
+    pk.start(sched, G, CH, mt, BN);
+    for (int ci = 0; ci < S && ci < nchunks; ++ci) {
+      load_chunk(pk, ci);
+      pk.next(sched, G, CH, nch, mt, BN);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
@@ -256,53 +385,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     regs_dec<kRegsCtl>();
     if (warp == 0) {
-      // ---------------------------------------------------------- TMA producer
-      // One thread feeds both rings: the A stages (with W8 on 8-bit tiles),
-      // each refilled once the MMAs of the group that held it are done, and on
-      // 4-bit tiles the packed W4 tiles, each refilled once unpacked.  It
-      // polls both, so neither ring waits on the other.  (L2 prefetch hints
-      // ahead of the rings measured slower: they compete with the loads for
-      // the TMA unit's requests.)
-      if (lane == 0) {
-        int ga = S < G ? S : G;  // next A group; the prologue issued groups 0 .. S-1
-        int gw = is4 ? 0 : G;    // next packed W4 group
-        long long idle_since = -1;
-        while (ga < G || gw < G) {
-          bool progressed = false;
-          // packed slot gw % kRaw last held group gw - kRaw; the unpack warps released it
-          if (gw < G &&
-              (gw < C::kRaw || mbar_try_wait(smem_u32(&rempty[gw % C::kRaw]), ((gw / C::kRaw) - 1) & 1))) {
-            load_raw(gw);
-            ++gw;
-            progressed = true;
-          }
-          // A stage ga % S last held group ga - S; it is free once that group is done
-          if (ga < G && mbar_try_wait(smem_u32(&done[(ga - S) % C::kDone]), ((ga - S) / C::kDone) & 1)) {
-            load_a(ga);
-            ++ga;
-            progressed = true;
-          }
-          if (progressed) {
-            idle_since = -1;
-            continue;
-          }
-          if (*abort_flag) break;
-          const long long now = clock64();
-          if (idle_since < 0) {
-            idle_since = now;
-          } else if (now - idle_since > (1ll << 32)) {
-            *abort_flag = 1;
-            record_status(kStatusTimeout);
-            break;
-          }
-          __nanosleep(64);
-        }
-        // let every copy this thread issued land before the CTA can exit
-        for (int g = (ga > S ? ga - S : 0); g < ga; ++g) (void)mbar_wait_drain(&full[g % S], (g / S) & 1, 1ll << 26);
-        if (is4)
-          for (int g = (gw > C::kRaw ? gw - C::kRaw : 0); g < gw; ++g)
-            (void)mbar_wait_drain(&rfull[g % C::kRaw], (g / C::kRaw) & 1, 1ll << 26);
-      }
+      // ---------------------------------------------------------- producer
+      if (lane == 0) drain_ring(produce(pk, S < nchunks ? S : nchunks));
     } else if (warp == 1 || warp == 3) {
       // ---------------------------------------------------------- MMA issuers
       // Two threads issue alternate groups (warp 1 the even ones, warp 3 the
@@ -314,14 +398,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         constexpr uint32_t idesc = idesc_i8(BN, kBM);
         const int who = warp == 1 ? 0 : 1;
-        for (int g = who; g < G; g += 2) {
-          const int s = g % S, b = g % C::kTBufs, a = g % C::kAccBufs;
-          if (!mbar_wait(&full[s], (g / S) & 1, abort_flag)) break;
-          if (is4 && !mbar_wait(&tfull[b], (g / C::kTBufs) & 1, abort_flag)) break;
-          // phase 0 of accempty[a] is the epilogue's bias fill; phase u+1 its drain of use u
-          if (!mbar_wait(&accempty[a], (g / C::kAccBufs) & 1, abort_flag)) break;
+        GroupCursor gc;
+        gc.start();
+        if (who) gc.next(G, CH);
+        for (; gc.gi < total; gc.next(G, CH), gc.next(G, CH)) {
+          const int gi = gc.gi, ci = gc.ci, j = gc.j;
+          const int st = ci % S, b = gi % C::kTBufs, a = gi % C::kAccBufs;
+          if (!mbar_wait(&full[st], (ci / S) & 1, abort_flag)) break;
+          if (is4 && !mbar_wait(&tfull[b], (gi / C::kTBufs) & 1, abort_flag)) break;
+          // phase 0 of accempty[a] is the epilogue's initial fill; phase u+1 its drain of use u
+          if (!mbar_wait(&accempty[a], (gi / C::kAccBufs) & 1, abort_flag)) break;
           tc_fence_after();
-          const uint32_t x_addr = smem_u32(stage_a(s));
+          const uint32_t x_addr = smem_u32(stage_a(st) + j * C::kABytes);
           const uint32_t d = tmem_base + static_cast<uint32_t>(a * kBM);
           if (is4) {
             const uint32_t wt = tmem_base + static_cast<uint32_t>(C::kTmemABase + b * C::kTmemABufCols);
@@ -329,78 +417,145 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < kKG / 32; ++kk)
               mma_i8_ts(d, wt + 8 * kk, sw128_kmajor_desc(x_addr + 32 * kk), idesc, 1u);
           } else {
-            const uint32_t w_addr = smem_u32(stage_w8(s));
+            const uint32_t w_addr = smem_u32(stage_w(st) + j * C::kW8Bytes);
 #pragma unroll
             for (int kk = 0; kk < kKG / 32; ++kk)
-              mma_i8(d, sw128_kmajor_desc(w_addr + 32 * kk), sw128_kmajor_desc(x_addr + 32 * kk), idesc, 1u);
+              mma_i8(d, sw128_kmajor_desc(w_addr + 32 * kk), sw128_kmajor_desc(x_addr + 32 * kk), idesc,
+                     1u);
           }
-          mma_commit(&done[g % C::kDone]);
+          mma_commit(&done[gi % C::kDone]);
         }
         mma_commit(&drain[who]);
         (void)mbar_wait_drain(&drain[who], 0, 1ll << 28);
       }
     } else {
       // ---------------------------------------------------------- scale table
-      // Slot `slot` of group g holds s_w of the tile's BN columns as fp32,
-      // followed by s_a of the tile's 128 rows.  Raw scales are prefetched
-      // kStgDist groups ahead with cp.async into a staging ring, so no load
-      // latency sits on the epilogue's path.
-      auto issue = [&](int g) {
-        if (g < G) {
-          const int i = g % C::kStgSlots;
-          cp_async_8(stg_sw(i) + 8 * lane, s_w + static_cast<int64_t>(g) * Np + n0 + 4 * lane);
-#pragma unroll
-          for (int j = 0; j < kBM / 32; ++j) {
-            const int row = lane + 32 * j;
-            const bool in = m0 + row < M;
-            cp_async_4(stg_sa(i) + row, s_a + (in ? static_cast<int64_t>(m0 + row) * G + g : 0), in ? 4u : 0u);
-          }
-        }
-        cp_async_commit();
+      // The entry of group gi holds, per channel of the tile, the float4
+      // {s_w, s_w, -1.5*2^23*s_w, -1.5*2^23*s_w} (the f32x2 operands of the
+      // bias-folding FMA), then s_a of the tile's 128 tokens.  A slot of
+      // kTabG groups is waited free before its first group and published
+      // after its last (or after the CTA's last group).
+      auto slot_free = [&](int gi) {
+        return gi % C::kTabG != 0 ||
+               warp_wait(&tabempty[(gi / C::kTabG) % C::kTabSlots], ((gi / (C::kTabG * C::kTabSlots)) & 1) ^ 1,
+                         abort_flag);
       };
-      pdl_wait();
-      // The row scales of this tile are whole rows of s_a [M, G] (one
-      // contiguous range) and its column scales one 2*BN-byte piece per group:
-      // bring both into L2 first, so the scattered 4-byte reads below hit there.
-      if (lane == 0) {
-        const int rows = M - m0 < kBM ? M - m0 : kBM;
-        const uint32_t sa_bytes = static_cast<uint32_t>(rows) * static_cast<uint32_t>(G) * 4u;
-        const float *sa_rows = s_a + static_cast<int64_t>(m0) * G;  // s_a is only 4-byte aligned
-        if (sa_bytes >= 16 && (reinterpret_cast<uintptr_t>(sa_rows) & 15u) == 0) bulk_prefetch_l2(sa_rows, sa_bytes & ~15u);
-      }
-      for (int g = lane; g < G; g += 32) bulk_prefetch_l2(s_w + static_cast<int64_t>(g) * Np + n0, BN * 2);
-      for (int g = 0; g < C::kStgDist; ++g) issue(g);
-      // output channel of every tile column (-1 past the set), published to
-      // the epilogue by the first tabfull arrival
-#pragma unroll
-      for (int i = 0; i < BN / 32; ++i) {
-        const int col = lane + 32 * i;
-        col_idx[col] = n0 + col < Nset ? __ldg(idx + n0 + col) : -1;
-      }
-      for (int g = 0; g < G; ++g) {
-        const int slot = g % C::kTabSlots, i = g % C::kStgSlots;
-        cp_async_wait<C::kStgDist - 1>();
-        __syncwarp();
-        if (!warp_wait(&tabempty[slot], ((g / C::kTabSlots) & 1) ^ 1, abort_flag)) break;
-        const uint2 raw = *reinterpret_cast<const uint2 *>(stg_sw(i) + 8 * lane);
+      auto slot_done = [&](int gi) {
+        if (gi % C::kTabG == C::kTabG - 1 || gi == total - 1) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tabfull[(gi / C::kTabG) % C::kTabSlots]);
+        }
+      };
+      auto publish = [&](int gi, const uint8_t *raw_sw, const float *sa_src, int sa_stride) {
+        // raw_sw: the tile's BN fp16 s_w of this group; sa_src[t * sa_stride]: s_a of token t
+        const uint2 raw = *reinterpret_cast<const uint2 *>(raw_sw + 8 * lane);
         const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&raw.x));
         const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&raw.y));
-        table(slot)[lane] = make_float4(a.x, a.y, b.x, b.y);
-        float *tsa = table_sa(slot);
-        const float *ssa = stg_sa(i);
+        float4 *tw = table_w(gi) + 4 * lane;
+        const float sws[4] = {a.x, a.y, b.x, b.y};
 #pragma unroll
-        for (int j = 0; j < kBM / 32; ++j) tsa[lane + 32 * j] = ssa[lane + 32 * j];
+        for (int c = 0; c < 4; ++c) {
+          const float cb = kCvtI2F ? 0.0f : -kI2FBias * sws[c];
+          tw[c] = make_float4(sws[c], sws[c], cb, cb);
+        }
+        float *tsa = table_sa(gi);
+#pragma unroll
+        for (int j = 0; j < kBM / 32; ++j) tsa[lane + 32 * j] = sa_src[(lane + 32 * j) * sa_stride];
+      };
+      if (vec_scales) {
+        // Vector path: per chunk of kScG groups of a tile, one 2-D box of s_w
+        // and one of s_a land in a raw stage (one copy round for both), then
+        // each group is converted into its table slot.  G % kScG == 0, so the
+        // chunks never straddle a tile and gi = chunk * kScG + group.
+        const int nsc = total / C::kScG;
+        const CUtensorMap *tmSw = is4 ? &tmSw4 : &tmSw8;
+        auto sc_raw = [&](int st) { return smem + C::kOffStg + st * C::kScBytes; };
+        const int nscc = G / C::kScG;  // raw chunks per tile
+        auto load_sc = [&](const ChunkCursor &k, int c) {
+          const int st = c % C::kScStages;
+          mbar_arrive_expect_tx(&scfull[st], static_cast<uint32_t>(C::kScBytes));
+          tma_load_2d(sc_raw(st), tmSw, &scfull[st], k.n0, k.g0);
+          tma_load_2d(sc_raw(st) + C::kScSwBytes, &tmSa, &scfull[st], k.g0, k.m0);
+        };
+        ChunkCursor sk;  // next raw chunk to load (lane 0)
+        if (lane == 0) {
+          prefetch_tmap(&tmSa);
+          prefetch_tmap(tmSw);
+          pdl_wait();
+          sk.start(sched, G, C::kScG, mt, BN);
+          for (int c = 0; c < C::kScStages && c < nsc; ++c) {
+            load_sc(sk, c);
+            sk.next(sched, G, C::kScG, nscc, mt, BN);
+          }
+        }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tabfull[slot]);
-        issue(g + C::kStgDist);
+        int c = 0;
+        for (; c < nsc; ++c) {
+          const int st = c % C::kScStages;
+          if (!warp_wait(&scfull[st], (c / C::kScStages) & 1, abort_flag)) break;
+          bool ok = true;
+          for (int jg = 0; jg < C::kScG; ++jg) {
+            const int gi = c * C::kScG + jg;
+            if (!slot_free(gi)) {
+              ok = false;
+              break;
+            }
+            publish(gi, sc_raw(st) + jg * BN * 2,
+                    reinterpret_cast<const float *>(sc_raw(st) + C::kScSwBytes) + jg, C::kScG);
+            slot_done(gi);
+          }
+          if (!ok) break;
+          __syncwarp();
+          if (lane == 0 && c + C::kScStages < nsc) {  // the stage is read: refill it
+            load_sc(sk, c + C::kScStages);
+            sk.next(sched, G, C::kScG, nscc, mt, BN);
+          }
+        }
+        // let the raw copies still in flight land before the CTA can exit
+        if (lane == 0) {
+          const int issued = nsc < c + C::kScStages ? nsc : c + C::kScStages;
+          for (int cc = (issued > C::kScStages ? issued - C::kScStages : 0); cc < issued; ++cc)
+            (void)mbar_wait_drain(&scfull[cc % C::kScStages], (cc / C::kScStages) & 1, 1ll << 26);
+        }
+      } else {
+        // Fallback: raw scales prefetched kStgDist groups ahead with cp.async
+        // into a staging ring, one group per slot.
+        ChunkCursor ik;  // group gi of the lookahead, as a chunk of one group
+        ik.start(sched, G, 1, mt, BN);
+        auto issue = [&](int gi) {
+          if (gi < total) {
+            const int g = ik.g0, m0 = ik.m0, n0 = ik.n0;
+            ik.next(sched, G, 1, G, mt, BN);
+            const int i = gi % C::kStgSlots;
+            cp_async_8(stg_sw(i) + 8 * lane, s_w + static_cast<int64_t>(g) * Np + n0 + 4 * lane);
+#pragma unroll
+            for (int j = 0; j < kBM / 32; ++j) {
+              const int row = lane + 32 * j;
+              const bool in = m0 + row < M;
+              cp_async_4(stg_sa(i) + row, s_a + (in ? static_cast<int64_t>(m0 + row) * G + g : 0), in ? 4u : 0u);
+            }
+          }
+          cp_async_commit();
+        };
+        pdl_wait();
+        for (int gi = 0; gi < C::kStgDist; ++gi) issue(gi);
+        for (int gi = 0; gi < total; ++gi) {
+          const int i = gi % C::kStgSlots;
+          cp_async_wait<C::kStgDist - 1>();
+          __syncwarp();
+          if (!slot_free(gi)) break;
+          publish(gi, stg_sw(i), stg_sa(i), 1);
+          slot_done(gi);
+          issue(gi + C::kStgDist);
+        }
+        cp_async_wait<0>();
       }
-      cp_async_wait<0>();
     }
-  } else if (warp >= 12) {
+  } else if (warp >= kXformWarp0) {
     regs_dec<kRegsXform>();
-    // ------------------------------------------------------------ 4-bit unpack
     if (is4) {
-      // Warp 12 + q writes TMEM lane quadrant q: thread `lane` unpacks weight
+      // ---------------------------------------------------------- 4-bit unpack
+      // Warp 20 + q writes TMEM lane quadrant q: thread `lane` unpacks weight
       // row rr = 32q + lane of the tile (64 packed bytes -> 128 int8 values)
       // and stores it as the 32 columns of its lane in the group's buffer.
       // The packed rows are 64 bytes apart, so lanes read their four 16-byte
@@ -411,20 +566,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int rot = (lane >> 1) & 3;
       const int zshift = (rr & 1) * 4;
       const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + C::kTmemABase;
-      for (int g = 0; g < G; ++g) {
-        const int r = g % C::kRaw, b = g % C::kTBufs;
-        if (!warp_wait(&rfull[r], (g / C::kRaw) & 1, abort_flag)) break;
-        // buffer b last held group g - kTBufs: free once that group's MMAs are done
-        if (g >= C::kTBufs) {
-          const int gp = g - C::kTBufs;
+      GroupCursor gc;
+      gc.start();
+      for (; gc.gi < total; gc.next(G, CH)) {
+        const int gi = gc.gi, ci = gc.ci, j = gc.j;
+        const int r = ci % S, b = gi % C::kTBufs;
+        if (j == 0 && !warp_wait(&full[r], (ci / S) & 1, abort_flag)) break;
+        // buffer b last held group gi - kTBufs: free once that group's MMAs are done
+        if (gi >= C::kTBufs) {
+          const int gp = gi - C::kTBufs;
           if (!warp_wait(&done[gp % C::kDone], (gp / C::kDone) & 1, abort_flag)) break;
           tc_fence_after();
         }
-        const uint8_t *src = raw_w4(r) + rr * 64;
+        const uint8_t *src = stage_w(r) + j * C::kW4Bytes + rr * 64;
         uint4 x[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) x[c] = *reinterpret_cast<const uint4 *>(src + (((c + rot) & 3) << 4));
-        const uint32_t zz = ((static_cast<uint32_t>(zmeta(r)[rr >> 1]) >> zshift) & 0xFu) * 0x01010101u;
+        const uint32_t zz =
+            ((static_cast<uint32_t>(zmeta(r)[j * C::kZBytes + (rr >> 1)]) >> zshift) & 0xFu) * 0x01010101u;
         // x[c] holds chunk (c + rot) & 3: rotate back by rot = (rot & 1) + (rot & 2)
         if (rot & 1) {
           const uint4 t3 = x[3];
@@ -455,7 +614,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           o[8 * c + 7] = sub_zero_bytes((x[c].w >> 4) & 0x0F0F0F0Fu, zz);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&rempty[r]);  // the packed tile is in registers
         tmem_st_32x32b_x32(trow + static_cast<uint32_t>(b * C::kTmemABufCols), o);
         tmem_st_wait();
         tc_fence_before();
@@ -467,139 +625,153 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_inc<kRegsEpi>();
     // ------------------------------------------------------------ epilogue
     // The accumulator is D[channel, token]: this thread owns channel `ch` of
-    // the tile (its TMEM lane) and the tokens half*CPT .. half*CPT+CPT-1.
-    constexpr int CPT = C::kColsPerThread;  // 64 token columns per thread
-    const int e = warp - 4;                 // 0..7
-    const int quad = warp & 3;              // TMEM lane quadrant of this warp
-    const int half = e >> 2;                // column half
+    // the tile (its TMEM lane) and the tokens part*32 .. part*32+31.
+    constexpr int CPT = C::kColsPerThread;
+    const int e = warp - 4;                 // 0 .. kEpiWarps - 1
+    const int quad = warp & 3;              // TMEM lane quadrant of this warp (= its SM sub-partition)
+    const int part = e >> 2;                // which CPT-column part of the 128 tokens
     const int ch = quad * 32 + lane;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + part * CPT;
 
-    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + half * CPT;
-    // Every accumulator starts at the bias 0x4b400000 (and is reset to it after
-    // each drain), so the int32 sum the MMAs leave there, read as a float, is
-    // 1.5*2^23 + P exactly: the bias trick with no per-element integer add.
+    // Every accumulator starts at the bias 0x4b400000 (and is reset to it
+    // after each drain), so the int32 sum the MMAs leave there, read as a
+    // float, is 1.5*2^23 + P exactly (kCvtI2F: at 0, so it is P).
+    constexpr uint32_t kPreset = kCvtI2F ? 0u : kI2FBiasBits;
 #pragma unroll
     for (int a = 0; a < C::kAccBufs; ++a)
 #pragma unroll
-      for (int c = 0; c < CPT; c += 32) tmem_st_32x32b_x32_fill(lane_base + a * kBM + c, kI2FBiasBits);
+      for (int c = 0; c < CPT; c += 32) tmem_st_32x32b_x32_fill(lane_base + a * kBM + c, kPreset);
     tmem_st_wait();
     tc_fence_before();
     __syncwarp();
     if (lane == 0)
       for (int a = 0; a < C::kAccBufs; ++a) mbar_arrive(&accempty[a]);
+    pdl_wait();  // before the idx reads below
 
-    float acc[CPT];
+    float2 acc[CPT / 2];
 #pragma unroll
-    for (int j = 0; j < CPT; ++j) acc[j] = 0.0f;
-
-    // Software pipeline over 16-column chunks: while one chunk is converted
-    // and accumulated, the tcgen05.ld of the next one (this group's next
-    // chunk, or the next group's first) is in flight.
-    constexpr int CW = 16, NCH = CPT / CW;
-    uint32_t rbuf[2][CW];
-    // v = bits of (1.5*2^23 + P) as float; u = fma(v, s_w, -1.5*2^23*s_w) is
-    // exactly fl(P * s_w): the bias term 1.5*2^23*s_w is exact for an
-    // fp16-valued s_w and the fma rounds v*s_w - 1.5*2^23*s_w = P*s_w once.
-    // Then acc += u * s_a.  tab holds the s_a of 4 consecutive tokens per float4.
-    auto convert = [&](uint32_t(&r)[CW], const float4 *tab, float2 sw2, float2 cb2, int c0) {
-#pragma unroll
-      for (int j = 0; j < CW / 4; ++j) {
-        const float4 sa = tab[j];
-        const float2 v0 = make_float2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]));
-        const float2 v1 = make_float2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
-        const float2 u0 = __ffma2_rn(v0, sw2, cb2);
-        const float2 u1 = __ffma2_rn(v1, sw2, cb2);
-        const float2 o0 = __ffma2_rn(u0, make_float2(sa.x, sa.y), make_float2(acc[c0 + 4 * j], acc[c0 + 4 * j + 1]));
-        const float2 o1 =
-            __ffma2_rn(u1, make_float2(sa.z, sa.w), make_float2(acc[c0 + 4 * j + 2], acc[c0 + 4 * j + 3]));
-        acc[c0 + 4 * j] = o0.x;
-        acc[c0 + 4 * j + 1] = o0.y;
-        acc[c0 + 4 * j + 2] = o1.x;
-        acc[c0 + 4 * j + 3] = o1.y;
-      }
-    };
-    auto dump = [&](uint32_t(&r)[CW], int g, int c0) {
-      if (n0 + ch < Nset) {
-        const int64_t nout = idx[n0 + ch];
-#pragma unroll 4
-        for (int j = 0; j < CW; ++j) {
-          const int m = m0 + half * CPT + c0 + j;
-          if (m < M) P[(static_cast<int64_t>(m) * N + nout) * G + g] = static_cast<int32_t>(r[j] - kI2FBiasBits);
+    for (int j = 0; j < CPT / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
+    // 32-bit shared addresses of the barriers and tables this role touches
+    const uint32_t a_done = smem_u32(done);
+    const uint32_t a_accempty = smem_u32(accempty);
+    const uint32_t a_tabfull = smem_u32(tabfull);
+    const uint32_t a_tabempty = smem_u32(tabempty);
+    const uint32_t a_tab = smem_u32(smem + C::kOffTab);
+    bool live = true;
+    int gi = 0;  // running group index
+    for (int tl = 0; live && tl < sched.count; ++tl) {
+      const int t = sched.tile(tl);
+      const int m0 = (t % mt) * kBM;
+      const int n0 = (t / mt) * BN;
+      const int nout = n0 + ch < Nset ? __ldg(idx + n0 + ch) : -1;  // output column of this thread's channel
+      for (int g = 0; g < G; ++g, ++gi) {
+        const int a = gi % C::kAccBufs, tslot = (gi / C::kTabG) % C::kTabSlots;
+        const uint32_t col = lane_base + static_cast<uint32_t>(a * kBM);
+        if (!warp_wait_u32(a_done + 8 * (gi % C::kDone), (gi / C::kDone) & 1, abort_flag)) {
+          live = false;
+          break;
         }
-      }
-    };
-
-    bool live = warp_wait(&done[0], 0, abort_flag);
-    if (live) {
-      tc_fence_after();
-      tmem_ld_32x32b_x16(lane_base, rbuf[0]);
-    }
-    for (int g = 0; live && g < G; ++g) {
-      const int a = g % C::kAccBufs, slot = g % C::kTabSlots;
-      const uint32_t col = lane_base + static_cast<uint32_t>(a * kBM);
-      if (!warp_wait(&tabfull[slot], (g / C::kTabSlots) & 1, abort_flag)) break;
-      const float sw = table_sw(slot)[ch];
-      const float2 sw2 = make_float2(sw, sw);
-      const float2 cb2 = make_float2(-kI2FBias * sw, -kI2FBias * sw);
-      const float4 *tab = reinterpret_cast<const float4 *>(table_sa(slot)) + half * (CPT / 4);
+        tc_fence_after();
+        // The group is drained in CPT/16 chunks of 16 columns.  With 8
+        // epilogue warps (registers to spare) the next chunk's TMEM load is
+        // in flight while the current one is converted; with 16, one chunk's
+        // registers at a time.
+#ifndef MIXLLM_EPI_CW
+#define MIXLLM_EPI_CW 16
+#endif
+        constexpr int CW = CPT > 32 ? MIXLLM_EPI_CW : 16, NCH = CPT / CW;
+        constexpr bool kDB = CPT > 32;
+        uint32_t rb[kDB ? 2 : 1][CW];
+        tmem_ld_cols(col, rb[0]);
+        if (gi % C::kTabG == 0 &&
+            !warp_wait_u32(a_tabfull + 8 * tslot, (gi / (C::kTabG * C::kTabSlots)) & 1, abort_flag)) {
+          tmem_ld_wait();
+          live = false;
+          break;
+        }
+        const uint32_t tab = a_tab + tslot * C::kTabSlotBytes + (gi % C::kTabG) * C::kTabBytes;
+        const float4 w = lds_f4(tab + 16 * ch);
+        const uint32_t tsa = tab + C::kTabWBytes + part * CPT * 4;
+        const float2 sw2 = make_float2(w.x, w.y);
+        const float2 cb2 = make_float2(w.z, w.w);
 #pragma unroll
-      for (int c = 0; c < NCH; ++c) {
-        tmem_ld_wait();
-        reg_fence(rbuf[c & 1]);
-        if (c + 1 < NCH) tmem_ld_32x32b_x16(col + CW * (c + 1), rbuf[(c + 1) & 1]);
-        tmem_st_32x32b_x16_fill(col + CW * c, kI2FBiasBits);  // hand the chunk back preset to the bias
-        if (c + 1 == NCH) {
-          // Every partial of group g is in registers and its accumulator is
-          // reset: release the accumulator before waiting for group g+1, so
-          // the MMAs can run kAccBufs groups ahead of this warp.
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&accempty[a]);
-          if (g + 1 < G) {
-            const int a1 = (g + 1) % C::kAccBufs;
-            live = warp_wait(&done[(g + 1) % C::kDone], ((g + 1) / C::kDone) & 1, abort_flag);
-            if (live) {
-              tc_fence_after();
-              tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(a1 * kBM), rbuf[(c + 1) & 1]);
+        for (int h = 0; h < NCH; ++h) {
+          uint32_t(&r)[CW] = rb[kDB ? (h & 1) : 0];
+          if (!kDB && h > 0) tmem_ld_cols(col + CW * h, r);
+          tmem_ld_wait();
+          reg_fence(r);
+          if (kDB && h + 1 < NCH) tmem_ld_cols(col + CW * (h + 1), rb[(h + 1) & 1]);
+          // hand the columns back preset (its wait is after the math)
+          tmem_fill_cols<CW>(col + CW * h, kPreset);
+          if constexpr (kDebugP) {
+            if (nout >= 0) {
+#pragma unroll 4
+              for (int j = 0; j < CW; ++j) {
+                const int m = m0 + part * CPT + CW * h + j;
+                const int32_t pv =
+                    kCvtI2F ? static_cast<int32_t>(r[j]) : static_cast<int32_t>(r[j] - kI2FBiasBits);
+                if (m < M) P[(static_cast<int64_t>(m) * N + nout) * G + g] = pv;
+              }
+            }
+          } else {
+            // u = fma(v, s_w, -1.5*2^23*s_w) = fl(P*s_w): the bias term is
+            // exact for an fp16-valued s_w and the fma rounds
+            // v*s_w - 1.5*2^23*s_w once (kCvtI2F: v = float(P), u = fl(v*s_w),
+            // the same value); then acc += u * s_a.  The table holds the s_a
+            // of 4 consecutive tokens per 16 bytes.
+#pragma unroll
+            for (int j = 0; j < CW / 4; ++j) {
+              const float4 sa = lds_f4(tsa + 16 * ((CW / 4) * h + j));
+              float2 v0, v1;
+              if constexpr (kCvtI2F) {
+                v0 = make_float2(__int2float_rn(static_cast<int>(r[4 * j])),
+                                 __int2float_rn(static_cast<int>(r[4 * j + 1])));
+                v1 = make_float2(__int2float_rn(static_cast<int>(r[4 * j + 2])),
+                                 __int2float_rn(static_cast<int>(r[4 * j + 3])));
+              } else {
+                v0 = make_float2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]));
+                v1 = make_float2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+              }
+              const float2 u0 = __ffma2_rn(v0, sw2, cb2);
+              const float2 u1 = __ffma2_rn(v1, sw2, cb2);
+              const int k = (CW / 2) * h + 2 * j;  // acc[k] holds tokens 2k, 2k+1
+              acc[k] = __ffma2_rn(u0, make_float2(sa.x, sa.y), acc[k]);
+              acc[k + 1] = __ffma2_rn(u1, make_float2(sa.z, sa.w), acc[k + 1]);
             }
           }
         }
-        if constexpr (kDebugP) {
-          dump(rbuf[c & 1], g, CW * c);
-        } else {
-          convert(rbuf[c & 1], tab + (CW / 4) * c, sw2, cb2, CW * c);
+        if (gi % C::kTabG == C::kTabG - 1 || gi == total - 1) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive_u32(a_tabempty + 8 * tslot);  // the table slot is read
         }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_u32(a_accempty + 8 * a);  // the accumulator is drained (and refilled)
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tabempty[slot]);  // table slot read for the last time
+      if constexpr (!kDebugP) {
+        // the tile's outputs, straight from the running sums: a warp store
+        // covers 32 channels of one token row (adjacent output columns for
+        // most of a sorted channel set)
+        const int mbase = m0 + part * CPT;
+        if (live && nout >= 0) {
+          // one running pointer down the column (not 32 precomputed addresses)
+          __half *yp = Y + static_cast<int64_t>(mbase) * N + nout;
+          const int rows = M - mbase;
+#pragma unroll
+          for (int j = 0; j < CPT / 2; ++j) {
+            if (2 * j < rows) *yp = __float2half_rn(acc[j].x);
+            yp += N;
+            if (2 * j + 1 < rows) *yp = __float2half_rn(acc[j].y);
+            yp += N;
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < CPT / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
+      }
     }
     tmem_ld_wait();
-
-    if constexpr (!kDebugP) {
-      // stage fp16 results as [token][channel]: column `ch`, token rows
-      // half*CPT .. +CPT (a warp's stores cover 64 contiguous bytes of a row)
-      uint8_t *st = smem + C::kOffRing;
-      __half *dst = reinterpret_cast<__half *>(st + half * CPT * C::kStagingStride) + ch;
-#pragma unroll
-      for (int j = 0; j < CPT; ++j) dst[j * (C::kStagingStride / 2)] = __float2half_rn(acc[j]);
-      named_bar_sync(1, kEpiThreads);
-      if (!*abort_flag) {
-        constexpr int CPL = BN / 32;  // columns per lane
-        int col_out[CPL];
-#pragma unroll
-        for (int i = 0; i < CPL; ++i) col_out[i] = col_idx[lane + 32 * i];
-        for (int rr = e; rr < kBM; rr += kEpiWarps) {
-          const int mm = m0 + rr;
-          if (mm >= M) break;
-          const __half *srow = reinterpret_cast<const __half *>(st + rr * C::kStagingStride);
-          __half *yrow = Y + static_cast<int64_t>(mm) * N;
-#pragma unroll
-          for (int i = 0; i < CPL; ++i)
-            if (col_out[i] >= 0) yrow[col_out[i]] = srow[lane + 32 * i];
-        }
-      }
-    }
+    tmem_st_wait();
   }
 
   tc_fence_before();
@@ -616,15 +788,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void *p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+  });
   return fn;
 }
 
@@ -671,7 +842,109 @@ static bool encode_2d_u8(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *map
   return true;
 }
 
-template <int BN, bool kDebugP>
+// An int8 [rows, K] matrix (W8 [N8, K], or A_q [M, K]) as a 3-D tensor (k
+// within a group, row, group) with 128 x box_rows x groups_per_box boxes:
+// whole groups of a block of rows, each 128-byte row swizzled.  Encodings are
+// cached by (base, K, rows, box).
+static bool encode_groups_3d(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *map, const void *W8, int64_t K,
+                             int64_t N8, int box_rows, int groups_per_box) {
+  struct Entry {
+    const void *base;
+    int64_t K, N8;
+    int rows, gpb;
+    bool valid;
+    CUtensorMap map;
+  };
+  static Entry table[32];
+  static int next = 0;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry &e : table)
+    if (e.valid && e.base == W8 && e.K == K && e.N8 == N8 && e.rows == box_rows && e.gpb == groups_per_box) {
+      *map = e.map;
+      return true;
+    }
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(N8), static_cast<cuuint64_t>(K / 128)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K), 128};  // bytes, dims 1 and 2
+  const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(groups_per_box)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(W8), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  table[next] = Entry{W8, K, N8, box_rows, groups_per_box, true, *map};
+  next = (next + 1) % 32;
+  return true;
+}
+
+// A 2-D tensor of `dtype` elements (dims inner x outer, row stride in bytes)
+// with box_inner x box_outer boxes, no swizzle.  Encodings are cached.
+static bool encode_2d(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *map, CUtensorMapDataType dtype,
+                      const void *base, int64_t inner, int64_t outer, int64_t row_bytes, int box_inner, int box_outer) {
+  struct Entry {
+    const void *base;
+    int64_t inner, outer, row_bytes;
+    int dtype, bi, bo;
+    bool valid;
+    CUtensorMap map;
+  };
+  static Entry table[32];
+  static int next = 0;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry &e : table)
+    if (e.valid && e.base == base && e.inner == inner && e.outer == outer && e.row_bytes == row_bytes &&
+        e.dtype == static_cast<int>(dtype) && e.bi == box_inner && e.bo == box_outer) {
+      *map = e.map;
+      return true;
+    }
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  table[next] = Entry{base, inner, outer, row_bytes, static_cast<int>(dtype), box_inner, box_outer, true, *map};
+  next = (next + 1) % 32;
+  return true;
+}
+
+// Number of SMs of the current device (cached per device ordinal).
+static int device_sm_count() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+// How many CTAs of the persistent grid take 4-bit and 8-bit tiles: one CTA
+// per tile while the tiles fit on the SMs, otherwise the SMs split in
+// proportion to each set's work (an 8-bit tile costs about as much as a
+// 4-bit one here: no unpack, but twice the shared-memory operand traffic).
+static void split_ctas(int64_t T4, int64_t T8, int sms, int *c4, int *c8) {
+  if (T4 + T8 <= sms) {
+    *c4 = static_cast<int>(T4);
+    *c8 = static_cast<int>(T8);
+    return;
+  }
+  int a = static_cast<int>((static_cast<double>(sms) * T4) / static_cast<double>(T4 + T8) + 0.5);
+  if (T4 > 0 && a < 1) a = 1;
+  if (T8 > 0 && a > sms - 1) a = sms - 1;
+  if (T8 == 0) a = sms;
+  if (T4 == 0) a = 0;
+  *c4 = static_cast<int>(a < T4 ? a : T4);
+  *c8 = static_cast<int>((sms - a) < T8 ? (sms - a) : T8);
+}
+
+template <int BN, bool kDebugP, bool kCvtI2F>
 static cudaError_t launch_gemm_bn(const GemmArgs &a, cudaStream_t stream, const char **msg) {
   using C = GemmCfg<BN>;
   auto enc = get_encode_fn();
@@ -679,42 +952,68 @@ static cudaError_t launch_gemm_bn(const GemmArgs &a, cudaStream_t stream, const 
     *msg = "cuTensorMapEncodeTiled is not available from the driver";
     return cudaErrorNotSupported;
   }
-  CUtensorMap tmA, tmW8;
-  memset(&tmA, 0, sizeof(tmA));
+  CUtensorMap tmA4, tmA8, tmW8, tmZ;
+  memset(&tmA4, 0, sizeof(tmA4));
+  memset(&tmA8, 0, sizeof(tmA8));
   memset(&tmW8, 0, sizeof(tmW8));
-  if (!encode_2d_u8(enc, &tmA, a.A_q, a.K, a.M, kKG, kBM, true)) {
+  memset(&tmZ, 0, sizeof(tmZ));
+  // A_q in chunks of groups (one box per chunk and set), W8 likewise, the
+  // zero points of a 4-bit chunk as one 2-D box
+  if ((a.N4 > 0 && !encode_groups_3d(enc, &tmA4, a.A_q, a.K, a.M, kBM, C::kC4)) ||
+      (a.N8 > 0 && !encode_groups_3d(enc, &tmA8, a.A_q, a.K, a.M, kBM, C::kC8))) {
     *msg = "tensor map encoding of A_q failed";
     return cudaErrorInvalidValue;
   }
-  if (a.N8 > 0 && !encode_2d_u8(enc, &tmW8, a.W8, a.K, a.N8, kKG, BN, true)) {
+  if (a.N8 > 0 && !encode_groups_3d(enc, &tmW8, a.W8, a.K, a.N8, BN, C::kC8)) {
     *msg = "tensor map encoding of W8 failed";
     return cudaErrorInvalidValue;
   }
-  const int mt = static_cast<int>((a.M + kBM - 1) / kBM);
-  const int nt4 = static_cast<int>((a.N4 + BN - 1) / BN);
-  const int nt8 = static_cast<int>((a.N8 + BN - 1) / BN);
-  const int64_t grid = static_cast<int64_t>(mt) * (nt4 + nt8);
-  if (grid > 0x7FFFFFFF) {
+  if (a.N4 > 0 && !encode_2d_u8(enc, &tmZ, a.z4, padded_channels(a.N4) / 2, a.K / kKG, BN / 2, C::kC4, false)) {
+    *msg = "tensor map encoding of z4 failed";
+    return cudaErrorInvalidValue;
+  }
+  // The scales by TMA (4 groups of a tile per box) when s_a's rows are
+  // 16-byte multiples on a 16-byte aligned base; otherwise cp.async.
+  CUtensorMap tmSa, tmSw4, tmSw8;
+  memset(&tmSa, 0, sizeof(tmSa));
+  memset(&tmSw4, 0, sizeof(tmSw4));
+  memset(&tmSw8, 0, sizeof(tmSw8));
+  const int64_t G = a.K / kKG;
+  int vec = (G % C::kScG == 0 && (reinterpret_cast<uintptr_t>(a.s_a) & 15u) == 0) ? 1 : 0;
+  if (vec) {
+    const bool ok = encode_2d(enc, &tmSa, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.s_a, G, a.M, G * 4, C::kScG, kBM) &&
+                    (a.N4 == 0 || encode_2d(enc, &tmSw4, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.s_w4, padded_channels(a.N4),
+                                            G, padded_channels(a.N4) * 2, BN, C::kScG)) &&
+                    (a.N8 == 0 || encode_2d(enc, &tmSw8, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.s_w8, padded_channels(a.N8),
+                                            G, padded_channels(a.N8) * 2, BN, C::kScG));
+    if (!ok) vec = 0;
+  }
+  const int64_t mt = (a.M + kBM - 1) / kBM;
+  const int64_t T4 = mt * ((a.N4 + BN - 1) / BN);
+  const int64_t T8 = mt * ((a.N8 + BN - 1) / BN);
+  if (T4 + T8 > 0x7FFFFFFF || (T4 + T8) * (a.K / kKG) > 0x7FFFFFFF) {
     *msg = "too many tiles";
     return cudaErrorInvalidValue;
   }
-  auto kern = gemm_w4w8a8_kernel<BN, kDebugP>;
+  int c4 = 0, c8 = 0;
+  split_ctas(T4, T8, device_sm_count(), &c4, &c8);
+  auto kern = gemm_w4w8a8_kernel<BN, kDebugP, kCvtI2F>;
   int dev = 0;
   cudaGetDevice(&dev);
-  static unsigned long long configured = 0;  // one bit per device ordinal
-  if (dev < 64 && !(configured & (1ull << dev))) {
+  static std::atomic<unsigned long long> configured{0};  // one bit per device ordinal
+  if (dev < 64 && !(configured.load() & (1ull << dev))) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
     if (e != cudaSuccess) {
       *msg = "cudaFuncSetAttribute(MaxDynamicSharedMemorySize) failed";
       return e;
     }
-    configured |= 1ull << dev;
+    configured.fetch_or(1ull << dev);
   }
   // Launched as a programmatic dependent of the previous kernel in the stream:
   // the CTAs set up barriers and TMEM while that kernel finishes, and wait for
   // it (griddepcontrol.wait) before their first global read.
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.gridDim = dim3(static_cast<unsigned>(c4 + c8));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = C::kSmemAlloc;
   cfg.stream = stream;
@@ -724,18 +1023,23 @@ static cudaError_t launch_gemm_bn(const GemmArgs &a, cudaStream_t stream, const 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(
-      &cfg, kern, tmA, a.W4, tmW8, a.s_a, a.z4, static_cast<const __half *>(a.s_w4), a.idx4,
+      &cfg, kern, tmA4, tmA8, a.W4, tmW8, tmZ, tmSa, tmSw4, tmSw8, vec, a.s_a, static_cast<const __half *>(a.s_w4), a.idx4,
       static_cast<const __half *>(a.s_w8), a.idx8, static_cast<int>(a.M), static_cast<int>(a.K),
       static_cast<int>(a.N4), static_cast<int>(a.N8), static_cast<int>(padded_channels(a.N4)),
-      static_cast<int>(padded_channels(a.N8)), mt, nt4, static_cast<__half *>(a.Y), a.P);
+      static_cast<int>(padded_channels(a.N8)), static_cast<int>(mt), static_cast<int>(T4), static_cast<int>(T8), c4,
+      c8, static_cast<__half *>(a.Y), a.P);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) *msg = "launch of the fused GEMM failed";
   return e;
 }
 
 cudaError_t launch_gemm_w4w8a8(const GemmArgs &a, cudaStream_t stream, const char **msg) {
-  if (a.P) return launch_gemm_bn<128, true>(a, stream, msg);
-  return launch_gemm_bn<128, false>(a, stream, msg);
+  if (a.cvt_i2f) {
+    if (a.P) return launch_gemm_bn<128, true, true>(a, stream, msg);
+    return launch_gemm_bn<128, false, true>(a, stream, msg);
+  }
+  if (a.P) return launch_gemm_bn<128, true, false>(a, stream, msg);
+  return launch_gemm_bn<128, false, false>(a, stream, msg);
 }
 
 }  // namespace mixllm

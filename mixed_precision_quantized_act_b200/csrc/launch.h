@@ -34,6 +34,7 @@ struct GemmArgs {
   void *Y;     // fp16 [M, N4 + N8]
   int32_t *P;  // debug partials [M, N, G] or null
   const void *X = nullptr;  // fp16 [M, K] activations: the fused few-token path quantizes them itself
+  bool cvt_i2f = false;     // tiled GEMM only: plain int -> float convert instead of the bias trick (measurement)
 };
 
 // Returns a CUDA error, or cudaErrorNotSupported when the tensor-map encoder

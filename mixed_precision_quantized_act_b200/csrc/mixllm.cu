@@ -96,12 +96,14 @@ mixllm_status check_gemm(const int8_t *A_q, const float *s_a, int64_t M, int64_t
 
 mixllm_status gemm_common(const int8_t *A_q, const float *s_a, int64_t M, int64_t K, const uint8_t *W4,
                           const uint8_t *z4, const void *s_w4, const int32_t *idx4, int64_t N4, const int8_t *W8,
-                          const void *s_w8, const int32_t *idx8, int64_t N8, void *Y, int32_t *P, void *stream) {
+                          const void *s_w8, const int32_t *idx8, int64_t N8, void *Y, int32_t *P, void *stream,
+                          bool cvt_i2f = false) {
   bool empty = false;
   mixllm_status st = check_gemm(A_q, s_a, M, K, W4, z4, s_w4, idx4, N4, W8, s_w8, idx8, N8, Y, P, &empty);
   if (st != MIXLLM_OK) return st;
   if (empty) return ok();
   mixllm::GemmArgs a{A_q, s_a, M, K, W4, z4, s_w4, idx4, N4, W8, s_w8, idx8, N8, Y, P};
+  a.cvt_i2f = cvt_i2f;
   const char *msg = "";
   cudaError_t e = mixllm::launch_gemm_w4w8a8(a, static_cast<cudaStream_t>(stream), &msg);
   if (e == cudaErrorNotSupported) return fail(MIXLLM_ERR_UNSUPPORTED, "%s", msg);
@@ -205,6 +207,15 @@ mixllm_status mixllm_gemm_w4w8a8(const int8_t *A_q, const float *s_a, int64_t M,
                                  void *Y_f16, void *stream) {
   if (!Y_f16 && M > 0 && N4 + N8 > 0) return fail(MIXLLM_ERR_INVALID_ARG, "null Y");
   return gemm_common(A_q, s_a, M, K, W4, z4, s_w4_f16, idx4, N4, W8, s_w8_f16, idx8, N8, Y_f16, nullptr, stream);
+}
+
+mixllm_status mixllm_gemm_w4w8a8_plain_i2f(const int8_t *A_q, const float *s_a, int64_t M, int64_t K,
+                                           const uint8_t *W4, const uint8_t *z4, const void *s_w4_f16,
+                                           const int32_t *idx4, int64_t N4, const int8_t *W8, const void *s_w8_f16,
+                                           const int32_t *idx8, int64_t N8, void *Y_f16, void *stream) {
+  if (!Y_f16 && M > 0 && N4 + N8 > 0) return fail(MIXLLM_ERR_INVALID_ARG, "null Y");
+  return gemm_common(A_q, s_a, M, K, W4, z4, s_w4_f16, idx4, N4, W8, s_w8_f16, idx8, N8, Y_f16, nullptr, stream,
+                     true);
 }
 
 mixllm_status mixllm_gemm_debug_partials(const int8_t *A_q, const float *s_a, int64_t M, int64_t K,

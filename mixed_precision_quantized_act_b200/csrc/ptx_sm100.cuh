@@ -313,6 +313,54 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
 }
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// 16 or 32 consecutive columns of this warp's 32 lanes into r.
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[16]) { tmem_ld_32x32b_x16(taddr, r); }
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[32]) { tmem_ld_32x32b_x32(taddr, r); }
+// 16 or 32 consecutive columns of this warp's 32 lanes set to v.
+template <int W>
+__device__ __forceinline__ void tmem_fill_cols(uint32_t taddr, uint32_t v) {
+  static_assert(W == 16 || W == 32, "fill width");
+  if constexpr (W == 16) tmem_st_32x32b_x16_fill(taddr, v);
+  else tmem_st_32x32b_x32_fill(taddr, v);
+}
+
+
+// 16-byte shared-memory load from a 32-bit shared address.  Volatile with a
+// memory clobber: it stays after the barrier wait that publishes the data.
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
+  return v;
+}
+
+// Warp-uniform bounded wait on the mbarrier at a 32-bit shared address (see
+// warp_wait).
+__device__ __forceinline__ bool warp_wait_u32(uint32_t bar, uint32_t parity, volatile int *abort) {
+  if (__all_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity))) return true;
+  bool ok = true;
+  if (!mbar_try_wait(bar, parity)) {
+    const long long t0 = clock64();
+    while (true) {
+      if (mbar_try_wait_sleep(bar, parity, 20000u)) break;
+      if (*abort) {
+        ok = false;
+        break;
+      }
+      if (clock64() - t0 > (1ll << 32)) {
+        *abort = 1;
+        record_status(kStatusTimeout);
+        ok = false;
+        break;
+      }
+    }
+  }
+  return __all_sync(0xFFFFFFFFu, ok);
+}
+
+// Arrive (release) on the mbarrier at a 32-bit shared address.
+__device__ __forceinline__ void mbar_arrive_u32(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
 
 // ----------------------------------------------------------------- cp.async
 
