@@ -303,6 +303,10 @@ MIXLLM_API mixllm_status mixllm_linear_small_m(const void *X_f16, int64_t M, int
  *     asynchronous memset of the scratch, no allocation).
  *   * Calls that overlap in time on one device share the scratch and race:
  *     issue them to one stream, or order them with events.
+ *   * The scratch used is the current device's (cudaGetDevice at the call):
+ *     `stream` must belong to that device (or be NULL, its legacy default
+ *     stream); a stream of another device is not detected and the kernel
+ *     would read another device's memory.
  *   * Returns MIXLLM_ERR_UNSUPPORTED when the shape needs more scratch than
  *     the array holds (see mixllm_small_m_workspace_bytes), and
  *     MIXLLM_ERR_INVALID_ARG for M > 64.
@@ -314,6 +318,34 @@ MIXLLM_API mixllm_status mixllm_gemm_w4w8a8_small_m_noalloc(const int8_t *A_q, c
                                                  const int8_t *W8, const void *s_w8_f16,
                                                  const int32_t *idx8, int64_t N8,
                                                  void *Y_f16, void *stream);
+
+/*
+ * Debug form of one named few-token kernel, for parity tests: runs the kernel
+ * `kind` (a mixllm_small_m_kind) whatever mixllm_small_m_kernel would pick,
+ * and writes both Y (as mixllm_gemm_w4w8a8_small_m would with that kernel)
+ * and the per-group int32 partials of step 2 of the two-step dequantization
+ * (MLSys 2026 talk notes on MixLLM, §二段階逆量子化)
+ *   P[m, idx[n], g] = sum_{k in g} (W_q[n,k] - z[n,g]) * A_q[m,k]
+ * into
+ *   P          device, int32 [M, N4 + N8, K/128], 4-byte aligned, written
+ *              for every m < M and every listed column.
+ *   workspace  device, 16-byte aligned, at least
+ *              mixllm_small_m_debug_workspace_bytes(.., kind, ..) bytes,
+ *              zero-filled before its first use (calls leave it so).
+ * Which kinds a shape allows: the tensor-core kernel any 1 <= M <= 64; the
+ * split GEMV M <= 8; the persistent GEMV M <= 4 with M*K <= 32768 (rounded
+ * up to 1, 2, 4 tokens).  Other kinds return MIXLLM_ERR_UNSUPPORTED.  Other
+ * arguments and errors: as mixllm_gemm_w4w8a8_small_m.  Slow (uncoalesced
+ * stores of P); asynchronous on `stream`.
+ */
+MIXLLM_API mixllm_status mixllm_small_m_debug_workspace_bytes(int64_t M, int64_t K, int64_t N4, int64_t N8,
+                                                   int32_t kind, size_t *bytes);
+MIXLLM_API mixllm_status mixllm_small_m_debug_partials(const int8_t *A_q, const float *s_a, int64_t M, int64_t K,
+                                            const uint8_t *W4, const uint8_t *z4, const void *s_w4_f16,
+                                            const int32_t *idx4, int64_t N4, const int8_t *W8,
+                                            const void *s_w8_f16, const int32_t *idx8, int64_t N8,
+                                            int32_t kind, int32_t *P, void *Y_f16, void *workspace,
+                                            size_t workspace_bytes, void *stream);
 
 /*
  * Global mixed-precision search, step 1 (MLSys 2026 talk notes on MixLLM,

@@ -32,6 +32,7 @@ from ._lib import (  # noqa: F401
     select_top_t_workspace,
     selftest_wait_timeout,
     small_m_kernel,
+    small_m_debug_partials,
     small_m_workspace,
     small_m_workspace_bytes,
     sync_status,

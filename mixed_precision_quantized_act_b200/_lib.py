@@ -47,6 +47,11 @@ SIGNATURES = {
                                                   _vp, _vp, _vp, _i64, _vp, _vp, ctypes.c_size_t, _vp]),
     "mixllm_gemm_w4w8a8_small_m_noalloc": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64,
                                                           _vp, _vp, _vp, _i64, _vp, _vp]),
+    "mixllm_small_m_debug_workspace_bytes": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.c_int32,
+                                                            ctypes.POINTER(ctypes.c_size_t)]),
+    "mixllm_small_m_debug_partials": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64,
+                                                     _vp, _vp, _vp, _i64, ctypes.c_int32, _vp, _vp, _vp,
+                                                     ctypes.c_size_t, _vp]),
     "mixllm_sync_status": (ctypes.c_int, [_vp]),
     "mixllm_selftest_wait_timeout": (ctypes.c_int, [_u32, _vp]),
 }
@@ -314,6 +319,25 @@ def gemm_w4w8a8_small_m_noalloc_into(A_q, s_a, p: PackedLinear, Y, stream=None):
                                                      _ptr(p.s_w4), _ptr(p.idx4), p.N4, _ptr(p.W8), _ptr(p.s_w8),
                                                      _ptr(p.idx8), p.N8, _ptr(Y), _stream(stream)),
            "mixllm_gemm_w4w8a8_small_m_noalloc")
+
+
+def small_m_debug_partials(A_q, s_a, p: PackedLinear, kind: str, stream=None):
+    """Debug form of one named few-token kernel (one of SMALL_M_KERNELS, run
+    whatever the plan would pick): returns (Y fp16 [M, N], P int32 [M, N, K/128])."""
+    _need_cuda(A_q, s_a)
+    M, K = A_q.shape
+    k = SMALL_M_KERNELS.index(kind)
+    n = ctypes.c_size_t(0)
+    _check(load().mixllm_small_m_debug_workspace_bytes(M, K, p.N4, p.N8, k, ctypes.byref(n)),
+           "mixllm_small_m_debug_workspace_bytes")
+    ws = torch.zeros(max(n.value, 16), dtype=torch.uint8, device=A_q.device)
+    Y = torch.empty((M, p.N), dtype=torch.float16, device=A_q.device)
+    P = torch.zeros((M, p.N, K // GROUP), dtype=torch.int32, device=A_q.device)
+    _check(load().mixllm_small_m_debug_partials(_ptr(A_q), _ptr(s_a), M, K, _ptr(p.W4), _ptr(p.z4), _ptr(p.s_w4),
+                                                _ptr(p.idx4), p.N4, _ptr(p.W8), _ptr(p.s_w8), _ptr(p.idx8), p.N8,
+                                                k, _ptr(P), _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)),
+           "mixllm_small_m_debug_partials")
+    return Y, P
 
 
 def linear(X: torch.Tensor, p: PackedLinear, stream=None, workspace: torch.Tensor = None) -> torch.Tensor:

@@ -33,6 +33,7 @@
 // (gemv_w4w8a8.cuh): the same plan, workspace layout and split reduction.
 #pragma once
 
+#include <atomic>
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
@@ -164,7 +165,8 @@ __device__ __forceinline__ void sm_reg_fence(uint32_t (&r)[MP]) {
   }
 }
 
-template <int MP>
+// DBG: the int32 group partials also go to Pd [M, N, G] (output column order).
+template <int MP, bool DBG = false>
 __global__ void __launch_bounds__(kSmThreads, 1)
     gemm_small_m_kernel(const __grid_constant__ CUtensorMap tmX, const uint8_t *__restrict__ W4,
                         const __grid_constant__ CUtensorMap tmW8, const __grid_constant__ CUtensorMap tmZ,
@@ -173,7 +175,7 @@ __global__ void __launch_bounds__(kSmThreads, 1)
                         const int32_t *__restrict__ idx4, const __half *__restrict__ s_w8,
                         const int32_t *__restrict__ idx8, int M, int K, int N4, int N8, int N4p, int N8p, int nt4,
                         int ntiles, int S, __half *__restrict__ Y, float *__restrict__ ws_part,
-                        int *__restrict__ ws_cnt) {
+                        int *__restrict__ ws_cnt, int32_t *__restrict__ Pd) {
   using C = SmallMCfg<MP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -463,6 +465,10 @@ __global__ void __launch_bounds__(kSmThreads, 1)
     float acc[MP];
 #pragma unroll
     for (int t = 0; t < MP; ++t) acc[t] = 0.0f;
+    int32_t *pd = nullptr;  // DBG: this channel's partials of token 0, group g0
+    if constexpr (DBG) {
+      if (n0 + c < Nset) pd = Pd + static_cast<int64_t>(__ldg(idx + n0 + c)) * G + g0;
+    }
     bool live = warp_wait(tabready, 0, abort_flag);
     for (int i = 0; live && i < ng; ++i) {
       const int a = i % C::kAccBufs;
@@ -487,6 +493,11 @@ __global__ void __launch_bounds__(kSmThreads, 1)
         tmem_ld_wait();
         sm_reg_fence<CH>(r);
         sm_tmem_fill<CH>(col, kI2FBiasBits);  // hand the columns back preset to the bias
+        if constexpr (DBG) {
+          if (pd != nullptr)
+            for (int t = 0; t < CH; ++t)
+              if (h * CH + t < M) pd[static_cast<int64_t>(h * CH + t) * N * G + i] = static_cast<int32_t>(r[t] - kI2FBiasBits);
+        }
 #pragma unroll
         for (int t = 0; t < CH; t += 2) {
           const int tt = h * CH + t;
@@ -573,6 +584,7 @@ __global__ void __launch_bounds__(kSmThreads, 1)
 
 constexpr int kSmWave = 148;      // SMs of a B200: split-K fills one wave of CTAs
 constexpr int kGemvMaxM = 8;      // up to this many tokens the GEMV kernel runs
+constexpr int kSmallMMaxM = 64;   // the few-token path takes up to this many tokens
 // GEMV grid target: the CTAs that are resident at once on the 148 SMs
 constexpr int gemv_cta_target(int mt) { return kSmWave * gemv_min_blocks(mt); }
 constexpr int kGvpMinUnitsPerCta = 8;  // the persistent GEMV from this many 32 KiB units per CTA
@@ -581,9 +593,12 @@ constexpr int gemv_groups_max(int mt) {
                  : (mt == 2 ? GvCfg<2>::kGroupsMax : (mt == 4 ? GvCfg<4>::kGroupsMax : GvCfg<8>::kGroupsMax));
 }
 
-SmallMPlan plan_small_m(int64_t M, int64_t N4, int64_t N8, int64_t K) {
+// force: -1 plans by shape; 0, 1, 2 ask for the tensor-core kernel, the split
+// GEMV or the persistent GEMV (the caller checks that the shape allows it:
+// small_m_kernel_allowed).
+SmallMPlan plan_small_m(int64_t M, int64_t N4, int64_t N8, int64_t K, int force = -1) {
   SmallMPlan p{};
-  p.gemv = M <= kGemvMaxM;
+  p.gemv = force < 0 ? M <= kGemvMaxM : force != 0;
   if (p.gemv)
     p.mp = M <= 1 ? 1 : (M <= 2 ? 2 : (M <= 4 ? 4 : 8));
   else
@@ -602,8 +617,9 @@ SmallMPlan plan_small_m(int64_t M, int64_t N4, int64_t N8, int64_t K) {
   // 16 % faster) and loses below (8B gate_up, 6 units: 8 % slower).
   const int chunks4 = (p.groups + 3) / 4, chunks8 = (p.groups + 1) / 2;
   const int64_t U = static_cast<int64_t>(p.nt4) * chunks4 + static_cast<int64_t>(p.nt8) * chunks8;
-  if (p.gemv && p.mp <= kGvpMaxTokens && static_cast<int64_t>(p.mp) * K <= kGvpMaxTokenBytes &&
-      U >= static_cast<int64_t>(kGvpMinUnitsPerCta) * gemv_cta_target(p.mp)) {
+  const bool want_persistent =
+      force < 0 ? U >= static_cast<int64_t>(kGvpMinUnitsPerCta) * gemv_cta_target(p.mp) : force == 2;
+  if (p.gemv && p.mp <= kGvpMaxTokens && static_cast<int64_t>(p.mp) * K <= kGvpMaxTokenBytes && want_persistent) {
     p.persistent = true;
     p.chunks4 = chunks4;
     p.chunks8 = chunks8;
@@ -632,7 +648,7 @@ SmallMPlan plan_small_m(int64_t M, int64_t N4, int64_t N8, int64_t K) {
   return p;
 }
 
-template <int MP>
+template <int MP, bool DBG = false>
 static cudaError_t launch_small_m_mp(const GemmArgs &a, const SmallMPlan &p, void *ws, cudaStream_t stream,
                                      const char **msg) {
   using C = SmallMCfg<MP>;
@@ -664,17 +680,17 @@ static cudaError_t launch_small_m_mp(const GemmArgs &a, const SmallMPlan &p, voi
     *msg = "too many tiles";
     return cudaErrorInvalidValue;
   }
-  auto kern = gemm_small_m_kernel<MP>;
+  auto kern = gemm_small_m_kernel<MP, DBG>;
   int dev = 0;
   cudaGetDevice(&dev);
-  static unsigned long long configured = 0;  // one bit per device ordinal
-  if (dev < 64 && !(configured & (1ull << dev))) {
+  static std::atomic<unsigned long long> configured{0};  // one bit per device ordinal
+  if (dev < 64 && !(configured.load() & (1ull << dev))) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
     if (e != cudaSuccess) {
       *msg = "cudaFuncSetAttribute(MaxDynamicSharedMemorySize) failed";
       return e;
     }
-    configured |= 1ull << dev;
+    configured.fetch_or(1ull << dev);
   }
   float *ws_part = static_cast<float *>(ws);
   int *ws_cnt = p.splits > 1 ? reinterpret_cast<int *>(ws_part + p.part_floats) : nullptr;
@@ -692,13 +708,14 @@ static cudaError_t launch_small_m_mp(const GemmArgs &a, const SmallMPlan &p, voi
       &cfg, kern, tmX, a.W4, tmW8, tmZ, a.s_a, a.z4, static_cast<const __half *>(a.s_w4), a.idx4,
       static_cast<const __half *>(a.s_w8), a.idx8, static_cast<int>(a.M), static_cast<int>(a.K),
       static_cast<int>(a.N4), static_cast<int>(a.N8), static_cast<int>(padded_channels(a.N4)),
-      static_cast<int>(padded_channels(a.N8)), p.nt4, tiles, p.splits, static_cast<__half *>(a.Y), ws_part, ws_cnt);
+      static_cast<int>(padded_channels(a.N8)), p.nt4, tiles, p.splits, static_cast<__half *>(a.Y), ws_part, ws_cnt,
+      DBG ? a.P : nullptr);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) *msg = "launch of the small-M GEMM failed";
   return e;
 }
 
-template <int MT, bool FUSE = false>
+template <int MT, bool FUSE = false, bool DBG = false>
 static cudaError_t launch_gemv_mt(const GemmArgs &a, const SmallMPlan &p, void *ws, cudaStream_t stream,
                                   const char **msg) {
   static_assert(gemv_min_blocks(MT) * (gemv_smem_bytes<MT>() + 1024) <= 228 * 1024, "resident CTAs per SM");
@@ -721,17 +738,17 @@ static cudaError_t launch_gemv_mt(const GemmArgs &a, const SmallMPlan &p, void *
     *msg = "too many tiles";
     return cudaErrorInvalidValue;
   }
-  auto kern = gemv_w4w8a8_kernel<MT, FUSE>;
+  auto kern = gemv_w4w8a8_kernel<MT, FUSE, DBG>;
   int dev = 0;
   cudaGetDevice(&dev);
-  static unsigned long long configured = 0;  // one bit per device ordinal
-  if (dev < 64 && !(configured & (1ull << dev))) {
+  static std::atomic<unsigned long long> configured{0};  // one bit per device ordinal
+  if (dev < 64 && !(configured.load() & (1ull << dev))) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gemv_smem_bytes<MT>());
     if (e != cudaSuccess) {
       *msg = "cudaFuncSetAttribute(MaxDynamicSharedMemorySize) failed";
       return e;
     }
-    configured |= 1ull << dev;
+    configured.fetch_or(1ull << dev);
   }
   float *ws_part = static_cast<float *>(ws);
   int *ws_cnt = p.counters > 0 ? reinterpret_cast<int *>(ws_part + p.part_floats) : nullptr;
@@ -751,13 +768,13 @@ static cudaError_t launch_gemv_mt(const GemmArgs &a, const SmallMPlan &p, void *
       static_cast<const __half *>(a.s_w8), a.idx8, static_cast<int>(a.M), static_cast<int>(a.K),
       static_cast<int>(a.N4), static_cast<int>(a.N8), static_cast<int>(padded_channels(a.N4)),
       static_cast<int>(padded_channels(a.N8)), p.nt4, tiles, p.splits, p.splits8, static_cast<__half *>(a.Y), ws_part,
-      ws_cnt);
+      ws_cnt, DBG ? a.P : nullptr);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) *msg = "launch of the GEMV failed";
   return e;
 }
 
-template <int MT>
+template <int MT, bool DBG = false>
 static cudaError_t launch_gemv_persistent_mt(const GemmArgs &a, const SmallMPlan &p, void *ws, cudaStream_t stream,
                                              const char **msg) {
   static_assert(2 * (gvp_smem_bytes_max<MT>() + 1024) <= 228 * 1024, "two CTAs per SM");
@@ -774,17 +791,17 @@ static cudaError_t launch_gemv_persistent_mt(const GemmArgs &a, const SmallMPlan
       return cudaErrorInvalidValue;
     }
   }
-  auto kern = gemv_w4w8a8_persistent_kernel<MT>;
+  auto kern = gemv_w4w8a8_persistent_kernel<MT, DBG>;
   int dev = 0;
   cudaGetDevice(&dev);
-  static unsigned long long configured = 0;  // one bit per device ordinal
-  if (dev < 64 && !(configured & (1ull << dev))) {
+  static std::atomic<unsigned long long> configured{0};  // one bit per device ordinal
+  if (dev < 64 && !(configured.load() & (1ull << dev))) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gvp_smem_bytes_max<MT>());
     if (e != cudaSuccess) {
       *msg = "cudaFuncSetAttribute(MaxDynamicSharedMemorySize) failed";
       return e;
     }
-    configured |= 1ull << dev;
+    configured.fetch_or(1ull << dev);
   }
   GvpGeom geo{p.nt4, p.chunks4, p.chunks8, p.units, p.ctas};
   float *ws_part = static_cast<float *>(ws);
@@ -803,7 +820,7 @@ static cudaError_t launch_gemv_persistent_mt(const GemmArgs &a, const SmallMPlan
       &cfg, kern, tmW8, a.A_q, a.s_a, a.W4, a.z4, static_cast<const __half *>(a.s_w4), a.idx4,
       static_cast<const __half *>(a.s_w8), a.idx8, static_cast<int>(a.M), static_cast<int>(a.K),
       static_cast<int>(a.N4), static_cast<int>(a.N8), static_cast<int>(padded_channels(a.N4)),
-      static_cast<int>(padded_channels(a.N8)), geo, static_cast<__half *>(a.Y), ws_part, ws_cnt);
+      static_cast<int>(padded_channels(a.N8)), geo, static_cast<__half *>(a.Y), ws_part, ws_cnt, DBG ? a.P : nullptr);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) *msg = "launch of the persistent GEMV failed";
   return e;
@@ -863,6 +880,49 @@ cudaError_t launch_linear_small_m(const GemmArgs &a, void *ws, size_t ws_bytes, 
   q.s_a = s_a;
   q.X = nullptr;
   return launch_gemm_small_m(q, ws, p.bytes(), stream, msg);
+}
+
+bool small_m_kernel_allowed(int64_t M, int64_t N4, int64_t N8, int64_t K, int kind) {
+  if (M < 1 || M > kSmallMMaxM || kind < 0 || kind > 2) return false;
+  if (kind == 0) return true;
+  if (M > kGemvMaxM) return false;
+  const SmallMPlan p = plan_small_m(M, N4, N8, K, kind);
+  return kind == 2 ? p.persistent : !p.persistent;
+}
+
+size_t small_m_debug_workspace_bytes(int64_t M, int64_t N4, int64_t N8, int64_t K, int kind) {
+  return plan_small_m(M, N4, N8, K, kind).bytes();
+}
+
+cudaError_t launch_small_m_debug_partials(const GemmArgs &a, int kind, void *ws, size_t ws_bytes,
+                                          cudaStream_t stream, const char **msg) {
+  if (!small_m_kernel_allowed(a.M, a.N4, a.N8, a.K, kind)) {
+    *msg = "the requested few-token kernel cannot take this shape";
+    return cudaErrorInvalidValue;
+  }
+  const SmallMPlan p = plan_small_m(a.M, a.N4, a.N8, a.K, kind);
+  if (ws_bytes < p.bytes() || (p.bytes() > 0 && ws == nullptr)) {
+    *msg = "workspace too small for this shape";
+    return cudaErrorInvalidValue;
+  }
+  if (a.P == nullptr) {
+    *msg = "no partials buffer";
+    return cudaErrorInvalidValue;
+  }
+  if (kind == 2) {
+    if (p.mp == 1) return launch_gemv_persistent_mt<1, true>(a, p, ws, stream, msg);
+    if (p.mp == 2) return launch_gemv_persistent_mt<2, true>(a, p, ws, stream, msg);
+    return launch_gemv_persistent_mt<4, true>(a, p, ws, stream, msg);
+  }
+  if (kind == 1) {
+    if (p.mp == 1) return launch_gemv_mt<1, false, true>(a, p, ws, stream, msg);
+    if (p.mp == 2) return launch_gemv_mt<2, false, true>(a, p, ws, stream, msg);
+    if (p.mp == 4) return launch_gemv_mt<4, false, true>(a, p, ws, stream, msg);
+    return launch_gemv_mt<8, false, true>(a, p, ws, stream, msg);
+  }
+  if (p.mp == 16) return launch_small_m_mp<16, true>(a, p, ws, stream, msg);
+  if (p.mp == 32) return launch_small_m_mp<32, true>(a, p, ws, stream, msg);
+  return launch_small_m_mp<64, true>(a, p, ws, stream, msg);
 }
 
 int small_m_kernel_kind(int64_t M, int64_t N4, int64_t N8, int64_t K) {

@@ -112,10 +112,13 @@ __device__ __forceinline__ int4 lds_i4(const int8_t *p) { return *reinterpret_ca
 // codes a thread loads serve both rows; the runs are taken in an order
 // rotated by rp / 2 so that the 8 rows of a quarter warp read 8 different
 // bank groups.
-template <int MT>
+// DBG: P of row h, token m < mt also goes to pd[h][m * pd_tstride] (rows
+// whose pointer is null are skipped).
+template <int MT, bool DBG = false>
 __device__ __forceinline__ void gv_group4x2(const uint8_t *blk, int rp, const int8_t *a, int a_stride,
                                             const int *asum, const float *sa, int t_stride, const int (&z)[2],
-                                            const float (&sw)[2], float (&acc)[2][MT]) {
+                                            const float (&sw)[2], float (&acc)[2][MT], int32_t *pd0 = nullptr,
+                                            int32_t *pd1 = nullptr, int64_t pd_tstride = 0, int mt = 0) {
   int plo[2][MT][2], phi[2][MT][2];
 #pragma unroll
   for (int h = 0; h < 2; ++h)
@@ -150,6 +153,10 @@ __device__ __forceinline__ void gv_group4x2(const uint8_t *blk, int rp, const in
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
       const int P = (plo[h][m][0] + plo[h][m][1]) + ((phi[h][m][0] + phi[h][m][1]) >> 4) - z[h] * asum[m * t_stride];
+      if constexpr (DBG) {
+        int32_t *pd = h == 0 ? pd0 : pd1;
+        if (pd != nullptr && m < mt) pd[m * pd_tstride] = P;
+      }
       const float v = __uint_as_float(static_cast<uint32_t>(P) + kI2FBiasBits);
       acc[h][m] = __fmaf_rn(__fmaf_rn(v, sw[h], cb), sa[m * t_stride], acc[h][m]);
     }
@@ -158,10 +165,11 @@ __device__ __forceinline__ void gv_group4x2(const uint8_t *blk, int rp, const in
 
 // One 8-bit group of one channel row, all tokens (P = sum_k W_q*A_q, exact).
 // wrow: the row's 128 bytes of a 128-byte swizzled TMA box in shared memory
-// (16-byte chunk q of row r at chunk q ^ (r & 7)).
-template <int MT>
+// (16-byte chunk q of row r at chunk q ^ (r & 7)).  DBG: as gv_group4x2.
+template <int MT, bool DBG = false>
 __device__ __forceinline__ void gv_group8(const uint8_t *wrow, int r, const int8_t *a, int a_stride,
-                                          const float *sa, int t_stride, float sw, float (&acc)[MT]) {
+                                          const float *sa, int t_stride, float sw, float (&acc)[MT],
+                                          int32_t *pd = nullptr, int64_t pd_tstride = 0, int mt = 0) {
   int p[MT][4];
 #pragma unroll
   for (int m = 0; m < MT; ++m) p[m][0] = p[m][1] = p[m][2] = p[m][3] = 0;
@@ -181,6 +189,9 @@ __device__ __forceinline__ void gv_group8(const uint8_t *wrow, int r, const int8
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
     const int P = (p[m][0] + p[m][1]) + (p[m][2] + p[m][3]);
+    if constexpr (DBG) {
+      if (pd != nullptr && m < mt) pd[m * pd_tstride] = P;
+    }
     const float v = __uint_as_float(static_cast<uint32_t>(P) + kI2FBiasBits);
     acc[m] = __fmaf_rn(__fmaf_rn(v, sw, cb), sa[m * t_stride], acc[m]);
   }
@@ -196,7 +207,8 @@ __device__ __forceinline__ void gv_group8(const uint8_t *wrow, int r, const int8
 // only when the slice fits in a slot), then the slot is refilled with weights.
 // tmW8: the 8-bit weights as a 3-D tensor (k within a group, row, group)
 // with boxes of GvCfg<MT>::kChunk8 groups.
-template <int MT, bool FUSE>
+// DBG: the int32 group partials also go to Pd [M, N, G] (output column order).
+template <int MT, bool FUSE, bool DBG = false>
 __global__ void __launch_bounds__(kGvThreads, gemv_min_blocks(MT))
     gemv_w4w8a8_kernel(const __grid_constant__ CUtensorMap tmW8, const __half *__restrict__ X,
                        const int8_t *__restrict__ A_q,
@@ -204,7 +216,7 @@ __global__ void __launch_bounds__(kGvThreads, gemv_min_blocks(MT))
                        const __half *__restrict__ s_w4, const int32_t *__restrict__ idx4,
                        const __half *__restrict__ s_w8, const int32_t *__restrict__ idx8, int M, int K, int N4,
                        int N8, int N4p, int N8p, int nt4, int ntiles, int S4, int S8, __half *__restrict__ Y,
-                       float *__restrict__ ws_part, int *__restrict__ ws_cnt) {
+                       float *__restrict__ ws_part, int *__restrict__ ws_cnt, int32_t *__restrict__ Pd) {
   using C = GvCfg<MT>;
   constexpr int kGvSlots = C::kSlots, kGvSlotBytes = C::kSlotBytes, kGvChunk4 = C::kChunk4, kGvChunk8 = C::kChunk8;
   extern __shared__ uint8_t gv_dyn[];
@@ -372,14 +384,24 @@ __global__ void __launch_bounds__(kGvThreads, gemv_min_blocks(MT))
         if (i < ng) {
           const int z[2] = {(S.z[i][rp >> 1] >> ((rp & 1) * 4)) & 0xF, (S.z[i][(rp + 64) >> 1] >> ((rp & 1) * 4)) & 0xF};
           const float sw[2] = {__half2float(S.sw[i][rp]), __half2float(S.sw[i][rp + 64])};
-          gv_group4x2<MT>(slot + j4 * 8192, rp, &S.a[0][i * 128], C::kGroupsMax * 128, &S.asum[0][i], &S.sa[0][i],
-                          C::kGroupsMax, z, sw, acc);
+          int32_t *pd0 = nullptr, *pd1 = nullptr;
+          if constexpr (DBG) {
+            if (n0 + rp < Nset) pd0 = Pd + static_cast<int64_t>(__ldg(idx4 + n0 + rp)) * G + g0 + i;
+            if (n0 + rp + 64 < Nset) pd1 = Pd + static_cast<int64_t>(__ldg(idx4 + n0 + rp + 64)) * G + g0 + i;
+          }
+          gv_group4x2<MT, DBG>(slot + j4 * 8192, rp, &S.a[0][i * 128], C::kGroupsMax * 128, &S.asum[0][i],
+                               &S.sa[0][i], C::kGroupsMax, z, sw, acc, pd0, pd1, static_cast<int64_t>(N) * G, mt);
         }
       } else {
         const int i = c * chunk + j8;
-        if (i < ng)
-          gv_group8<MT>(slot + j8 * 16384 + r8 * 128, r8, &S.a[0][i * 128], C::kGroupsMax * 128, &S.sa[0][i],
-                        C::kGroupsMax, __half2float(S.sw[i][r8]), acc[0]);
+        if (i < ng) {
+          int32_t *pd = nullptr;
+          if constexpr (DBG) {
+            if (n0 + r8 < Nset) pd = Pd + static_cast<int64_t>(__ldg(idx8 + n0 + r8)) * G + g0 + i;
+          }
+          gv_group8<MT, DBG>(slot + j8 * 16384 + r8 * 128, r8, &S.a[0][i * 128], C::kGroupsMax * 128, &S.sa[0][i],
+                             C::kGroupsMax, __half2float(S.sw[i][r8]), acc[0], pd, static_cast<int64_t>(N) * G, mt);
+        }
       }
     } else if (threadIdx.x == 0 && drain_from < 0) {
       drain_from = c;
@@ -530,7 +552,8 @@ struct GvpGeom {  // the unit sequence
   }
 };
 
-template <int MT>
+// DBG: the int32 group partials also go to Pd [M, N, G] (output column order).
+template <int MT, bool DBG = false>
 __global__ void __launch_bounds__(kGvThreads, 2)
     gemv_w4w8a8_persistent_kernel(const __grid_constant__ CUtensorMap tmW8, const int8_t *__restrict__ A_q,
                                   const float *__restrict__ s_a, const uint8_t *__restrict__ W4,
@@ -538,7 +561,7 @@ __global__ void __launch_bounds__(kGvThreads, 2)
                                   const int32_t *__restrict__ idx4, const __half *__restrict__ s_w8,
                                   const int32_t *__restrict__ idx8, int M, int K, int N4, int N8, int N4p, int N8p,
                                   GvpGeom geo, __half *__restrict__ Y, float *__restrict__ ws_part,
-                                  int *__restrict__ ws_cnt) {
+                                  int *__restrict__ ws_cnt, int32_t *__restrict__ Pd) {
   extern __shared__ uint8_t gv_dyn[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(gv_dyn) + 1023) & ~uintptr_t(1023));
   const int G = K >> 7;
@@ -691,12 +714,24 @@ __global__ void __launch_bounds__(kGvThreads, 2)
           const int z[2] = {(ms[j4 * 64 + (rp >> 1)] >> ((rp & 1) * 4)) & 0xF,
                             (ms[j4 * 64 + ((rp + 64) >> 1)] >> ((rp & 1) * 4)) & 0xF};
           const float sw[2] = {__half2float(msw[j4 * 128 + rp]), __half2float(msw[j4 * 128 + rp + 64])};
-          gv_group4x2<MT>(slot + j4 * 8192, rp, sA + g * 128, K, sAsum + g, sSa + g, G, z, sw, acc);
+          int32_t *pd0 = nullptr, *pd1 = nullptr;
+          if constexpr (DBG) {
+            const int n0 = t * 128;
+            if (n0 + rp < N4) pd0 = Pd + static_cast<int64_t>(__ldg(idx4 + n0 + rp)) * G + g;
+            if (n0 + rp + 64 < N4) pd1 = Pd + static_cast<int64_t>(__ldg(idx4 + n0 + rp + 64)) * G + g;
+          }
+          gv_group4x2<MT, DBG>(slot + j4 * 8192, rp, sA + g * 128, K, sAsum + g, sSa + g, G, z, sw, acc, pd0, pd1,
+                               static_cast<int64_t>(N) * G, M < MT ? M : MT);
         }
       } else if (j8 < ng) {
         const int g = g0 + j8;
-        gv_group8<MT>(slot + j8 * 16384 + r8 * 128, r8, sA + g * 128, K, sSa + g, G,
-                      __half2float(msw[j8 * 128 + r8]), acc[0]);
+        int32_t *pd = nullptr;
+        if constexpr (DBG) {
+          const int n0 = (t - geo.nt4) * 128;
+          if (n0 + r8 < N8) pd = Pd + static_cast<int64_t>(__ldg(idx8 + n0 + r8)) * G + g;
+        }
+        gv_group8<MT, DBG>(slot + j8 * 16384 + r8 * 128, r8, sA + g * 128, K, sSa + g, G,
+                           __half2float(msw[j8 * 128 + r8]), acc[0], pd, static_cast<int64_t>(N) * G, M < MT ? M : MT);
       }
     } else if (threadIdx.x == 0 && drain_from < 0) {
       drain_from = k;

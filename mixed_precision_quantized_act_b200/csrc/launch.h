@@ -44,11 +44,17 @@ cudaError_t launch_gemm_w4w8a8(const GemmArgs &a, cudaStream_t stream, const cha
 // Few-token variant (M <= 64): split-K over the groups with a workspace of
 // small_m_workspace_bytes() bytes: fp32 partial sums, then one int32 counter
 // per tile (zero before the first call; every call returns them to zero).
-// Y only; no debug partials.
+// Y only (the debug partials: launch_small_m_debug_partials).
 cudaError_t launch_gemm_small_m(const GemmArgs &a, void *ws, size_t ws_bytes, cudaStream_t stream, const char **msg);
 size_t small_m_workspace_bytes(int64_t M, int64_t N4, int64_t N8, int64_t K);
 // 0: tensor-core kernel, 1: split GEMV, 2: persistent GEMV (mixllm_small_m_kind)
 int small_m_kernel_kind(int64_t M, int64_t N4, int64_t N8, int64_t K);
+// Debug form of one named few-token kernel (kind as above, whatever the plan
+// would pick): Y, and the int32 group partials into a.P [M, N, G].
+bool small_m_kernel_allowed(int64_t M, int64_t N4, int64_t N8, int64_t K, int kind);
+size_t small_m_debug_workspace_bytes(int64_t M, int64_t N4, int64_t N8, int64_t K, int kind);
+cudaError_t launch_small_m_debug_partials(const GemmArgs &a, int kind, void *ws, size_t ws_bytes,
+                                          cudaStream_t stream, const char **msg);
 // The few-token layer from fp16 X (quantization included): the split GEMV
 // quantizes in its prologue when its slice of X fits a ring slot; otherwise
 // the quantizer writes A_q / s_a into the workspace first.  a.X is required,

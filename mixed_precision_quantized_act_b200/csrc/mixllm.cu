@@ -272,6 +272,52 @@ mixllm_status mixllm_gemm_w4w8a8_small_m(const int8_t *A_q, const float *s_a, in
   return ok();
 }
 
+mixllm_status mixllm_small_m_debug_workspace_bytes(int64_t M, int64_t K, int64_t N4, int64_t N8, int32_t kind,
+                                                   size_t *bytes) {
+  mixllm_status st = check_k(K, MIXLLM_GROUP);
+  if (st != MIXLLM_OK) return st;
+  if (!bytes) return fail(MIXLLM_ERR_INVALID_ARG, "null bytes");
+  if (M < 1 || M > 64) return fail(MIXLLM_ERR_INVALID_ARG, "the small-M path takes 1 <= M <= 64");
+  if (N4 < 0 || N8 < 0 || N4 + N8 > 0x7FFFFFF0) return fail(MIXLLM_ERR_INVALID_ARG, "bad N4 / N8");
+  if (!mixllm::small_m_kernel_allowed(M, N4, N8, K, kind))
+    return fail(MIXLLM_ERR_UNSUPPORTED, "few-token kernel %d cannot take M = %lld, K = %lld", static_cast<int>(kind),
+                static_cast<long long>(M), static_cast<long long>(K));
+  *bytes = mixllm::small_m_debug_workspace_bytes(M, N4, N8, K, kind);
+  return ok();
+}
+
+mixllm_status mixllm_small_m_debug_partials(const int8_t *A_q, const float *s_a, int64_t M, int64_t K,
+                                            const uint8_t *W4, const uint8_t *z4, const void *s_w4_f16,
+                                            const int32_t *idx4, int64_t N4, const int8_t *W8,
+                                            const void *s_w8_f16, const int32_t *idx8, int64_t N8, int32_t kind,
+                                            int32_t *P, void *Y_f16, void *workspace, size_t workspace_bytes,
+                                            void *stream) {
+  if (M < 1 || M > 64) return fail(MIXLLM_ERR_INVALID_ARG, "the small-M path takes 1 <= M <= 64");
+  if (N4 + N8 > 0 && (!Y_f16 || !P)) return fail(MIXLLM_ERR_INVALID_ARG, "null Y or P");
+  bool empty = false;
+  mixllm_status st =
+      check_gemm(A_q, s_a, M, K, W4, z4, s_w4_f16, idx4, N4, W8, s_w8_f16, idx8, N8, Y_f16, nullptr, &empty);
+  if (st != MIXLLM_OK) return st;
+  if (empty) return ok();
+  if (!mixllm::small_m_kernel_allowed(M, N4, N8, K, kind))
+    return fail(MIXLLM_ERR_UNSUPPORTED, "few-token kernel %d cannot take M = %lld, K = %lld", static_cast<int>(kind),
+                static_cast<long long>(M), static_cast<long long>(K));
+  if (!aligned(P, 4)) return fail(MIXLLM_ERR_INVALID_ARG, "P must be 4-byte aligned");
+  const size_t need = mixllm::small_m_debug_workspace_bytes(M, N4, N8, K, kind);
+  if (workspace_bytes < need)
+    return fail(MIXLLM_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu this shape needs",
+                workspace_bytes, need);
+  if (need > 0 && (!workspace || !aligned(workspace, 16)))
+    return fail(MIXLLM_ERR_INVALID_ARG, "workspace must be a 16-byte aligned device buffer");
+  mixllm::GemmArgs a{A_q, s_a, M, K, W4, z4, s_w4_f16, idx4, N4, W8, s_w8_f16, idx8, N8, Y_f16, P};
+  const char *msg = "";
+  cudaError_t e = mixllm::launch_small_m_debug_partials(a, kind, workspace, workspace_bytes,
+                                                        static_cast<cudaStream_t>(stream), &msg);
+  if (e == cudaErrorNotSupported) return fail(MIXLLM_ERR_UNSUPPORTED, "%s", msg);
+  if (e != cudaSuccess) return fail(MIXLLM_ERR_CUDA, "%s: %s", msg, cudaGetErrorString(e));
+  return ok();
+}
+
 mixllm_status mixllm_gemm_w4w8a8_small_m_noalloc(const int8_t *A_q, const float *s_a, int64_t M, int64_t K,
                                                  const uint8_t *W4, const uint8_t *z4, const void *s_w4_f16,
                                                  const int32_t *idx4, int64_t N4, const int8_t *W8,

@@ -6,11 +6,14 @@ import pytest
 
 torch = pytest.importorskip("torch")
 
+import oracle  # noqa: E402
 import mixed_precision_quantized_act_b200 as mx  # noqa: E402
 from mixed_precision_quantized_act_b200 import workloads as wl  # noqa: E402
 from mixed_precision_quantized_act_b200.layer import LinearChain  # noqa: E402
 
 pytestmark = pytest.mark.gpu
+
+REL, ABS_RMS = 2.0 ** -9, 1e-3
 
 
 @pytest.fixture(scope="module")
@@ -61,5 +64,13 @@ def test_graph_replay_equals_eager_and_single_calls(dev, M):
     for l, p, x, y in zip(layers, packed, chain.inputs, chain.outputs):
         ref = mx.linear(x, p)
         assert torch.equal(ref.view(torch.int16), y.view(torch.int16)), l.name
+    # and every linear of the replayed chain against the oracle on its inputs
+    for l, x, y in zip(layers, chain.inputs, chain.outputs):
+        X = x.cpu().numpy()
+        A_o, s_o = oracle.quantize_act(X)
+        Y_o = oracle.gemm_w4w8a8(A_o, s_o, oracle.Quantized(wl.make_w(l, 31), wl.make_bitmap(l, 31))).astype(np.float64)
+        rms = float(np.sqrt(np.mean(Y_o ** 2)))
+        err = np.abs(y.cpu().numpy().astype(np.float64) - Y_o)
+        assert (err <= REL * np.abs(Y_o) + ABS_RMS * rms).all(), l.name
     chain.release()
     assert chain.ops() == sum(2 * M * l.N * l.K for l in layers)

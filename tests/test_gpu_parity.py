@@ -258,6 +258,106 @@ def test_full_size_sampled_rows(dev, layer):
     assert torch.isfinite(Y).all()
 
 
+# full-size launches of the partials debug path: the headline shape (G = 32)
+# and one shape of each larger workload family (long K, a bit mix, multi-wave)
+FULL_P = [wl.Q_PROJ_P10, wl.LLAMA8B_LAYER[3], [l for l in wl.BIT_MIX if "p50" in l.name][0], wl.LLAMA70B[1]]
+
+
+@pytest.mark.parametrize("layer", FULL_P, ids=lambda l: l.name)
+def test_full_size_partials_sampled(dev, layer):
+    """The int32 group partials of a full-size launch, bit-exact on sampled
+    token rows (first, middle and last M tiles and an M-tile boundary) x
+    sampled output columns from both channel sets."""
+    X, W, is8 = layer_inputs(layer, 4)
+    A_q, s_a, p, _ = gpu_layer(dev, X, W, is8)
+    P = mx.gemm_debug_partials(A_q, s_a, p)
+    mx.sync_status()
+    assert P.shape == (layer.M, layer.N, layer.K // 128)
+    rows = np.array(sorted(set([0, 127, 128, layer.M // 2, layer.M - 1])))
+    rng = np.random.default_rng(7)
+    c8 = np.flatnonzero(is8)
+    c4 = np.flatnonzero(is8 == 0)
+    cols = np.sort(np.concatenate([rng.choice(c4, min(384, c4.size), replace=False),
+                                   rng.choice(c8, min(128, c8.size), replace=False),
+                                   [0, layer.N - 1]])).astype(np.int64)
+    cols = np.unique(cols)
+    A_ref, _ = oracle.quantize_act(X[rows])
+    P_ref = oracle.group_partials(A_ref, oracle.Quantized(W[cols], is8[cols]))
+    Pg = P[torch.from_numpy(rows).to(dev)][:, torch.from_numpy(cols).to(dev)].cpu().numpy()
+    assert np.array_equal(Pg, P_ref)
+    del P
+
+
+def _extreme_layer(dev, M, K, n4, n8, w_mag, seed):
+    """Weights whose every group is constant (+w_mag or -w_mag per channel and
+    group) and activations of +-1 per (token, group): every 4-bit product is
+    (q - z) * a = +-15 * 127 and every 8-bit one +-127 * 127, so each group
+    partial reaches the bound of its set, +-243840 or +-2064512."""
+    rng = np.random.default_rng(seed)
+    G = K // 128
+    N = n4 + n8
+    sw = rng.choice([-1.0, 1.0], size=(N, G)).astype(np.float32)
+    W = np.repeat(sw, 128, axis=1) * np.float32(w_mag)
+    sx = rng.choice([-1.0, 1.0], size=(M, G)).astype(np.float16)
+    X = np.repeat(sx, 128, axis=1)
+    is8 = np.zeros(N, np.uint8)
+    is8[rng.choice(N, n8, replace=False)] = 1
+    return X, W, is8
+
+
+def test_partials_reach_the_bounds_of_both_sets(dev):
+    M, K, n4, n8 = 130, 512, 200, 60
+    X, W, is8 = _extreme_layer(dev, M, K, n4, n8, 0.5, 11)
+    A_q, s_a, p, Y = gpu_layer(dev, X, W, is8)
+    P = mx.gemm_debug_partials(A_q, s_a, p).cpu().numpy()
+    mx.sync_status()
+    A_ref, s_ref = oracle.quantize_act(X)
+    P_ref = oracle.group_partials(A_ref, oracle.Quantized(W, is8))
+    assert np.array_equal(P, P_ref)
+    mag = np.abs(P)
+    assert (mag[:, is8 == 0] == 15 * 127 * 128).all()
+    assert (mag[:, is8 == 1] == 127 * 127 * 128).all()
+    assert (P == 243840).any() and (P == -243840).any()
+    assert (P == 2064512).any() and (P == -2064512).any()
+    Y_ref = oracle.gemm_w4w8a8(A_ref, s_ref, oracle.Quantized(W, is8))
+    assert_y_close(Y.cpu().numpy(), Y_ref, "extreme partials")
+
+
+def test_y_overflow_to_inf_matches_oracle(dev):
+    """Large weights drive some outputs past the fp16 range: those are +-inf
+    on both sides (same sign), and the rest stay within the tolerance."""
+    M, K, n4, n8 = 64, 1024, 160, 40
+    X, W, is8 = _extreme_layer(dev, M, K, n4, n8, 100.0, 12)
+    # one channel in each set with small weights: finite, mixed with the inf ones
+    W[np.flatnonzero(is8 == 0)[0]] *= np.float32(1e-3)
+    W[np.flatnonzero(is8 == 1)[0]] *= np.float32(1e-3)
+    A_q, s_a, p, Y = gpu_layer(dev, X, W, is8)
+    A_ref, s_ref = oracle.quantize_act(X)
+    Y_ref = oracle.gemm_w4w8a8(A_ref, s_ref, oracle.Quantized(W, is8)).astype(np.float64)
+    Yg = Y.cpu().numpy().astype(np.float64)
+    inf_ref = np.isinf(Y_ref)
+    assert inf_ref.any() and (~inf_ref).any()
+    assert np.array_equal(np.isinf(Yg), inf_ref)
+    assert np.array_equal(np.sign(Yg[inf_ref]), np.sign(Y_ref[inf_ref]))
+    assert not np.isnan(Yg).any()
+    fin = ~inf_ref
+    rms = float(np.sqrt(np.mean(Y_ref[fin] ** 2)))
+    err = np.abs(Yg[fin] - Y_ref[fin])
+    assert (err <= REL * np.abs(Y_ref[fin]) + ABS_RMS * rms).all()
+
+
+@pytest.mark.parametrize("layer", [wl.TINY, SMALL[6], wl.Q_PROJ_P10], ids=lambda l: l.name)
+def test_plain_i2f_ablation_gives_the_same_bytes(dev, layer):
+    """The plain int->float convert and the bias trick both round P*s_w once,
+    so the two forms of the tiled kernel write bit-identical Y."""
+    X, W, is8 = layer_inputs(layer, 8)
+    A_q, s_a, p, Y = gpu_layer(dev, X, W, is8)
+    Y2 = torch.full_like(Y, float("nan"))
+    mx.gemm_w4w8a8_plain_i2f_into(A_q, s_a, p, Y2)
+    mx.sync_status()
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+
+
 def test_hang_guard_reports_timeout_and_context_survives(dev):
     from mixed_precision_quantized_act_b200 import _lib
     mx.sync_status()

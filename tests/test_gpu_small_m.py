@@ -149,3 +149,54 @@ def test_small_m_linear_dispatch_and_validation(dev):
         mx.gemm_w4w8a8_small_m(A65, s65, p, ws)
     assert ei.value.status == _lib.ERR_INVALID_ARG
     mx.sync_status()
+
+
+# Every few-token kernel on shapes of its own range and on shapes the plan
+# would give to another kernel: exact int32 group partials and Y of the
+# kernel that ran.  (kind, layer): token bounds 1 / 2 / 4 / 8 of the GEMVs,
+# 16 / 32 / 64 of the tensor-core kernel, ragged N, multiple splits, both sets.
+DEBUG_CASES = [
+    ("GEMV split-K", _layer("dbg_gs_m1", 1, 300, 384, 37)),
+    ("GEMV split-K", _layer("dbg_gs_m3", 3, 1000, 2048, 101)),
+    ("GEMV split-K", _layer("dbg_gs_m8", 8, 640, 4096, 64)),
+    ("GEMV split-K", wl.Q_PROJ_P10.with_m(2)),
+    ("GEMV persistent", _layer("dbg_gp_m1", 1, 1000, 2048, 101)),
+    ("GEMV persistent", _layer("dbg_gp_m2", 2, 300, 1024, 37)),
+    ("GEMV persistent", _layer("dbg_gp_m4", 4, 640, 8192, 64)),
+    ("tensor-core split-K", _layer("dbg_tc_m1", 1, 300, 384, 37)),
+    ("tensor-core split-K", _layer("dbg_tc_m9", 9, 1000, 1024, 101)),
+    ("tensor-core split-K", _layer("dbg_tc_m32", 32, 640, 2048, 64)),
+    ("tensor-core split-K", _layer("dbg_tc_m64_p0", 64, 512, 512, 0)),
+    ("tensor-core split-K", wl.Q_PROJ_P10.with_m(40)),
+]
+
+
+@pytest.mark.parametrize("kind,layer", DEBUG_CASES, ids=lambda v: v if isinstance(v, str) else v.name)
+def test_small_m_kernel_partials_bit_exact(dev, kind, layer):
+    X, W, is8 = wl.make_x(layer, 13), wl.make_w(layer, 13), wl.make_bitmap(layer, 13)
+    A_q, s_a = mx.quantize_act(torch.from_numpy(X).to(dev))
+    p = mx.pack_weights(torch.from_numpy(W).to(dev), torch.from_numpy(is8).to(dev))
+    Y, P = mx.small_m_debug_partials(A_q, s_a, p, kind)
+    mx.sync_status()
+    A_ref, s_ref = oracle.quantize_act(X)
+    q = oracle.Quantized(W, is8)
+    assert np.array_equal(P.cpu().numpy(), oracle.group_partials(A_ref, q))
+    assert_y_close(Y.cpu().numpy(), oracle.gemm_w4w8a8(A_ref, s_ref, q), f"{kind} {layer.name}")
+
+
+def test_small_m_debug_rejects_kernels_outside_their_range(dev):
+    layer = _layer("dbg_reject", 9, 256, 512, 16)
+    p = mx.empty_packed(layer.N, layer.K, layer.N8, dev)
+    A_q = torch.zeros((9, layer.K), dtype=torch.int8, device=dev)
+    s_a = torch.zeros((9, layer.K // 128), dtype=torch.float32, device=dev)
+    for kind in ("GEMV split-K", "GEMV persistent"):
+        with pytest.raises(_lib.MixLLMError) as ei:
+            mx.small_m_debug_partials(A_q, s_a, p, kind)
+        assert ei.value.status == _lib.ERR_UNSUPPORTED
+    # the persistent GEMV keeps every token's codes resident: M*K <= 32768
+    with pytest.raises(_lib.MixLLMError) as ei:
+        mx.small_m_debug_partials(A_q[:4].repeat(1, 32)[:, :16384].contiguous(),
+                                  torch.zeros((4, 128), dtype=torch.float32, device=dev),
+                                  mx.empty_packed(256, 16384, 16, dev), "GEMV persistent")
+    assert ei.value.status == _lib.ERR_UNSUPPORTED
+    mx.sync_status()

@@ -22,9 +22,9 @@ The ring sizes are read from the kernel's source, so a change to them is
 checked here; the last tests plant mistakes (a done ring shorter than a
 stage's worth of groups, a stage released by its last group's commit alone,
 a scale-table slot released after the first of its groups) and expect the
-model to find them.  (An unpack warp that skipped its wait for the MMAs of
-the buffer's previous group would be no mistake with these sizes: the chunk
-it unpacks lands only after those MMAs, which the model confirms.)
+model to find them; and that the unpack's own wait for its buffer's previous
+MMAs matters exactly when the unpacked buffers are fewer than the groups two
+stages hold.
 """
 import os
 import random
@@ -281,11 +281,11 @@ def test_kernel_protocol_holds_under_random_interleavings(G, tiles, is4):
         Model(G, tiles, is4, c, random.Random(seed * 1000 + G * 10 + tiles)).run()
 
 
-def _finds(c, is4, release_last_only=False, table_early=False, runs=120):
+def _finds(c, is4, release_last_only=False, table_early=False, unpack_no_wait=False, runs=120):
     found = 0
     for seed in range(runs):
         try:
-            Model(8, 3, is4, c, random.Random(seed), release_last_only, table_early).run()
+            Model(8, 3, is4, c, random.Random(seed), release_last_only, table_early, unpack_no_wait).run()
         except Violation:
             found += 1
     return found
@@ -310,11 +310,13 @@ def test_model_finds_a_table_slot_released_early():
     assert _finds(kernel_constants(), True, table_early=True) > 0
 
 
-def test_model_confirms_the_unpack_wait_is_implied():
-    """With 2 stages of 4 groups and 8 unpacked buffers, the packed bytes of
-    group gi land only after the MMAs of group gi - 8: dropping the unpack's
-    own wait for them breaks nothing (the kernel keeps it, so other ring sizes
-    stay safe)."""
+def test_unpack_wait_matters_exactly_when_buffers_are_fewer_than_staged_groups():
+    """The unpack's wait for the MMAs of its buffer's previous group is
+    implied by the stage ring when kTBufs >= kStages * kC4 (the chunk it
+    unpacks lands only after those MMAs) and needed otherwise: dropping it is
+    caught then, and harmless with the larger buffer count."""
     c = kernel_constants()
-    for seed in range(40):
-        Model(8, 3, True, c, random.Random(seed), unpack_no_wait=True).run()
+    needed = c["kTBufs"] < c["kStages"] * c["kC4"]
+    assert needed == (_finds(c, True, unpack_no_wait=True) > 0)
+    big = dict(c, kTBufs=c["kStages"] * c["kC4"], kDone=max(c["kDone"], c["kStages"] * c["kC4"]))
+    assert _finds(big, True, unpack_no_wait=True) == 0

@@ -55,6 +55,27 @@ def test_no_alloc_matches_the_workspace_entry_point_twice_in_a_row(dev, layer):
     assert (err <= REL * np.abs(Y_o) + ABS_RMS * rms).all()
 
 
+def test_no_alloc_runs_the_persistent_gemv_on_a_large_layer(dev):
+    # 70B gate_up at one token: the plan picks the persistent GEMV, whose
+    # scratch (unit partials + counters) must also come from the static array
+    layer = wl.LLAMA70B[2].with_m(1)
+    assert mx.small_m_kernel(1, layer.K, layer.N - layer.N8, layer.N8) == "GEMV persistent"
+    g = torch.Generator(device="cpu").manual_seed(5)
+    X = (torch.randn((1, layer.K), generator=g) * 0.5).to(torch.float16).to(dev)
+    W = (torch.randn((layer.N, layer.K), generator=g) * 0.02).to(dev)
+    is8 = torch.from_numpy(wl.make_bitmap(layer, 5)).to(dev)
+    A_q, s_a = mx.quantize_act(X)
+    p = mx.pack_weights(W, is8)
+    del W
+    ws = mx.small_m_workspace(1, p, dev)
+    Y_ref = mx.gemm_w4w8a8_small_m(A_q, s_a, p, ws)
+    for _ in range(2):
+        Y = torch.full_like(Y_ref, float("nan"))
+        mx.gemm_w4w8a8_small_m_noalloc_into(A_q, s_a, p, Y)
+        mx.sync_status()
+        assert torch.equal(Y.view(torch.int16), Y_ref.view(torch.int16))
+
+
 def test_no_alloc_rejects_a_shape_larger_than_its_scratch(dev):
     # 70B down at M=64: 7 splits x 65 tiles x 64 x 128 fp32 partials = 14.9 MB > 8 MiB
     layer = wl.LLAMA70B[3]
