@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="argument and rank plumbing only (gloo on CPU, no kernels): rank 0 prints the "
+                         "configuration, every rank's batch seed and the max over ranks of a stand-in time")
     return ap.parse_args()
 
 
@@ -159,27 +162,55 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ oracle leg
 
-def oracle_rate(layer, X, W, is8, target_s):
-    """Time the CPU oracle (quantize + two-step GEMM), single-threaded, on
-    token rows of the workload, cycling through the batch until about
-    `target_s` seconds of work; returns (TOPS-equivalent, seconds, rows)."""
+def _oracle_rows_worker(name, seed, r0, target_s, sub_cols, start, out_q):
+    """One host core's share of the oracle baseline: quantize + two-step GEMM
+    on token rows r0, r0+1, ... (cycling over the batch) until about
+    `target_s` seconds; puts (rows, seconds) on out_q."""
     import oracle
+    layer = wl.by_name(name)
+    X, W, is8 = wl.make_x(layer, seed), wl.make_w(layer, seed), wl.make_bitmap(layer, seed)
+    if sub_cols is not None:
+        W, is8 = W[:sub_cols], is8[:sub_cols]
     Wq = oracle.Quantized(W, is8)  # offline weight quantization, not timed
+    A, s = oracle.quantize_act(X[r0:r0 + 1])  # warm-up and calibration row
     t0 = time.perf_counter()
-    A, s = oracle.quantize_act(X[:1])
     oracle.gemm_w4w8a8(A, s, Wq)
-    t1 = max(time.perf_counter() - t0, 1e-6)
-    rows = int(max(1, target_s / t1))
-    done, dt = 0, 0.0
+    per_row = max(time.perf_counter() - t0, 1e-6)
+    rows = int(max(1, target_s / per_row))
+    start.wait()  # every process has quantized its weights and calibrated
+    done, r, t0 = 0, r0, time.perf_counter()
     while done < rows:
-        r0 = done % layer.M
-        n = min(rows - done, layer.M - r0)
-        t0 = time.perf_counter()
-        A, s = oracle.quantize_act(X[r0:r0 + n])
+        r = r % layer.M
+        n = min(rows - done, layer.M - r)
+        A, s = oracle.quantize_act(X[r:r + n])
         oracle.gemm_w4w8a8(A, s, Wq)
-        dt += time.perf_counter() - t0
         done += n
-    return 2.0 * rows * layer.N * layer.K / dt / 1e12, dt, rows
+        r += n
+    out_q.put((done, time.perf_counter() - t0))
+
+
+def oracle_rate(layer, seed, target_s, cores=None, sub_cols=None):
+    """Time the CPU oracle (quantize + two-step GEMM, unmodified) on the
+    box's host cores: one spawned process per core, each on its own token
+    rows of the workload, started together; returns (TOPS-equivalent over all
+    rows / the slowest process's time, seconds, rows, cores).  Spawned, not
+    forked: the parent may already hold a CUDA context."""
+    import multiprocessing as mp
+    cores = cores or os.cpu_count() or 1
+    ctx = mp.get_context("spawn")
+    start, out_q = ctx.Barrier(cores), ctx.Queue()
+    procs = [ctx.Process(target=_oracle_rows_worker,
+                         args=(layer.name, seed, (i * layer.M) // cores, target_s, sub_cols, start, out_q))
+             for i in range(cores)]
+    for pr in procs:
+        pr.start()
+    res = [out_q.get() for _ in procs]
+    for pr in procs:
+        pr.join()
+    rows = sum(r for r, _ in res)
+    secs = max(t for _, t in res)
+    n = min(layer.N, sub_cols) if sub_cols else layer.N
+    return 2.0 * rows * n * layer.K / secs / 1e12, secs, rows, cores
 
 
 # ------------------------------------------------------------------ reference arm
@@ -416,10 +447,11 @@ def run_ours(args, layer, rank, world, local_rank):
     if rank == 0:
         cpu = None
         if world == 1:
-            rate, secs, rows = oracle_rate(layer, X, W, is8, args.cpu_seconds)
-            cpu = {"value": rate, "unit": UNIT, "cores": 1, "host_cores": os.cpu_count(), "kind": "oracle",
+            rate, secs, rows, cores = oracle_rate(layer, args.seed, args.cpu_seconds)
+            cpu = {"value": rate, "unit": UNIT, "cores": cores, "host_cores": os.cpu_count(), "kind": "oracle",
                    "sample": f"{rows} token rows (cycling over the {layer.M}-row batch) x all {layer.N} "
-                             f"channels x K={layer.K}, quantize + two-step GEMM, {secs:.1f} s single-threaded"}
+                             f"channels x K={layer.K}, quantize + two-step GEMM, one process per host core "
+                             f"on its own rows, {secs:.1f} s (slowest process)"}
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True, "scaling": "weak",
@@ -669,8 +701,41 @@ def run_search(args, rank, world, local_rank):
     }
 
 
+def run_dry(args, rank, world):
+    """The launch plumbing of a multi-GPU run without a GPU: the process group
+    (gloo), each rank's batch seed, the barrier and the max over ranks of a
+    per-rank time, and the whole-job unit count, as the timed runs use them."""
+    import torch.distributed as tdist
+    dp.init("gloo", timeout_s=60)
+    try:
+        name = args.workload
+        if name.startswith(LAYER_WORKLOAD) or name == SEARCH_WORKLOAD:
+            config, m = {"workload": name, "parallelism": f"dp{world}"}, None
+        else:
+            layer = layer_for(name)
+            config, m = config_of(layer, world), layer.M
+        seed = dp.batch_seed(args.seed, rank)
+        seeds = [None] * world
+        if world > 1:
+            tdist.all_gather_object(seeds, seed)
+        else:
+            seeds = [seed]
+        dp.barrier(world)
+        tmax = dp.max_over_ranks(1.0 + 0.25 * rank, world)  # stand-in per-rank time (ms)
+        if rank == 0:
+            print(json.dumps({"dry_run": True, "impl": args.impl, "n_gpus": args.gpus, "world": world,
+                              "steps": args.steps, "warmup": args.warmup, "config": config, "seeds": seeds,
+                              "ms_per_step_max_over_ranks": tmax,
+                              "units": dp.total_units(m, world) if m is not None else None}), flush=True)
+    finally:
+        dp.shutdown(world)
+
+
 def main():
     args = parse()
+    if args.dry_run:
+        run_dry(args, int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")))
+        return
     if args.workload == SEARCH_WORKLOAD:
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "the search workload has no reference arm; "

@@ -61,6 +61,33 @@ def max_over_ranks(x: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def shard_rows(m_total: int, rank: int, world: int) -> tuple:
+    """Token rows [start, stop) of a global batch of `m_total` rows that rank
+    `rank` of `world` takes: contiguous shards whose sizes differ by at most
+    one, the larger ones first (strong scaling: a fixed batch split over GPUs)."""
+    base, extra = divmod(m_total, world)
+    start = rank * base + min(rank, extra)
+    return start, start + base + (1 if rank < extra else 0)
+
+
+def gather_rows(local: torch.Tensor, m_total: int, world: int) -> torch.Tensor:
+    """The ranks' row shards (as cut by shard_rows) put back together in rank
+    order on every rank.  Shards are padded to the largest for all_gather."""
+    if world == 1:
+        return local
+    if local.element_size() < 4:  # narrow types go through int32 (not every backend gathers them)
+        narrow = {1: torch.int8, 2: torch.int16}[local.element_size()]
+        wide = gather_rows(local.view(narrow).to(torch.int32), m_total, world)
+        return wide.to(narrow).view(local.dtype)
+    rows = [shard_rows(m_total, r, world) for r in range(world)]
+    width = max(stop - start for start, stop in rows)
+    pad = torch.zeros((width,) + tuple(local.shape[1:]), dtype=local.dtype, device=local.device)
+    pad[:local.shape[0]] = local
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad)
+    return torch.cat([parts[r][:stop - start] for r, (start, stop) in enumerate(rows)])
+
+
 def total_units(units_per_rank: int, world: int) -> int:
     """Work done by the whole job when each rank processes `units_per_rank`."""
     return units_per_rank * world

@@ -8,6 +8,7 @@ import socket
 import subprocess
 import sys
 import textwrap
+import json
 
 import pytest
 
@@ -84,3 +85,68 @@ def test_missing_rank_times_out_instead_of_hanging():
     """, ranks=[0], timeout=90)
     rc, out, err = outs[0]
     assert "joined" not in out
+
+
+def test_shard_rows_cover_the_batch_once():
+    sys.path.insert(0, ROOT)
+    from mixed_precision_quantized_act_b200 import dist as d
+    for m in (0, 1, 7, 37, 512):
+        for world in (1, 2, 3, 8):
+            cuts = [d.shard_rows(m, r, world) for r in range(world)]
+            assert cuts[0][0] == 0 and cuts[-1][1] == m
+            assert all(a[1] == b[0] for a, b in zip(cuts, cuts[1:]))
+            sizes = [b - a for a, b in cuts]
+            assert max(sizes) - min(sizes) <= 1
+
+
+def test_two_ranks_token_shards_reassemble_the_single_rank_layer():
+    """Each gloo rank quantizes and multiplies its own token shard with the
+    oracle layer; the gathered A_q, s_a and Y equal one rank's result on the
+    whole batch, bit for bit (the rows of a batch are independent)."""
+    outs = _run_ranks("""
+        import numpy as np
+        import oracle
+        from mixed_precision_quantized_act_b200 import workloads as wl
+        info = d.init("gloo", timeout_s=60)
+        layer = wl.Linear("dp_shard", 37, 200, 256, ((0, 200, 21),), 3)
+        X, W, is8 = wl.make_x(layer, 4), wl.make_w(layer, 4), wl.make_bitmap(layer, 4)
+        q = oracle.Quantized(W, is8)
+        r0, r1 = d.shard_rows(layer.M, info.rank, info.world)
+        A, s = oracle.quantize_act(X[r0:r1])
+        Y = oracle.gemm_w4w8a8(A, s, q)
+        A_all = d.gather_rows(torch.from_numpy(A), layer.M, info.world).numpy()
+        s_all = d.gather_rows(torch.from_numpy(s), layer.M, info.world).numpy()
+        Y_all = d.gather_rows(torch.from_numpy(Y), layer.M, info.world).numpy()
+        A_1, s_1 = oracle.quantize_act(X)
+        Y_1 = oracle.gemm_w4w8a8(A_1, s_1, q)
+        ok = (np.array_equal(A_all, A_1) and np.array_equal(s_all.view(np.uint32), s_1.view(np.uint32))
+              and np.array_equal(Y_all.view(np.uint16), Y_1.view(np.uint16)))
+        print(json.dumps({"rank": info.rank, "rows": [r0, r1], "ok": bool(ok)}))
+        d.shutdown(info.world)
+    """, timeout=180)
+    res = []
+    for rc, out, err in outs:
+        assert rc == 0, err
+        res.append(json.loads(out.strip().splitlines()[-1]))
+    assert sorted(tuple(r["rows"]) for r in res) == [(0, 19), (19, 37)]
+    assert all(r["ok"] for r in res)
+
+
+def test_bench_two_rank_dry_run_through_torchrun():
+    """bench.py --gpus 2 as the driver launches it (torch.distributed.run, two
+    ranks), with --dry-run: gloo instead of NCCL and no kernels, so the
+    argument, rank and max-over-ranks plumbing is checked on CPU."""
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--gpus", "2", "--steps", "5", "--warmup", "3", "--dry-run"]
+    p = subprocess.run(cmd, capture_output=True, text=True, timeout=180, cwd=ROOT)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [l for l in p.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1  # rank 0 alone prints
+    line = json.loads(lines[0])
+    assert line["dry_run"] and line["world"] == 2 and line["n_gpus"] == 2
+    assert line["seeds"] == [0, 1]
+    assert line["ms_per_step_max_over_ranks"] == 1.25
+    assert line["units"] == 2 * line["config"]["M"]
+    assert line["config"]["parallelism"].startswith("dp2")
