@@ -55,7 +55,10 @@ typedef enum {
     MIXLLM_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad size      */
     MIXLLM_ERR_UNSUPPORTED = 2, /* group != 128, K % 128 != 0, no sm_100a  */
     MIXLLM_ERR_CUDA = 3,        /* a CUDA runtime call failed              */
-    MIXLLM_ERR_TIMEOUT = 4      /* a device-side wait gave up              */
+    MIXLLM_ERR_TIMEOUT = 4,     /* a device-side wait gave up              */
+    MIXLLM_ERR_BOUNDS = 5       /* checked build: a kernel's range check of
+                                   a tensor- or shared-memory access failed
+                                   (the access was skipped)                */
 } mixllm_status;
 
 #define MIXLLM_GROUP 128
@@ -388,8 +391,9 @@ MIXLLM_API mixllm_status mixllm_select_top_t(const float *S, int64_t n, int64_t 
 /*
  * Waits for `stream`, then reads and clears the device status word of the
  * current device.  Returns MIXLLM_ERR_TIMEOUT if a kernel of this library
- * gave up a wait since the last call, MIXLLM_ERR_CUDA if the stream reports
- * a CUDA error, MIXLLM_OK otherwise.  SYNCHRONOUS.
+ * gave up a wait since the last call, MIXLLM_ERR_BOUNDS if (checked build
+ * only) a range check failed, MIXLLM_ERR_CUDA if the stream reports a CUDA
+ * error, MIXLLM_OK otherwise.  SYNCHRONOUS.
  */
 MIXLLM_API mixllm_status mixllm_sync_status(void *stream);
 
@@ -401,6 +405,24 @@ MIXLLM_API mixllm_status mixllm_sync_status(void *stream);
  * with mixllm_sync_status().
  */
 MIXLLM_API mixllm_status mixllm_selftest_wait_timeout(uint32_t limit_us, void *stream);
+
+/*
+ * 1 if this is the checked build of the library (every tensor- and
+ * shared-memory access of the GEMM kernels is range-checked first; a failed
+ * check skips the access and records MIXLLM_ERR_BOUNDS), 0 for the release
+ * build.  Pure host function.
+ */
+MIXLLM_API int mixllm_checked_build(void);
+
+/*
+ * Self-test of the checked build's range checks: launches one small kernel
+ * that checks a tensor-memory column range and a shared-memory range which
+ * both lie outside their windows (no access is made), so a checked build
+ * records MIXLLM_ERR_BOUNDS in the device status word.  The release build
+ * returns MIXLLM_ERR_UNSUPPORTED and launches nothing.  Asynchronous; read
+ * the result with mixllm_sync_status().
+ */
+MIXLLM_API mixllm_status mixllm_selftest_bounds(void *stream);
 
 #ifdef __cplusplus
 }

@@ -30,7 +30,9 @@ from ._lib import (  # noqa: F401
     select_top_t,
     select_top_t_into,
     select_top_t_workspace,
+    selftest_bounds,
     selftest_wait_timeout,
+    checked_build,
     small_m_kernel,
     small_m_debug_partials,
     small_m_workspace,

@@ -17,8 +17,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libmixllm_b200.so")
 GROUP = 128
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
-_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIMEOUT"}
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = 0, 1, 2, 3, 4, 5
+_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIMEOUT", 5: "BOUNDS"}
 
 # Every entry point declared in include/mixllm.h, with (restype, argtypes).
 _i64, _i32, _u32, _vp = ctypes.c_int64, ctypes.c_int32, ctypes.c_uint32, ctypes.c_void_p
@@ -54,6 +54,8 @@ SIGNATURES = {
                                                      ctypes.c_size_t, _vp]),
     "mixllm_sync_status": (ctypes.c_int, [_vp]),
     "mixllm_selftest_wait_timeout": (ctypes.c_int, [_u32, _vp]),
+    "mixllm_checked_build": (ctypes.c_int, []),
+    "mixllm_selftest_bounds": (ctypes.c_int, [_vp]),
 }
 
 
@@ -67,11 +69,14 @@ _lock = threading.Lock()
 _lib = None
 
 
-def load(path: str = LIB_PATH):
-    """Load the CUDA library (raises if it was not built)."""
+def load(path: str = None):
+    """Load the CUDA library (raises if it was not built).  The path defaults
+    to the in-tree release build; the environment variable MIXLLM_LIBRARY
+    names another build of the same library (e.g. the checked one)."""
     global _lib
     with _lock:
         if _lib is None:
+            path = path or os.environ.get("MIXLLM_LIBRARY") or LIB_PATH
             if not os.path.exists(path):
                 raise RuntimeError(
                     f"{path} is missing: build it with `python -m mixed_precision_quantized_act_b200.build`")
@@ -351,6 +356,17 @@ def linear(X: torch.Tensor, p: PackedLinear, stream=None, workspace: torch.Tenso
 
 def sync_status(stream=None):
     _check(load().mixllm_sync_status(_stream(stream)), "mixllm_sync_status")
+
+
+def checked_build() -> bool:
+    """True when the loaded library is the range-checked build."""
+    return bool(load().mixllm_checked_build())
+
+
+def selftest_bounds(stream=None):
+    """Checked build: makes the range checks fire without an access (read the
+    result with sync_status); the release build raises UNSUPPORTED."""
+    _check(load().mixllm_selftest_bounds(_stream(stream)), "mixllm_selftest_bounds")
 
 
 def selftest_wait_timeout(limit_us: int, stream=None):

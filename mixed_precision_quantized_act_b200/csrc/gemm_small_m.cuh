@@ -221,12 +221,21 @@ __global__ void __launch_bounds__(kSmThreads, 1)
   // where local group i lives: its chunk's stage, its offset in the chunk, the phase of the stage
   auto gstage = [&](int i) { return (i / gpc) % nst; };
   auto gphase = [&](int i) { return static_cast<uint32_t>(((i / gpc) / nst) & 1); };
+  // checked builds: the shared-memory window every access must stay in
+  const uint32_t smem_lo = smem_u32(smem), smem_hi = smem_lo + static_cast<uint32_t>(C::kSmemBytes);
+  (void)smem_lo, (void)smem_hi;
   auto load = [&](int c) {  // chunk c (local groups c*gpc ..) into stage c % nst
     const int s = c % nst, i0 = c * gpc, g = g0 + i0;
     const int n = min(gpc, ng - i0);
     // boxes always land whole (groups past the CTA's last come from the next
     // split or are zero past K; tokens past M are zero) and are never read
     const uint32_t wb = is4 ? static_cast<uint32_t>(n) * C::kW4Bytes : static_cast<uint32_t>(C::kChunkWBytes);
+    if (!(chk_smem(smem_u32(stage_x(s)), C::kGpc4 * C::kXBytes, smem_lo, smem_hi) &&
+          chk_smem(smem_u32(stage_w(s)), wb, smem_lo, smem_hi) &&
+          (!is4 || chk_smem(smem_u32(zmeta(s)), C::kGpc4 * 64u, smem_lo, smem_hi)))) {
+      mbar_arrive_expect_tx(&full[s], 0u);  // checked build: no copy, the phase completes empty
+      return;
+    }
     mbar_arrive_expect_tx(&full[s], wb + static_cast<uint32_t>(C::kGpc4 * C::kXBytes) + (is4 ? C::kGpc4 * 64u : 0u));
     tma_load_3d(stage_x(s), &tmX, &full[s], 0, 0, g);
     if (is4) {
@@ -301,7 +310,15 @@ __global__ void __launch_bounds__(kSmThreads, 1)
         tc_fence_after();
         const uint32_t b_addr = smem_u32(stage_x(s) + j * C::kXBytes);  // tokens: MP rows x 128 k
         const uint32_t d = tmem_base + static_cast<uint32_t>(a * MP);
-        if (is4 && C::kTmemW) {  // weights: 128 channels x 128 k, unpacked into tensor memory
+        bool in_range = chk_tmem(d, tmem_base, C::kTmemCols, MP, 128) && chk_smem(b_addr, C::kXBytes, smem_lo, smem_hi);
+        if (is4 && C::kTmemW)
+          in_range = in_range && chk_tmem(tmem_base + static_cast<uint32_t>(C::kTmemABase + b * 32), tmem_base,
+                                          C::kTmemCols, 32, 128);
+        else
+          in_range = in_range && chk_smem(smem_u32(is4 ? tbuf(b) : stage_w(s) + j * C::kWBytes), 16384, smem_lo, smem_hi);
+        if (!in_range) {
+          // checked build: the group's MMAs are skipped, its commit still signals
+        } else if (is4 && C::kTmemW) {  // weights: 128 channels x 128 k, unpacked into tensor memory
           const uint32_t wt = tmem_base + static_cast<uint32_t>(C::kTmemABase + b * 32);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) mma_i8_ts(d, wt + 8 * kk, sw128_kmajor_desc(b_addr + 32 * kk), idesc, 1u);
@@ -392,7 +409,8 @@ __global__ void __launch_bounds__(kSmThreads, 1)
           o[8 * k + 6] = sm_sub_zero_bytes((x[k].z >> 4) & 0x0F0F0F0Fu, zz);
           o[8 * k + 7] = sm_sub_zero_bytes((x[k].w >> 4) & 0x0F0F0F0Fu, zz);
         }
-        tmem_st_32x32b_x32(trow + static_cast<uint32_t>(b * 32), o);
+        if (chk_tmem(trow + static_cast<uint32_t>(b * 32), tmem_base, C::kTmemCols, 32))
+          tmem_st_32x32b_x32(trow + static_cast<uint32_t>(b * 32), o);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -455,7 +473,9 @@ __global__ void __launch_bounds__(kSmThreads, 1)
     // Every accumulator starts at the bias 0x4b400000 and is reset to it after
     // each drain, so the int32 sum read as a float is 1.5*2^23 + P exactly.
 #pragma unroll
-    for (int a = 0; a < C::kAccBufs; ++a) sm_tmem_fill<MP>(lane_base + static_cast<uint32_t>(a * MP), kI2FBiasBits);
+    for (int a = 0; a < C::kAccBufs; ++a)
+      if (chk_tmem(lane_base + static_cast<uint32_t>(a * MP), tmem_base, C::kTmemCols, MP))
+        sm_tmem_fill<MP>(lane_base + static_cast<uint32_t>(a * MP), kI2FBiasBits);
     tmem_st_wait();
     tc_fence_before();
     __syncwarp();
@@ -489,10 +509,11 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       for (int h = 0; h < MP / CH; ++h) {
         uint32_t r[CH];
         const uint32_t col = lane_base + static_cast<uint32_t>(a * MP + h * CH);
-        sm_tmem_ld<CH>(col, r);
+        const bool col_ok = chk_tmem(col, tmem_base, C::kTmemCols, CH);
+        if (col_ok) sm_tmem_ld<CH>(col, r);
         tmem_ld_wait();
         sm_reg_fence<CH>(r);
-        sm_tmem_fill<CH>(col, kI2FBiasBits);  // hand the columns back preset to the bias
+        if (col_ok) sm_tmem_fill<CH>(col, kI2FBiasBits);  // hand the columns back preset to the bias
         if constexpr (DBG) {
           if (pd != nullptr)
             for (int t = 0; t < CH; ++t)

@@ -290,6 +290,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nchunks = sched.count * nch;   // chunks this CTA loads
   const int a_bytes = CH * C::kABytes;
   const int stage_bytes = is4 ? C::kStage4 : C::kStage8;
+  // checked builds: the shared-memory window every access must stay in
+  const uint32_t smem_lo = smem_u32(smem), smem_hi = smem_lo + static_cast<uint32_t>(C::kSmemBytes);
+  (void)smem_lo, (void)smem_hi;
   auto stage_a = [&](int s) { return smem + C::kOffRing + s * stage_bytes; };
   auto stage_w = [&](int s) { return smem + C::kOffRing + s * stage_bytes + a_bytes; };
   auto zmeta = [&](int s) { return smem + C::kOffZ + s * C::kC4 * C::kZBytes; };
@@ -311,11 +314,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int s = ci % S;
     if (is4) {
       const uint32_t wb = static_cast<uint32_t>(k.ng * C::kW4Bytes);
+      if (!(chk_smem(smem_u32(stage_a(s)), a_bytes, smem_lo, smem_hi) &&
+            chk_smem(smem_u32(stage_w(s)), wb, smem_lo, smem_hi) &&
+            chk_smem(smem_u32(zmeta(s)), C::kC4 * C::kZBytes, smem_lo, smem_hi))) {
+        mbar_arrive_expect_tx(&full[s], 0u);  // checked build: no copy, the phase completes empty
+        return;
+      }
       mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(a_bytes) + wb + static_cast<uint32_t>(C::kC4 * C::kZBytes));
       tma_load_3d(stage_a(s), tmA, &full[s], 0, k.m0, k.g0);
       bulk_load(stage_w(s), W4 + (static_cast<int64_t>(k.n0 >> 7) * G + k.g0) * C::kW4Bytes, wb, &full[s]);
       tma_load_2d(zmeta(s), &tmZ, &full[s], k.n0 >> 1, k.g0);
     } else {
+      if (!(chk_smem(smem_u32(stage_a(s)), a_bytes, smem_lo, smem_hi) &&
+            chk_smem(smem_u32(stage_w(s)), a_bytes, smem_lo, smem_hi))) {
+        mbar_arrive_expect_tx(&full[s], 0u);
+        return;
+      }
       mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(2 * a_bytes));
       tma_load_3d(stage_a(s), tmA, &full[s], 0, k.m0, k.g0);
       tma_load_3d(stage_w(s), &tmW8, &full[s], 0, k.n0, k.g0);
@@ -411,7 +425,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t x_addr = smem_u32(stage_a(st) + j * C::kABytes);
           const uint32_t d = tmem_base + static_cast<uint32_t>(a * kBM);
-          if (is4) {
+          bool in_range = chk_tmem(d, tmem_base, C::kTmemCols, kBM, 128) && chk_smem(x_addr, C::kABytes, smem_lo, smem_hi);
+          if (is4)
+            in_range = in_range && chk_tmem(tmem_base + static_cast<uint32_t>(C::kTmemABase + b * C::kTmemABufCols),
+                                            tmem_base, C::kTmemCols, C::kTmemABufCols, 128);
+          else
+            in_range = in_range && chk_smem(smem_u32(stage_w(st) + j * C::kW8Bytes), C::kW8Bytes, smem_lo, smem_hi);
+          if (!in_range) {
+            // checked build: the group's MMAs are skipped, its commit still signals
+          } else if (is4) {
             const uint32_t wt = tmem_base + static_cast<uint32_t>(C::kTmemABase + b * C::kTmemABufCols);
 #pragma unroll
             for (int kk = 0; kk < kKG / 32; ++kk)
@@ -448,6 +470,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto publish = [&](int gi, const uint8_t *raw_sw, const float *sa_src, int sa_stride) {
         // raw_sw: the tile's BN fp16 s_w of this group; sa_src[t * sa_stride]: s_a of token t
+        if (!(chk_smem(smem_u32(table_w(gi)), C::kTabBytes, smem_lo, smem_hi) &&
+              chk_smem(smem_u32(raw_sw), BN * 2, smem_lo, smem_hi) &&
+              chk_smem(smem_u32(sa_src), static_cast<uint32_t>(((kBM - 1) * sa_stride + 1) * 4), smem_lo, smem_hi)))
+          return;  // checked build: the entry is left as it was
         const uint2 raw = *reinterpret_cast<const uint2 *>(raw_sw + 8 * lane);
         const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&raw.x));
         const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&raw.y));
@@ -473,6 +499,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nscc = G / C::kScG;  // raw chunks per tile
         auto load_sc = [&](const ChunkCursor &k, int c) {
           const int st = c % C::kScStages;
+          if (!chk_smem(smem_u32(sc_raw(st)), C::kScBytes, smem_lo, smem_hi)) {
+            mbar_arrive_expect_tx(&scfull[st], 0u);  // checked build: no copy
+            return;
+          }
           mbar_arrive_expect_tx(&scfull[st], static_cast<uint32_t>(C::kScBytes));
           tma_load_2d(sc_raw(st), tmSw, &scfull[st], k.n0, k.g0);
           tma_load_2d(sc_raw(st) + C::kScSwBytes, &tmSa, &scfull[st], k.g0, k.m0);
@@ -579,11 +609,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
         }
         const uint8_t *src = stage_w(r) + j * C::kW4Bytes + rr * 64;
+        const bool in_range =
+            warp_all_checked(chk_smem(smem_u32(src), 64, smem_lo, smem_hi) &&
+                             chk_smem(smem_u32(zmeta(r) + j * C::kZBytes + (rr >> 1)), 1, smem_lo, smem_hi)) &&
+            chk_tmem(trow + static_cast<uint32_t>(b * C::kTmemABufCols), tmem_base, C::kTmemCols, C::kTmemABufCols);
         uint4 x[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) x[c] = *reinterpret_cast<const uint4 *>(src + (((c + rot) & 3) << 4));
+        for (int c = 0; c < 4; ++c)
+          x[c] = in_range ? *reinterpret_cast<const uint4 *>(src + (((c + rot) & 3) << 4)) : make_uint4(0, 0, 0, 0);
         const uint32_t zz =
-            ((static_cast<uint32_t>(zmeta(r)[j * C::kZBytes + (rr >> 1)]) >> zshift) & 0xFu) * 0x01010101u;
+            in_range ? ((static_cast<uint32_t>(zmeta(r)[j * C::kZBytes + (rr >> 1)]) >> zshift) & 0xFu) * 0x01010101u
+                     : 0u;
         // x[c] holds chunk (c + rot) & 3: rotate back by rot = (rot & 1) + (rot & 2)
         if (rot & 1) {
           const uint4 t3 = x[3];
@@ -614,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           o[8 * c + 7] = sub_zero_bytes((x[c].w >> 4) & 0x0F0F0F0Fu, zz);
         }
         __syncwarp();
-        tmem_st_32x32b_x32(trow + static_cast<uint32_t>(b * C::kTmemABufCols), o);
+        if (in_range) tmem_st_32x32b_x32(trow + static_cast<uint32_t>(b * C::kTmemABufCols), o);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -640,7 +676,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int a = 0; a < C::kAccBufs; ++a)
 #pragma unroll
-      for (int c = 0; c < CPT; c += 32) tmem_st_32x32b_x32_fill(lane_base + a * kBM + c, kPreset);
+      for (int c = 0; c < CPT; c += 32)
+        if (chk_tmem(lane_base + a * kBM + c, tmem_base, C::kTmemCols, 32)) tmem_st_32x32b_x32_fill(lane_base + a * kBM + c, kPreset);
     tmem_st_wait();
     tc_fence_before();
     __syncwarp();
@@ -682,7 +719,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int CW = CPT > 32 ? MIXLLM_EPI_CW : 16, NCH = CPT / CW;
         constexpr bool kDB = CPT > 32;
         uint32_t rb[kDB ? 2 : 1][CW];
-        tmem_ld_cols(col, rb[0]);
+        // checked build: this warp's CPT accumulator columns (uniform over the warp)
+        const bool acc_ok = chk_tmem(col, tmem_base, C::kTmemCols, CPT);
+        if (acc_ok) tmem_ld_cols(col, rb[0]);
         if (gi % C::kTabG == 0 &&
             !warp_wait_u32(a_tabfull + 8 * tslot, (gi / (C::kTabG * C::kTabSlots)) & 1, abort_flag)) {
           tmem_ld_wait();
@@ -690,19 +729,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const uint32_t tab = a_tab + tslot * C::kTabSlotBytes + (gi % C::kTabG) * C::kTabBytes;
-        const float4 w = lds_f4(tab + 16 * ch);
         const uint32_t tsa = tab + C::kTabWBytes + part * CPT * 4;
+        const bool tab_ok = warp_all_checked(chk_smem(tab + 16 * ch, 16, smem_lo, smem_hi) &&
+                                             chk_smem(tsa, CPT * 4, smem_lo, smem_hi));
+        const float4 w = tab_ok ? lds_f4(tab + 16 * ch) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         const float2 sw2 = make_float2(w.x, w.y);
         const float2 cb2 = make_float2(w.z, w.w);
 #pragma unroll
         for (int h = 0; h < NCH; ++h) {
           uint32_t(&r)[CW] = rb[kDB ? (h & 1) : 0];
-          if (!kDB && h > 0) tmem_ld_cols(col + CW * h, r);
+          if (acc_ok && !kDB && h > 0) tmem_ld_cols(col + CW * h, r);
           tmem_ld_wait();
           reg_fence(r);
-          if (kDB && h + 1 < NCH) tmem_ld_cols(col + CW * (h + 1), rb[(h + 1) & 1]);
+          if (acc_ok && kDB && h + 1 < NCH) tmem_ld_cols(col + CW * (h + 1), rb[(h + 1) & 1]);
           // hand the columns back preset (its wait is after the math)
-          tmem_fill_cols<CW>(col + CW * h, kPreset);
+          if (acc_ok) tmem_fill_cols<CW>(col + CW * h, kPreset);
           if constexpr (kDebugP) {
             if (nout >= 0) {
 #pragma unroll 4
@@ -721,7 +762,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // of 4 consecutive tokens per 16 bytes.
 #pragma unroll
             for (int j = 0; j < CW / 4; ++j) {
-              const float4 sa = lds_f4(tsa + 16 * ((CW / 4) * h + j));
+              const float4 sa = tab_ok ? lds_f4(tsa + 16 * ((CW / 4) * h + j)) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
               float2 v0, v1;
               if constexpr (kCvtI2F) {
                 v0 = make_float2(__int2float_rn(static_cast<int>(r[4 * j])),

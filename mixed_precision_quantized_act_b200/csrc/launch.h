@@ -69,6 +69,7 @@ cudaError_t launch_gemm_small_m_noalloc(const GemmArgs &a, cudaStream_t stream, 
 size_t small_m_scratch_capacity();
 
 cudaError_t launch_selftest_wait_timeout(uint32_t limit_us, cudaStream_t stream);
+cudaError_t launch_selftest_bounds(cudaStream_t stream);
 
 // Global mixed-precision search (search.cuh).
 cudaError_t launch_channel_salience(const float *W, int64_t N, int64_t K, const float *G, int64_t D, float *S,

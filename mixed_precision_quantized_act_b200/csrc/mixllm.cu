@@ -437,8 +437,21 @@ mixllm_status mixllm_sync_status(void *stream) {
     e = cudaMemcpyToSymbol(mixllm::g_status, &zero, sizeof(int));
     if (e != cudaSuccess) return cuda_fail(e, "status clear");
     if (status == mixllm::kStatusTimeout) return fail(MIXLLM_ERR_TIMEOUT, "a device-side wait gave up");
+    if (status == mixllm::kStatusBounds)
+      return fail(MIXLLM_ERR_BOUNDS, "a range check of the checked build failed (the access was skipped)");
     return fail(MIXLLM_ERR_INVALID_ARG, "device reported status %d", status);
   }
+  return ok();
+}
+
+int mixllm_checked_build(void) { return MIXLLM_CHECKED ? 1 : 0; }
+
+mixllm_status mixllm_selftest_bounds(void *stream) {
+  if (!MIXLLM_CHECKED) return fail(MIXLLM_ERR_UNSUPPORTED, "the release build has no range checks");
+  mixllm_status st = check_device();
+  if (st != MIXLLM_OK) return st;
+  cudaError_t e = mixllm::launch_selftest_bounds(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
   return ok();
 }
 

@@ -14,12 +14,60 @@ namespace mixllm {
 // library is one translation unit, so this header holds the definition.
 __device__ int g_status = 0;
 
-enum : int { kStatusOk = 0, kStatusTimeout = 4, kStatusBadBitmap = 1 };
+enum : int { kStatusOk = 0, kStatusTimeout = 4, kStatusBadBitmap = 1, kStatusBounds = 5 };
 
 __device__ __forceinline__ void record_status(int code) { atomicCAS(&g_status, 0, code); }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ------------------------------------------------------------ checked build
+// With MIXLLM_CHECKED=1 (a separate build of the library, off in release)
+// the GEMM kernels range-check every tensor-memory and shared-memory access
+// before making it: a failed check records kStatusBounds in the status word
+// and the access is skipped (nothing traps).  Release builds compile the
+// checks away.
+#ifndef MIXLLM_CHECKED
+#define MIXLLM_CHECKED 0
+#endif
+
+// nlanes lanes x ncols columns from TMEM address taddr (lane in bits
+// 31..16, column in 15..0) stay within lanes 0..127 and the alloc_cols
+// columns allocated at base.
+__device__ __forceinline__ bool chk_tmem(uint32_t taddr, uint32_t base, int alloc_cols, int ncols, int nlanes = 32) {
+#if MIXLLM_CHECKED
+  const uint32_t lane = taddr >> 16, col = taddr & 0xFFFFu, c0 = base & 0xFFFFu;
+  const bool ok = lane + static_cast<uint32_t>(nlanes) <= 128u && col >= c0 &&
+                  col + static_cast<uint32_t>(ncols) <= c0 + static_cast<uint32_t>(alloc_cols);
+  if (!ok) record_status(kStatusBounds);
+  return ok;
+#else
+  (void)taddr, (void)base, (void)alloc_cols, (void)ncols, (void)nlanes;
+  return true;
+#endif
+}
+
+// The check result agreed by the whole warp (checked builds; true otherwise).
+__device__ __forceinline__ bool warp_all_checked(bool ok) {
+#if MIXLLM_CHECKED
+  return __all_sync(0xFFFFFFFFu, ok);
+#else
+  (void)ok;
+  return true;
+#endif
+}
+
+// bytes at shared address addr stay within [lo, hi).
+__device__ __forceinline__ bool chk_smem(uint32_t addr, uint32_t bytes, uint32_t lo, uint32_t hi) {
+#if MIXLLM_CHECKED
+  const bool ok = addr >= lo && addr + bytes <= hi && addr + bytes >= addr;
+  if (!ok) record_status(kStatusBounds);
+  return ok;
+#else
+  (void)addr, (void)bytes, (void)lo, (void)hi;
+  return true;
+#endif
 }
 
 // ----------------------------------------------------------------- mbarrier

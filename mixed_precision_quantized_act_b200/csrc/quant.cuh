@@ -45,61 +45,78 @@ namespace mixllm {
 // the codes are returned packed, lowest k first; returns s_a.  Shared by
 // quantize_act_kernel and the fused decode GEMV.
 __device__ __forceinline__ float quant_act_8x16(const uint4 raw, unsigned mask, uint32_t (&packed)[2]) {
+  // the eight values stay packed as fp16 pairs and are widened where used
   const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw);
-  float x[8];
+  auto xval = [&](int i) {
+    const float2 f = __half22float2(h2[i >> 1]);
+    return (i & 1) ? f.y : f.x;
+  };
+  __half2 m2 = __habs2(h2[0]);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __half22float2(h2[i]);
-    x[2 * i] = f.x;
-    x[2 * i + 1] = f.y;
-  }
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  for (int i = 1; i < 4; ++i) m2 = __hmax2(m2, __habs2(h2[i]));
+  float amax = fmaxf(__low2float(m2), __high2float(m2));
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(mask, amax, o));
   const float s = __fdiv_rn(amax, 127.0f);
   packed[0] = packed[1] = 0u;
   if (s != 0.0f) {
+    // Integers below 2^22 in magnitude are rounded and converted with the
+    // 1.5*2^23 offset: fl(t + 1.5*2^23) - 1.5*2^23 is rint(t) (ties to even,
+    // the default rounding of the add), and the bits of fl(q + 1.5*2^23) are
+    // 0x4b400000 + q.  The explicit _rn intrinsics keep the compiler from
+    // fusing the multiply into the add.
+    constexpr float kMagic = 12582912.0f;
     const float r = __frcp_rn(s);
     const float half_s = 0.5f * s;
     const float margin = s * 0x1p-14f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int q0 = __float2int_rn(x[i] * r);
-      const float e = __fmaf_rn(-static_cast<float>(q0), s, x[i]);  // exact remainder x - q0*s
+      const float xi = xval(i);
+      const float q0 = __fadd_rn(__fadd_rn(__fmul_rn(xi, r), kMagic), -kMagic);  // rint(fl(x * (1/s)))
+      const float e = __fmaf_rn(-q0, s, xi);  // exact remainder x - q0*s
       const float d = fabsf(e) - half_s;
-      int qi;
+      float qf;
       if (fabsf(d) > margin) {
-        qi = d > 0.0f ? q0 + (e > 0.0f ? 1 : -1) : q0;
+        qf = d > 0.0f ? q0 + (e > 0.0f ? 1.0f : -1.0f) : q0;
       } else {
-        qi = __float2int_rn(__fdiv_rn(x[i], s));  // near a half-integer: the IEEE quotient, rounded
+        // near a half-integer: the IEEE quotient, rounded
+        qf = __fadd_rn(__fadd_rn(__fdiv_rn(xi, s), kMagic), -kMagic);
       }
-      qi = max(-127, min(127, qi));
-      packed[i >> 2] |= (static_cast<uint32_t>(qi) & 0xFFu) << ((i & 3) * 8);
+      qf = fminf(127.0f, fmaxf(-127.0f, qf));
+      const uint32_t qi = static_cast<uint32_t>(__float_as_int(__fadd_rn(qf, kMagic)) - 0x4b400000);
+      packed[i >> 2] |= (qi & 0xFFu) << ((i & 3) * 8);
     }
   }
   return s;
 }
 
-__global__ void __launch_bounds__(256) quantize_act_kernel(const __half *__restrict__ X, int64_t M, int64_t K,
-                                                           int8_t *__restrict__ A_q, float *__restrict__ s_a) {
+// One half-warp per (token, group): 16 lanes x one 16-byte load.  The grid
+// is one wave of 8 blocks per SM where the layer allows (the register bound
+// below), so every load of a layer's activations is in flight at once and
+// the kernel costs about one load round trip.  I: the index type (32-bit
+// when M*K fits, which keeps the kernel within that bound).
+constexpr int kQuantThreads = 256;
+
+template <typename I>
+__global__ void __launch_bounds__(kQuantThreads, sizeof(I) == 4 ? 8 : 1) quantize_act_kernel(const __half *__restrict__ X, I M, I K,
+                                                                        int8_t *__restrict__ A_q,
+                                                                        float *__restrict__ s_a) {
   // the GEMM that consumes A_q and s_a may start its prologue now; it reads
   // them only after this grid has completed
   pdl_launch_dependents();
-  const int64_t G = K >> 7;
-  const int64_t total = M * G;
+  const I G = K >> 7;
+  const I total = M * G;
   const int lane16 = threadIdx.x & 15;
   const unsigned mask = 0xFFFFu << (threadIdx.x & 16);
-  const int64_t stride = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 4;
-  for (int64_t hw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4; hw < total; hw += stride) {
-    const int64_t m = hw / G, g = hw - m * G;
-    const int64_t off = m * K + (g << 7) + lane16 * 8;
+  const I stride = (static_cast<I>(gridDim.x) * blockDim.x) >> 4;
+  for (I hw = (static_cast<I>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4; hw < total; hw += stride) {
+    const I m = hw / G, g = hw - m * G;
+    const I off = m * K + (g << 7) + lane16 * 8;
     const uint4 raw = *reinterpret_cast<const uint4 *>(X + off);
     uint32_t packed[2];
     const float s = quant_act_8x16(raw, mask, packed);
     *reinterpret_cast<uint2 *>(A_q + off) = make_uint2(packed[0], packed[1]);
-    if (lane16 == 0) s_a[m * G + g] = s;
+    if (lane16 == 0) s_a[hw] = s;  // s_a[m, g] is element m*G + g = hw
   }
 }
 
@@ -310,9 +327,14 @@ static int grid_for(int64_t threads_needed, int block) {
 
 cudaError_t launch_quantize_act(const void *X, int64_t M, int64_t K, int8_t *A_q, float *s_a, cudaStream_t stream) {
   const int64_t groups = M * (K >> 7);
-  const int64_t blocks = (groups + 15) / 16;
+  constexpr int kPerBlock = kQuantThreads / 16;  // groups per block and pass
+  const int64_t blocks = (groups + kPerBlock - 1) / kPerBlock;
   const int grid = static_cast<int>(blocks < 148 * 64 ? blocks : 148 * 64);
-  quantize_act_kernel<<<grid, 256, 0, stream>>>(static_cast<const __half *>(X), M, K, A_q, s_a);
+  if (M * K < (int64_t{1} << 31))
+    quantize_act_kernel<uint32_t><<<grid, kQuantThreads, 0, stream>>>(
+        static_cast<const __half *>(X), static_cast<uint32_t>(M), static_cast<uint32_t>(K), A_q, s_a);
+  else
+    quantize_act_kernel<int64_t><<<grid, kQuantThreads, 0, stream>>>(static_cast<const __half *>(X), M, K, A_q, s_a);
   return cudaGetLastError();
 }
 
@@ -335,6 +357,23 @@ cudaError_t launch_pack_w8(const float *W, int64_t N, int64_t K, const int32_t *
   const int64_t warps = N8p * (K >> 7);
   pack_w8_kernel<<<grid_for(warps * 32, 256), 256, 0, stream>>>(W, N, K, idx8, N8, N8p, W8,
                                                                  static_cast<__half *>(s_w8));
+  return cudaGetLastError();
+}
+
+// The checked build's range checks on ranges that lie outside their windows:
+// one column past a 32-column allocation, lanes 112..143, and 16 bytes that
+// straddle the end of the dynamic shared memory.  Nothing is accessed.
+__global__ void selftest_bounds_kernel(uint32_t tmem_base) {
+  extern __shared__ uint8_t dyn[];
+  const uint32_t lo = smem_u32(dyn), hi = lo + 256;
+  bool ok = chk_tmem(tmem_base + 1, tmem_base, 32, 32);
+  ok = chk_tmem(tmem_base + (112u << 16), tmem_base, 32, 1) && ok;
+  ok = chk_smem(hi - 8, 16, lo, hi) && ok;
+  if (ok && threadIdx.x == 0) record_status(kStatusBadBitmap);  // unreachable in a checked build
+}
+
+cudaError_t launch_selftest_bounds(cudaStream_t stream) {
+  selftest_bounds_kernel<<<1, 32, 256, stream>>>(0u);
   return cudaGetLastError();
 }
 
