@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--i2f", choices=["bias", "plain"], default="bias",
+                    help="tiled GEMM's int32->float step: the 0x4b400000 bias trick (the method) or, as the "
+                         "ablation of the fast-I2F design point, a plain convert per element (same Y)")
     ap.add_argument("--dry-run", action="store_true",
                     help="argument and rank plumbing only (gloo on CPU, no kernels): rank 0 prints the "
                          "configuration, every rank's batch seed and the max over ranks of a stand-in time")
@@ -278,6 +281,9 @@ def run_ours(args, layer, rank, world, local_rank):
 
         def gemm(i=0):
             mx.gemm_w4w8a8_small_m_into(A_q, s_a, copies[i % len(copies)], Y, ws, stream)
+    elif args.i2f == "plain":
+        def gemm(i=0):
+            mx.gemm_w4w8a8_plain_i2f_into(A_q, s_a, p, Y, stream)
     else:
         def gemm(i=0):
             mx.gemm_w4w8a8_into(A_q, s_a, p, Y, stream)
@@ -447,7 +453,8 @@ def run_ours(args, layer, rank, world, local_rank):
             if small:
                 mx.gemm_w4w8a8_small_m_into(A_q, s_a, wsets[i % len(wsets)], Yds[b], ws, stream)
             else:
-                mx.gemm_w4w8a8_into(A_q, s_a, wsets[i % len(wsets)], Yds[b], stream)
+                (mx.gemm_w4w8a8_plain_i2f_into if args.i2f == "plain" else mx.gemm_w4w8a8_into)(
+                    A_q, s_a, wsets[i % len(wsets)], Yds[b], stream)
             x_free[b].record(stream)
             y_ready[b].record(stream)
             with torch.cuda.stream(d2h):
@@ -515,7 +522,9 @@ def run_ours(args, layer, rank, world, local_rank):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded N(0,1) X with x20 outlier "
-            "columns, N(0,0.02) W, random 8-bit channel set)", "config": config_of(layer, world, len(copies) if small else 0),
+            "columns, N(0,0.02) W, random 8-bit channel set)",
+            "config": dict(config_of(layer, world, len(copies) if small else 0),
+                           **({"i2f": "plain int->float convert (ablation)"} if args.i2f == "plain" and not small else {})),
             "gemm_kernel": {"path": mx.small_m_kernel(layer.M, layer.K, p.N4, p.N8) if small else "tiled",
                             "ms": t_gemm, "tops": gemm_tops,
                             "frac_of_int8_peak": gemm_tops / int8_peak,
