@@ -141,6 +141,21 @@ MIXLLM_API mixllm_status mixllm_pack_weights(const float *W, int64_t N, int64_t 
                                   int8_t *W8, void *s_w8_f16, int32_t *idx8, void *stream);
 
 /*
+ * The same offline quantization and pre-pack on the host CPU, for weights in
+ * host memory (converting a checkpoint without a GPU): the quantizers,
+ * rounding (IEEE fp32 division, round half to even, fp16 round to nearest)
+ * and packed layout of mixllm_pack_weights, byte for byte.  Every pointer is
+ * HOST memory (W fp32 [N, K] row-major; is8 uint8 [N]; the outputs sized by
+ * mixllm_packed_sizes); nothing touches a device, nothing runs on the layer's
+ * hot path.  SYNCHRONOUS.  Returns MIXLLM_ERR_INVALID_ARG (outputs
+ * untouched) when the bit map flags a number of channels other than N8.
+ */
+MIXLLM_API mixllm_status mixllm_pack_weights_host(const float *W, int64_t N, int64_t K, const uint8_t *is8,
+                                       int64_t N8, int32_t group,
+                                       uint8_t *W4, uint8_t *z4, void *s_w4_f16, int32_t *idx4,
+                                       int8_t *W8, void *s_w8_f16, int32_t *idx8);
+
+/*
  * The fused W4.4A8 GEMM: one launch covers both channel sets.  For each
  * output channel n of a set and token m,
  *   P_g = sum_{k in group g} (W_q[n,k] - z[n,g]) * A_q[m,k]   (int32 exact,

@@ -24,6 +24,7 @@ from ._lib import (  # noqa: F401
     linear_small_m_workspace,
     load,
     pack_weights,
+    pack_weights_host,
     packed_sizes,
     quantize_act,
     quantize_act_into,

@@ -27,6 +27,8 @@ SIGNATURES = {
     "mixllm_last_error": (ctypes.c_char_p, []),
     "mixllm_packed_sizes": (ctypes.c_int, [_i64, _i64, _i64, _i32, ctypes.POINTER(ctypes.c_size_t)]),
     "mixllm_quantize_act": (ctypes.c_int, [_vp, _i64, _i64, _i32, _vp, _vp, _vp]),
+    "mixllm_pack_weights_host": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i64, _i32,
+                                                _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "mixllm_pack_weights": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i64, _i32,
                                            _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "mixllm_gemm_w4w8a8": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64,
@@ -169,6 +171,12 @@ class PackedLinear:
         return sum(t.numel() * t.element_size() for t in
                    (self.W4, self.z4, self.s_w4, self.idx4, self.W8, self.s_w8, self.idx8))
 
+    def to(self, device) -> "PackedLinear":
+        """The same packed layer with every buffer on `device` (a copy)."""
+        return PackedLinear(self.N, self.K, self.N4, self.N8,
+                            *(t.to(device).contiguous() for t in
+                              (self.W4, self.z4, self.s_w4, self.idx4, self.W8, self.s_w8, self.idx8)))
+
 
 def padded(n: int) -> int:
     return (n + 255) // 256 * 256
@@ -205,6 +213,23 @@ def pack_weights(W: torch.Tensor, is8: torch.Tensor, stream=None) -> PackedLinea
     _check(load().mixllm_pack_weights(_ptr(W), N, K, _ptr(is8), N8, GROUP, _ptr(p.W4), _ptr(p.z4),
                                       _ptr(p.s_w4), _ptr(p.idx4), _ptr(p.W8), _ptr(p.s_w8),
                                       _ptr(p.idx8), _stream(stream)), "mixllm_pack_weights")
+    return p
+
+
+def pack_weights_host(W: torch.Tensor, is8: torch.Tensor) -> PackedLinear:
+    """The same pack on the host CPU (mixllm_pack_weights_host): W fp32 [N, K]
+    and is8 uint8 [N] in host memory -> a PackedLinear of CPU tensors with the
+    same bytes as pack_weights (move it to a device with PackedLinear.to)."""
+    _require(not W.is_cuda and not is8.is_cuda, "W and is8 must be host (CPU) tensors")
+    _require(W.dtype == torch.float32 and W.is_contiguous() and W.dim() == 2, "W must be a contiguous fp32 [N, K]")
+    _require(is8.dtype == torch.uint8 and is8.is_contiguous() and is8.numel() == W.shape[0],
+             "is8 must be a contiguous uint8 [N]")
+    N, K = W.shape
+    N8 = int((is8 != 0).sum().item())
+    p = empty_packed(N, K, N8, "cpu")
+    _check(load().mixllm_pack_weights_host(_ptr(W), N, K, _ptr(is8), N8, GROUP, _ptr(p.W4), _ptr(p.z4),
+                                           _ptr(p.s_w4), _ptr(p.idx4), _ptr(p.W8), _ptr(p.s_w8), _ptr(p.idx8)),
+           "mixllm_pack_weights_host")
     return p
 
 

@@ -224,7 +224,12 @@ __global__ void __launch_bounds__(kSmThreads, 1)
   // checked builds: the shared-memory window every access must stay in
   const uint32_t smem_lo = smem_u32(smem), smem_hi = smem_lo + static_cast<uint32_t>(C::kSmemBytes);
   (void)smem_lo, (void)smem_hi;
-  auto load = [&](int c) {  // chunk c (local groups c*gpc ..) into stage c % nst
+  // chunk c (local groups c*gpc ..) into stage c % nst: `weights` arms the
+  // stage's barrier for the whole round and issues the weight copies (the
+  // packed layer: constant, so they may run before the grid dependency
+  // resolves); `tokens` issues the token box (written by the kernel before
+  // this one: only after pdl_wait)
+  auto load = [&](int c, bool weights, bool tokens) {
     const int s = c % nst, i0 = c * gpc, g = g0 + i0;
     const int n = min(gpc, ng - i0);
     // boxes always land whole (groups past the CTA's last come from the next
@@ -233,20 +238,25 @@ __global__ void __launch_bounds__(kSmThreads, 1)
     if (!(chk_smem(smem_u32(stage_x(s)), C::kGpc4 * C::kXBytes, smem_lo, smem_hi) &&
           chk_smem(smem_u32(stage_w(s)), wb, smem_lo, smem_hi) &&
           (!is4 || chk_smem(smem_u32(zmeta(s)), C::kGpc4 * 64u, smem_lo, smem_hi)))) {
-      mbar_arrive_expect_tx(&full[s], 0u);  // checked build: no copy, the phase completes empty
+      if (weights) mbar_arrive_expect_tx(&full[s], 0u);  // checked build: no copy, the phase completes empty
       return;
     }
-    mbar_arrive_expect_tx(&full[s], wb + static_cast<uint32_t>(C::kGpc4 * C::kXBytes) + (is4 ? C::kGpc4 * 64u : 0u));
-    tma_load_3d(stage_x(s), &tmX, &full[s], 0, 0, g);
-    if (is4) {
-      // the tile's packed groups are contiguous 8 KB blocks: one bulk copy
-      bulk_load(stage_w(s), W4 + (static_cast<int64_t>(n0 >> 7) * G + g) * C::kW4Bytes, wb, &full[s]);
-      tma_load_2d(zmeta(s), &tmZ, &full[s], n0 >> 1, g);
-    } else {
-      tma_load_3d(stage_w(s), &tmW8, &full[s], 0, n0, g);
+    if (weights) {
+      mbar_arrive_expect_tx(&full[s], wb + static_cast<uint32_t>(C::kGpc4 * C::kXBytes) + (is4 ? C::kGpc4 * 64u : 0u));
+      if (is4) {
+        // the tile's packed groups are contiguous 8 KB blocks: one bulk copy
+        bulk_load(stage_w(s), W4 + (static_cast<int64_t>(n0 >> 7) * G + g) * C::kW4Bytes, wb, &full[s]);
+        tma_load_2d(zmeta(s), &tmZ, &full[s], n0 >> 1, g);
+      } else {
+        tma_load_3d(stage_w(s), &tmW8, &full[s], 0, n0, g);
+      }
     }
+    if (tokens) tma_load_3d(stage_x(s), &tmX, &full[s], 0, 0, g);
   };
 
+  // the next kernel of the stream may launch now: it reads nothing this one
+  // writes before its own dependency wait
+  pdl_launch_dependents();
   if (threadIdx.x == 0) {
     prefetch_tmap(&tmX);
     prefetch_tmap(is4 ? &tmZ : &tmW8);
@@ -275,11 +285,14 @@ __global__ void __launch_bounds__(kSmThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      // every global read of this grid comes after this wait (here, in the
-      // scale warp, or in roles ordered after these loads by barriers)
-      pdl_wait();
+      // The first stages' weights stream in while the kernel before this
+      // one (the quantizer, or the previous layer) finishes; every read of
+      // data that kernel writes comes after this pdl_wait (here, in the
+      // scale warp, or in roles ordered after these loads by barriers).
       int issued = nch < nst ? nch : nst;
-      for (int c = 0; c < issued; ++c) load(c);
+      for (int c = 0; c < issued; ++c) load(c, true, false);
+      pdl_wait();
+      for (int c = 0; c < issued; ++c) load(c, false, true);
       for (int c = nst; c < nch; ++c) {
         // the stage last held chunk c - nst: free once both issuers' MMAs of it are done
         // (each issuer commits in its own order; there is none between the two)
@@ -288,7 +301,7 @@ __global__ void __launch_bounds__(kSmThreads, 1)
         bool ok = mbar_wait(&done[last % C::kDone], (last / C::kDone) & 1, abort_flag);
         ok = ok && mbar_wait(&done[(last - 1) % C::kDone], ((last - 1) / C::kDone) & 1, abort_flag);
         if (!ok) break;
-        load(c);
+        load(c, true, true);
         issued = c + 1;
       }
       for (int c = (issued > nst ? issued - nst : 0); c < issued; ++c)
@@ -338,10 +351,10 @@ __global__ void __launch_bounds__(kSmThreads, 1)
     // One batch of asynchronous copies for all of this CTA's groups, then a
     // single wait: s_w (fp16, 8 bytes per lane per group, contiguous per
     // group) and s_a (4 bytes per token per group; zero for padding tokens).
-    pdl_wait();
     __half *tsw = reinterpret_cast<__half *>(tab_sw);
-    for (int i = 0; i < ng; ++i)
+    for (int i = 0; i < ng; ++i)  // the layer's scales: constant, before the dependency wait
       cp_async_8(tsw + i * 128 + 4 * lane, s_w + static_cast<int64_t>(g0 + i) * Np + n0 + 4 * lane);
+    pdl_wait();  // s_a is written by the kernel before this one
     for (int e = lane; e < ng * MP; e += 32) {
       const int i = e / MP, t = e - i * MP;
       const bool in = t < M;

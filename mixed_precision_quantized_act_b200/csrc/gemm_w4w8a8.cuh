@@ -310,29 +310,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   // its ng groups (one contiguous bulk copy) and their zero points (one 2-D
   // box), or the 8-bit tiles (one 3-D box).
   const CUtensorMap *tmA = is4 ? &tmA4 : &tmA8;
-  auto load_chunk = [&](const ChunkCursor &k, int ci) {
+  // weights: arm the stage's barrier for the whole round and issue the
+  // weight copies (the packed layer is constant: they may run before the
+  // grid dependency resolves); tokens: the A_q box (written by the quantizer
+  // before this kernel: only after pdl_wait)
+  auto load_chunk = [&](const ChunkCursor &k, int ci, bool weights = true, bool tokens = true) {
     const int s = ci % S;
     if (is4) {
       const uint32_t wb = static_cast<uint32_t>(k.ng * C::kW4Bytes);
       if (!(chk_smem(smem_u32(stage_a(s)), a_bytes, smem_lo, smem_hi) &&
             chk_smem(smem_u32(stage_w(s)), wb, smem_lo, smem_hi) &&
             chk_smem(smem_u32(zmeta(s)), C::kC4 * C::kZBytes, smem_lo, smem_hi))) {
-        mbar_arrive_expect_tx(&full[s], 0u);  // checked build: no copy, the phase completes empty
+        if (weights) mbar_arrive_expect_tx(&full[s], 0u);  // checked build: no copy, the phase completes empty
         return;
       }
-      mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(a_bytes) + wb + static_cast<uint32_t>(C::kC4 * C::kZBytes));
-      tma_load_3d(stage_a(s), tmA, &full[s], 0, k.m0, k.g0);
-      bulk_load(stage_w(s), W4 + (static_cast<int64_t>(k.n0 >> 7) * G + k.g0) * C::kW4Bytes, wb, &full[s]);
-      tma_load_2d(zmeta(s), &tmZ, &full[s], k.n0 >> 1, k.g0);
+      if (weights) {
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(a_bytes) + wb + static_cast<uint32_t>(C::kC4 * C::kZBytes));
+        bulk_load(stage_w(s), W4 + (static_cast<int64_t>(k.n0 >> 7) * G + k.g0) * C::kW4Bytes, wb, &full[s]);
+        tma_load_2d(zmeta(s), &tmZ, &full[s], k.n0 >> 1, k.g0);
+      }
+      if (tokens) tma_load_3d(stage_a(s), tmA, &full[s], 0, k.m0, k.g0);
     } else {
       if (!(chk_smem(smem_u32(stage_a(s)), a_bytes, smem_lo, smem_hi) &&
             chk_smem(smem_u32(stage_w(s)), a_bytes, smem_lo, smem_hi))) {
-        mbar_arrive_expect_tx(&full[s], 0u);
+        if (weights) mbar_arrive_expect_tx(&full[s], 0u);
         return;
       }
-      mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(2 * a_bytes));
-      tma_load_3d(stage_a(s), tmA, &full[s], 0, k.m0, k.g0);
-      tma_load_3d(stage_w(s), &tmW8, &full[s], 0, k.n0, k.g0);
+      if (weights) {
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(2 * a_bytes));
+        tma_load_3d(stage_w(s), &tmW8, &full[s], 0, k.n0, k.g0);
+      }
+      if (tokens) tma_load_3d(stage_a(s), tmA, &full[s], 0, k.m0, k.g0);
     }
   };
   // The producer: stage ci % S is refilled with chunk ci once the MMAs of
@@ -376,14 +384,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < C::kScStages; ++s) mbar_init(&scfull[s], 1);
     *abort_flag = 0;
     fence_mbar_init();
-    // Every global read of this grid comes after a pdl_wait: here, in the
-    // scale warp and the epilogue, and in the roles ordered after these
-    // loads by barriers.
-    pdl_wait();
-    // the first stages need nothing but their barriers: start them before the CTA-wide sync
+    // The first stages need nothing but their barriers: start them before
+    // the CTA-wide sync.  Their weights stream in while the quantizer before
+    // this kernel finishes; every read of data it writes comes after this
+    // pdl_wait (here, in the scale warp and the epilogue, and in the roles
+    // ordered after these loads by barriers).
     pk.start(sched, G, CH, mt, BN);
+    {
+      ChunkCursor wk = pk;
+      for (int ci = 0; ci < S && ci < nchunks; ++ci) {
+        load_chunk(wk, ci, true, false);
+        wk.next(sched, G, CH, nch, mt, BN);
+      }
+    }
+    pdl_wait();
     for (int ci = 0; ci < S && ci < nchunks; ++ci) {
-      load_chunk(pk, ci);
+      load_chunk(pk, ci, false, true);
       pk.next(sched, G, CH, nch, mt, BN);
     }
   }

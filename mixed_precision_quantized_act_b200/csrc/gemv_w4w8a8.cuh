@@ -242,6 +242,9 @@ __global__ void __launch_bounds__(kGvThreads, gemv_min_blocks(MT))
   const int nch = (ng + chunk - 1) / chunk;
   const uint8_t *w4_tile = is4 ? W4 + (static_cast<int64_t>(t_in_set) * G + g0) * 8192 : nullptr;
 
+  // the next kernel of the stream may launch now: it reads nothing this one
+  // writes before its own dependency wait
+  pdl_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGvSlots; ++s) mbar_init(&S.full[s], 1);
     mbar_init(&S.a_full, 1);
@@ -249,9 +252,6 @@ __global__ void __launch_bounds__(kGvThreads, gemv_min_blocks(MT))
     fence_mbar_init();
     if (!is4) prefetch_tmap(&tmW8);
   }
-  // every global read of this grid comes after this wait (the tokens' codes
-  // and scales are written by the kernel before this one)
-  pdl_wait();
   __syncthreads();  // barriers initialized
 
   // chunk c of this CTA's groups into slot c % 2
@@ -274,41 +274,17 @@ __global__ void __launch_bounds__(kGvThreads, gemv_min_blocks(MT))
   // s_a rows as bulk copies too when they are 16-byte pieces (the CTAs of a
   // split read the same few lines: one request per token instead of a warp's loads)
   const bool sa_bulk = !FUSE && ((g0 | ng | G) & 3) == 0 && (reinterpret_cast<uintptr_t>(s_a) & 15) == 0;
+  // The first weight chunks stream in while the kernel before this one
+  // finishes (the packed layer is constant); the tokens' codes, scales or
+  // activations, which that kernel writes, are read only after pdl_wait.
   int issued = 0;
-  if (FUSE && threadIdx.x == 0) {
-    // the tokens' fp16 activations of groups [g0, g1) into the second slot, one
-    // bulk copy per token, and the first weight chunk into the first
-    mbar_arrive_expect_tx(&S.a_full, static_cast<uint32_t>(mt * ng * 256));
-    for (int m = 0; m < mt; ++m)
-      bulk_load(ring + kGvSlotBytes + m * ng * 256, X + static_cast<int64_t>(m) * K + g0 * 128,
-                static_cast<uint32_t>(ng * 256), &S.a_full);
-    issue(issued++);
+  if (threadIdx.x == 0) {
+    if (FUSE)
+      issue(issued++);  // the first chunk into the first slot (the second takes the activations)
+    else
+      for (; issued < kGvSlots && issued < nch; ++issued) issue(issued);
   }
-  if (!FUSE && threadIdx.x == 0) {
-    // the tokens' codes (and scales) of groups [g0, g1): one bulk copy per token, first
-    mbar_arrive_expect_tx(&S.a_full, static_cast<uint32_t>(mt * ng * (128 + (sa_bulk ? 4 : 0))));
-    for (int m = 0; m < mt; ++m) {
-      bulk_load(&S.a[m][0], A_q + static_cast<int64_t>(m) * K + g0 * 128, static_cast<uint32_t>(ng * 128), &S.a_full);
-      if (sa_bulk)
-        bulk_load(&S.sa[m][0], s_a + static_cast<int64_t>(m) * G + g0, static_cast<uint32_t>(ng * 4), &S.a_full);
-    }
-    for (; issued < kGvSlots && issued < nch; ++issued) issue(issued);
-  }
-
-  // stage the tokens' scales, and the tile's zero points and channel scales
-  // of groups [g0, g1), while the codes and weights are on their way
-  {
-    for (int e = threadIdx.x; e < (MT - mt) * ng * 8; e += kGvThreads)  // tokens past M: zero codes
-      *reinterpret_cast<int4 *>(&S.a[mt + e / (ng * 8)][(e % (ng * 8)) * 16]) = make_int4(0, 0, 0, 0);
-    for (int e = threadIdx.x; e < MT * ng; e += kGvThreads) {
-      const int m = e / ng, i = e - m * ng;
-      if (m >= mt) {
-        S.sa[m][i] = 0.0f;
-        if (FUSE) S.asum[m][i] = 0;
-      } else if (!FUSE && !sa_bulk) {
-        S.sa[m][i] = s_a[static_cast<int64_t>(m) * G + g0 + i];
-      }
-    }
+  {  // the tile's channel scales and zero points of groups [g0, g1): constant too
     const __half *swp = is4 ? s_w4 + static_cast<int64_t>(g0) * N4p + n0 : s_w8 + static_cast<int64_t>(g0) * N8p + n0;
     const int64_t sws = is4 ? N4p : N8p;
     for (int e = threadIdx.x; e < ng * 16; e += kGvThreads) {  // 16 pieces of 8 scales per group
@@ -320,6 +296,39 @@ __global__ void __launch_bounds__(kGvThreads, gemv_min_blocks(MT))
         const int i = e >> 2, q = e & 3;
         *reinterpret_cast<uint4 *>(&S.z[i][q * 16]) =
             *reinterpret_cast<const uint4 *>(z4 + static_cast<int64_t>(g0 + i) * (N4p >> 1) + (n0 >> 1) + q * 16);
+      }
+    }
+  }
+  pdl_wait();
+  if (FUSE && threadIdx.x == 0) {
+    // the tokens' fp16 activations of groups [g0, g1) into the second slot, one
+    // bulk copy per token
+    mbar_arrive_expect_tx(&S.a_full, static_cast<uint32_t>(mt * ng * 256));
+    for (int m = 0; m < mt; ++m)
+      bulk_load(ring + kGvSlotBytes + m * ng * 256, X + static_cast<int64_t>(m) * K + g0 * 128,
+                static_cast<uint32_t>(ng * 256), &S.a_full);
+  }
+  if (!FUSE && threadIdx.x == 0) {
+    // the tokens' codes (and scales) of groups [g0, g1): one bulk copy per token
+    mbar_arrive_expect_tx(&S.a_full, static_cast<uint32_t>(mt * ng * (128 + (sa_bulk ? 4 : 0))));
+    for (int m = 0; m < mt; ++m) {
+      bulk_load(&S.a[m][0], A_q + static_cast<int64_t>(m) * K + g0 * 128, static_cast<uint32_t>(ng * 128), &S.a_full);
+      if (sa_bulk)
+        bulk_load(&S.sa[m][0], s_a + static_cast<int64_t>(m) * G + g0, static_cast<uint32_t>(ng * 4), &S.a_full);
+    }
+  }
+
+  // stage the tokens' scales while the codes and weights are on their way
+  {
+    for (int e = threadIdx.x; e < (MT - mt) * ng * 8; e += kGvThreads)  // tokens past M: zero codes
+      *reinterpret_cast<int4 *>(&S.a[mt + e / (ng * 8)][(e % (ng * 8)) * 16]) = make_int4(0, 0, 0, 0);
+    for (int e = threadIdx.x; e < MT * ng; e += kGvThreads) {
+      const int m = e / ng, i = e - m * ng;
+      if (m >= mt) {
+        S.sa[m][i] = 0.0f;
+        if (FUSE) S.asum[m][i] = 0;
+      } else if (!FUSE && !sa_bulk) {
+        S.sa[m][i] = s_a[static_cast<int64_t>(m) * G + g0 + i];
       }
     }
     if (FUSE) {
@@ -596,9 +605,9 @@ __global__ void __launch_bounds__(kGvThreads, 2)
     fence_mbar_init();
     if (geo.nt4 * static_cast<int64_t>(geo.C4) < u1) prefetch_tmap(&tmW8);
   }
-  // every global read of this grid comes after this wait (the tokens' codes
-  // and scales are written by the kernel before this one)
-  pdl_wait();
+  // the next kernel of the stream may launch now: it reads nothing this one
+  // writes before its own dependency wait
+  pdl_launch_dependents();
   __syncthreads();  // barriers initialized
 
   // The next unit to issue, as (tile, chunk): advanced one unit per issue.
@@ -647,15 +656,19 @@ __global__ void __launch_bounds__(kGvThreads, 2)
   // s_a rows as bulk copies too when they are 16-byte pieces (every CTA reads
   // the same few lines: one request per token instead of a warp's loads)
   const bool sa_bulk = (G & 3) == 0 && (reinterpret_cast<uintptr_t>(s_a) & 15) == 0;
+  // The first two units (weights, zero points, scales: the constant packed
+  // layer) stream in while the kernel before this one finishes; the tokens'
+  // codes and scales, which that kernel writes, are read after pdl_wait.
+  for (int k = 0; k < 2 && k < nk; ++k) issue();
+  pdl_wait();
   if (threadIdx.x == 0) {
-    // the tokens' codes (and scales) of all K: one bulk copy per token, ahead of the weights
+    // the tokens' codes (and scales) of all K: one bulk copy per token
     mbar_arrive_expect_tx(a_full, static_cast<uint32_t>(mt * K + (sa_bulk ? mt * G * 4 : 0)));
     for (int m = 0; m < mt; ++m) {
       bulk_load(sA + m * K, A_q + static_cast<int64_t>(m) * K, static_cast<uint32_t>(K), a_full);
       if (sa_bulk) bulk_load(sSa + m * G, s_a + static_cast<int64_t>(m) * G, static_cast<uint32_t>(G * 4), a_full);
     }
   }
-  for (int k = 0; k < 2 && k < nk; ++k) issue();
 
   // the tokens' scales, zero codes for tokens past M, then the sum of each
   // (token, group)'s 128 codes once they have landed

@@ -14,6 +14,7 @@
 #include "gemm_small_m.cuh"
 #include "search.cuh"
 #include "launch.h"
+#include "pack_host.cuh"
 #include "quant.cuh"
 
 namespace {
@@ -198,6 +199,31 @@ mixllm_status mixllm_pack_weights(const float *W, int64_t N, int64_t K, const ui
                   static_cast<long long>(N8));
     return fail(MIXLLM_ERR_TIMEOUT, "a device wait gave up during the pack");
   }
+  return ok();
+}
+
+mixllm_status mixllm_pack_weights_host(const float *W, int64_t N, int64_t K, const uint8_t *is8, int64_t N8,
+                                       int32_t group, uint8_t *W4, uint8_t *z4, void *s_w4_f16, int32_t *idx4,
+                                       int8_t *W8, void *s_w8_f16, int32_t *idx8) {
+  mixllm_status st = check_k(K, group);
+  if (st != MIXLLM_OK) return st;
+  if (N < 0 || N8 < 0 || N8 > N) return fail(MIXLLM_ERR_INVALID_ARG, "need 0 <= N8 <= N");
+  if (N > 0x7FFFFFF0) return fail(MIXLLM_ERR_INVALID_ARG, "N beyond the supported range");
+  if (N == 0) return ok();
+  const int64_t N4 = N - N8;
+  if (!W || !is8) return fail(MIXLLM_ERR_INVALID_ARG, "null W or is8");
+  if (N4 > 0 && (!W4 || !z4 || !s_w4_f16 || !idx4)) return fail(MIXLLM_ERR_INVALID_ARG, "null 4-bit output");
+  if (N8 > 0 && (!W8 || !s_w8_f16 || !idx8)) return fail(MIXLLM_ERR_INVALID_ARG, "null 8-bit output");
+  // the channel lists go to the caller's buffers only once the map is known to be consistent
+  int64_t n8 = 0;
+  for (int64_t n = 0; n < N; ++n) n8 += is8[n] != 0;
+  if (n8 != N8)
+    return fail(MIXLLM_ERR_INVALID_ARG, "the bit map flags %lld channels, not N8 = %lld", static_cast<long long>(n8),
+                static_cast<long long>(N8));
+  (void)mixllm::host_split_channels(is8, N, N8, idx4, idx8);
+  if (N4 > 0)
+    mixllm::host_pack_w4(W, K, idx4, N4, mixllm::padded_channels(N4), W4, z4, static_cast<__half *>(s_w4_f16));
+  if (N8 > 0) mixllm::host_pack_w8(W, K, idx8, N8, mixllm::padded_channels(N8), W8, static_cast<__half *>(s_w8_f16));
   return ok();
 }
 

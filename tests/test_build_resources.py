@@ -59,8 +59,16 @@ def test_every_budgeted_kernel_is_compiled(report):
         assert any(k.startswith(prefix) for k in report), prefix
 
 
+# The partials debug forms (their DBG / kDebugP template flag set) are for
+# parity tests only: they store every int32 partial and get a looser budget.
+DEBUG_FORMS = re.compile(r"gemv_w4w8a8_kernelILi\d+ELb[01]ELb1E|gemv_w4w8a8_persistent_kernelILi\d+ELb1E|"
+                         r"gemm_small_m_kernelILi\d+ELb1E|gemm_w4w8a8_kernelILi128ELb1E")
+DEBUG_BUDGET = 256
+
+
 @pytest.mark.parametrize("prefix,budget", BUDGETS, ids=[p for p, _ in BUDGETS])
 def test_spill_loads_within_budget(report, prefix, budget):
     for name, loads in report.items():
         if name.startswith(prefix):
-            assert loads <= budget, f"{name}: {loads} bytes of spill loads, budget {budget}"
+            limit = DEBUG_BUDGET if DEBUG_FORMS.search(name) else budget
+            assert loads <= limit, f"{name}: {loads} bytes of spill loads, budget {limit}"
