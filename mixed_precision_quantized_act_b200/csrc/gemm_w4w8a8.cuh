@@ -172,6 +172,8 @@ struct GemmCfg {
   static_assert(kABytes % 1024 == 0 && kW8Bytes % 1024 == 0 && kW4Bytes % 1024 == 0, "1024-byte aligned tiles");
   static_assert(kTabBytes % 16 == 0 && kStgBytes % 16 == 0 && kOffTab % 16 == 0 && kOffStg % 128 == 0, "alignment");
   static_assert(kScBytes % 128 == 0 && kScSwBytes % 128 == 0, "TMA destinations");
+  // each stage's zero points are a 2-D TMA box: 128-byte aligned destinations
+  static_assert(kOffZ % 128 == 0 && (kC4 * kZBytes) % 128 == 0, "zero-point stages are TMA destinations");
   static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
 };
 
