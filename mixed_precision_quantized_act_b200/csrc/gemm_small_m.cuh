@@ -104,6 +104,8 @@ struct SmallMCfg {
   static constexpr int kSmemAlloc = kSmemBytes + 1024;
   static_assert(kXBytes % 1024 == 0 && kRingBytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static_assert(2 * (kChunkWBytes + kGpc4 * kXBytes) <= kRingBytes, "two stages must fit");
+  // each stage's zero points are a 2-D TMA box: 128-byte aligned destinations
+  static_assert(kOffZ % 128 == 0 && (kGpc4 * 64) % 128 == 0, "zero-point stages are TMA destinations");
   static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
 };
 
