@@ -339,7 +339,7 @@ __device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
 
 // Warp-uniform bounded wait.  Every lane tests the barrier and the warp votes
 // (measured on B200: ~16 cycles for a phase that has already completed, ten
-// times less than one lane polling and broadcasting its verdict); if the
+// times less than one lane polling and broadcasting its result); if the
 // phase is still open every lane falls back to the bounded wait, and the
 // vote reconverges the warp.  Returns false (on every lane) if the wait gave
 // up.
