@@ -54,9 +54,16 @@ constexpr int kSmRegsCtl = 88, kSmRegsUnpack = 72, kSmRegsEpi = 200;
 static_assert(128 * kSmRegsCtl + 256 * kSmRegsUnpack + 128 * kSmRegsEpi <= 65536, "register split");
 constexpr int kSmGroupsMax = 32;  // groups per CTA (bounds the scale tables)
 
-template <int MP>
+// DUO (16 tokens only): two CTAs per SM -- a two-stage ring and 64
+// registers a thread -- so that on layers with a wave of tiles or more
+// (every CTA resident at once) one CTA's copy and drain latencies overlap
+// the other's.  One CTA per SM with the deeper ring is faster for the
+// smaller layers, which the plan gives more splits instead.
+template <int MP, bool DUO = false>
 struct SmallMCfg {
   static_assert(MP == 16 || MP == 32 || MP == 64, "token tile");
+  static_assert(!DUO || MP == 16, "two CTAs per SM: 16 tokens only");
+  static constexpr int kMinBlocks = DUO ? 2 : 1;
   // The ring holds stages of several groups each (four 4-bit groups, or two
   // 8-bit ones: 32 KiB of weights), loaded with one copy per operand: a CTA's
   // copy rate grows with the bytes per copy, so per-group copies of 8 KiB
@@ -67,7 +74,11 @@ struct SmallMCfg {
   // they would take doubles the ring: 4 stages instead of 2); shared memory
   // for 64 tokens, whose stages are too large for a third one to fit.
   static constexpr bool kTmemW = MP <= 32;
-  static constexpr int kRingBytes = kTmemW ? 192 * 1024 : 128 * 1024;
+  static constexpr int kRingBytes = DUO ? 80 * 1024 : (kTmemW ? 192 * 1024 : 128 * 1024);
+  static constexpr int kRegsCtl = DUO ? 40 : kSmRegsCtl;
+  static constexpr int kRegsUnpack = DUO ? 56 : kSmRegsUnpack;
+  static constexpr int kRegsEpi = DUO ? 88 : kSmRegsEpi;
+  static_assert(128 * kRegsCtl + 256 * kRegsUnpack + 128 * kRegsEpi <= 65536 / kMinBlocks, "register split");
   static constexpr int kGpc4 = 4, kGpc8 = 2;                // groups per chunk
   static constexpr int kChunkWBytes = 32768;
   static constexpr int kMaxStages = 16;
@@ -120,6 +131,7 @@ struct SmallMPlan {
   // persistent GEMV (M <= kGemvMaxM and M*K within its resident-token bound):
   // `ctas` CTAs share `units` 32 KiB units evenly; workspace [ctas][2][MP][128]
   bool persistent;
+  bool duo;  // 16 tokens, two CTAs per SM (SmallMCfg DUO)
   int units, ctas, chunks4, chunks8;
   size_t part_floats, counters;
   size_t bytes() const { return part_floats * 4 + counters * 4; }
@@ -168,8 +180,8 @@ __device__ __forceinline__ void sm_reg_fence(uint32_t (&r)[MP]) {
 }
 
 // DBG: the int32 group partials also go to Pd [M, N, G] (output column order).
-template <int MP, bool DBG = false>
-__global__ void __launch_bounds__(kSmThreads, 1)
+template <int MP, bool DBG = false, bool DUO = false>
+__global__ void __launch_bounds__(kSmThreads, SmallMCfg<MP, DUO>::kMinBlocks)
     gemm_small_m_kernel(const __grid_constant__ CUtensorMap tmX, const uint8_t *__restrict__ W4,
                         const __grid_constant__ CUtensorMap tmW8, const __grid_constant__ CUtensorMap tmZ,
                         const float *__restrict__ s_a,
@@ -178,7 +190,7 @@ __global__ void __launch_bounds__(kSmThreads, 1)
                         const int32_t *__restrict__ idx8, int M, int K, int N4, int N8, int N4p, int N8p, int nt4,
                         int ntiles, int S, __half *__restrict__ Y, float *__restrict__ ws_part,
                         int *__restrict__ ws_cnt, int32_t *__restrict__ Pd) {
-  using C = SmallMCfg<MP>;
+  using C = SmallMCfg<MP, DUO>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
@@ -283,7 +295,7 @@ __global__ void __launch_bounds__(kSmThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp < 4) {
-    regs_dec<kSmRegsCtl>();
+    regs_dec<C::kRegsCtl>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -368,7 +380,7 @@ __global__ void __launch_bounds__(kSmThreads, 1)
     if (lane == 0) mbar_arrive(tabready);
   }
   } else if (warp < 12) {
-    regs_dec<kSmRegsUnpack>();
+    regs_dec<C::kRegsUnpack>();
     // ------------------------------------------------------------ 4-bit unpack
     // Warps 4 + q and 8 + q both write TMEM lane quadrant q and take alternate
     // groups.  Thread `lane` unpacks weight row rr = 32q + lane of the tile
@@ -480,7 +492,7 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       }
     }
   } else {
-    regs_inc<kSmRegsEpi>();
+    regs_inc<C::kRegsEpi>();
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;        // TMEM lane quadrant: channels q*32 .. q*32+31 of the tile
     const int c = q * 32 + lane;   // this thread's channel in the tile
@@ -677,6 +689,10 @@ SmallMPlan plan_small_m(int64_t M, int64_t N4, int64_t N8, int64_t K, int force 
     int S = tiles > 0 ? kSmWave / tiles : 1;
     if (S < 1) S = 1;
     p.splits = p.splits8 = clamp_s(S);
+    // 16 tokens with CTAs for most of two per SM: two CTAs per SM (measured
+    // on B200: 8B gate_up 30.9 -> 25.1 us, 70B gate_up 112 -> 84 us; with
+    // one CTA per SM, on q_proj and 8B down, the shallower ring lost 20-50 %)
+    p.duo = p.mp == 16 && static_cast<int64_t>(tiles) * p.splits >= 3 * kSmWave / 2;
   }
   const int smax = p.splits > p.splits8 ? p.splits : p.splits8;
   p.part_floats = smax > 1 ? static_cast<size_t>(smax) * tiles * p.mp * 128 : 0;
@@ -684,10 +700,10 @@ SmallMPlan plan_small_m(int64_t M, int64_t N4, int64_t N8, int64_t K, int force 
   return p;
 }
 
-template <int MP, bool DBG = false>
+template <int MP, bool DBG = false, bool DUO = false>
 static cudaError_t launch_small_m_mp(const GemmArgs &a, const SmallMPlan &p, void *ws, cudaStream_t stream,
                                      const char **msg) {
-  using C = SmallMCfg<MP>;
+  using C = SmallMCfg<MP, DUO>;
   auto enc = get_encode_fn();
   if (!enc) {
     *msg = "cuTensorMapEncodeTiled is not available from the driver";
@@ -716,7 +732,7 @@ static cudaError_t launch_small_m_mp(const GemmArgs &a, const SmallMPlan &p, voi
     *msg = "too many tiles";
     return cudaErrorInvalidValue;
   }
-  auto kern = gemm_small_m_kernel<MP, DBG>;
+  auto kern = gemm_small_m_kernel<MP, DBG, DUO>;
   int dev = 0;
   cudaGetDevice(&dev);
   static std::atomic<unsigned long long> configured{0};  // one bit per device ordinal
@@ -956,7 +972,8 @@ cudaError_t launch_small_m_debug_partials(const GemmArgs &a, int kind, void *ws,
     if (p.mp == 4) return launch_gemv_mt<4, false, true>(a, p, ws, stream, msg);
     return launch_gemv_mt<8, false, true>(a, p, ws, stream, msg);
   }
-  if (p.mp == 16) return launch_small_m_mp<16, true>(a, p, ws, stream, msg);
+  if (p.mp == 16)
+    return p.duo ? launch_small_m_mp<16, true, true>(a, p, ws, stream, msg) : launch_small_m_mp<16, true>(a, p, ws, stream, msg);
   if (p.mp == 32) return launch_small_m_mp<32, true>(a, p, ws, stream, msg);
   return launch_small_m_mp<64, true>(a, p, ws, stream, msg);
 }
@@ -984,7 +1001,8 @@ cudaError_t launch_gemm_small_m(const GemmArgs &a, void *ws, size_t ws_bytes, cu
     if (p.mp == 4) return launch_gemv_mt<4>(a, p, ws, stream, msg);
     return launch_gemv_mt<8>(a, p, ws, stream, msg);
   }
-  if (p.mp == 16) return launch_small_m_mp<16>(a, p, ws, stream, msg);
+  if (p.mp == 16)
+    return p.duo ? launch_small_m_mp<16, false, true>(a, p, ws, stream, msg) : launch_small_m_mp<16>(a, p, ws, stream, msg);
   if (p.mp == 32) return launch_small_m_mp<32>(a, p, ws, stream, msg);
   return launch_small_m_mp<64>(a, p, ws, stream, msg);
 }

@@ -168,6 +168,9 @@ DEBUG_CASES = [
     ("tensor-core split-K", _layer("dbg_tc_m32", 32, 640, 2048, 64)),
     ("tensor-core split-K", _layer("dbg_tc_m64_p0", 64, 512, 512, 0)),
     ("tensor-core split-K", wl.Q_PROJ_P10.with_m(40)),
+    # 224 tiles of 16 tokens: the two-CTAs-per-SM form
+    ("tensor-core split-K", _layer("dbg_tc_m16_wide", 16, 28672, 256, 2800)),
+    ("tensor-core split-K", _layer("dbg_tc_m11_wide", 11, 28672, 384, 2800)),
 ]
 
 

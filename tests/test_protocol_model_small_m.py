@@ -38,8 +38,9 @@ def kernel_constants():
         "kGpc8": num(r"kGpc4 = \d+, kGpc8 = (\d+);"),
         "kChunkWBytes": num(r"constexpr int kChunkWBytes = (\d+);"),
         "kUnpackWarps": num(r"constexpr int kSmUnpackWarps = (\d+);"),
-        "kRingTmem": num(r"kRingBytes = kTmemW \? (\d+) \* 1024") * 1024,
-        "kRingSmem": num(r"kRingBytes = kTmemW \? \d+ \* 1024 : (\d+) \* 1024") * 1024,
+        "kRingDuo": num(r"kRingBytes = DUO \? (\d+) \* 1024") * 1024,
+        "kRingTmem": num(r"kTmemW \? (\d+) \* 1024 : \d+ \* 1024\)") * 1024,
+        "kRingSmem": num(r"kTmemW \? \d+ \* 1024 : (\d+) \* 1024\)") * 1024,
     }
     assert "static constexpr int kDone = kMaxStages;" in text
     assert "static constexpr bool kTmemW = MP <= 32;" in text
@@ -48,19 +49,19 @@ def kernel_constants():
     return c
 
 
-def stages_for(c, MP):
-    ring = c["kRingTmem"] if MP <= 32 else c["kRingSmem"]
+def stages_for(c, MP, duo=False):
+    ring = c["kRingDuo"] if duo else (c["kRingTmem"] if MP <= 32 else c["kRingSmem"])
     stage = c["kChunkWBytes"] + c["kGpc4"] * MP * 128
     return min(ring // stage, c["kMaxStages"]) & ~1
 
 
 class SmallMModel:
-    def __init__(self, ng, is4, MP, c, rng, nst=None):
+    def __init__(self, ng, is4, MP, c, rng, nst=None, duo=False):
         self.ng, self.is4, self.MP, self.c, self.rng = ng, is4, MP, c, rng
         self.tmem = MP <= 32
         self.gpc = c["kGpc4"] if is4 else c["kGpc8"]
         self.nch = (ng + self.gpc - 1) // self.gpc
-        self.nst = nst if nst is not None else stages_for(c, MP)
+        self.nst = nst if nst is not None else stages_for(c, MP, duo)
         assert self.nst >= 1
         uw = c["kUnpackWarps"]
         self.full = [Bar(f"full[{s}]", 1) for s in range(c["kMaxStages"])]
@@ -216,6 +217,17 @@ def test_small_m_protocol_holds_under_random_interleavings(ng, is4, MP):
     c = kernel_constants()
     for seed in range(25):
         SmallMModel(ng, is4, MP, c, random.Random(seed * 100 + ng)).run()
+
+
+@pytest.mark.parametrize("is4", [True, False], ids=["4bit", "8bit"])
+@pytest.mark.parametrize("ng", [1, 2, 3, 5, 8, 13, 32])
+def test_two_ctas_per_sm_form_of_16_tokens(ng, is4):
+    """The 16-token form that shares an SM with a second CTA: its shallower
+    ring (two stages) under the same protocol."""
+    c = kernel_constants()
+    assert stages_for(c, 16, duo=True) == 2
+    for seed in range(25):
+        SmallMModel(ng, is4, 16, c, random.Random(seed * 100 + ng), duo=True).run()
 
 
 @pytest.mark.parametrize("nst", [1, 3, 5])
