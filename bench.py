@@ -57,6 +57,10 @@ def parse():
     ap.add_argument("--i2f", choices=["bias", "plain"], default="bias",
                     help="tiled GEMM's int32->float step: the 0x4b400000 bias trick (the method) or, as the "
                          "ablation of the fast-I2F design point, a plain convert per element (same Y)")
+    ap.add_argument("--step", choices=["split", "fused"], default="split",
+                    help="M > 64: split = quantize_act, then the GEMM as its programmatic dependent "
+                         "(mixllm_linear's form); fused = one launch of the tiled GEMM that quantizes X "
+                         "itself (mixllm_linear_one_launch); each line also times the other form")
     ap.add_argument("--dry-run", action="store_true",
                     help="argument and rank plumbing only (gloo on CPU, no kernels): rank 0 prints the "
                          "configuration, every rank's batch seed and the max over ranks of a stand-in time")
@@ -288,9 +292,23 @@ def run_ours(args, layer, rank, world, local_rank):
         def gemm(i=0):
             mx.gemm_w4w8a8_into(A_q, s_a, p, Y, stream)
 
-    def step(i=0):
+    def split_step(i=0):
         mx.quantize_act_into(Xd, A_q, s_a, stream)
         gemm(i)
+
+    # M > 64: the tiled GEMM that quantizes X itself (one launch) when asked
+    # for; the line times the other form too (not with the plain-convert ablation)
+    one_ok = not small and args.i2f != "plain" and layer.G % 4 == 0
+    fused = one_ok and args.step == "fused"
+    if one_ok:
+        ws_lin = mx.linear_workspace(layer.M, p, dev)
+
+        def one_step(i=0):
+            mx.linear_into(Xd, p, Y, ws_lin, stream, one_launch=True)
+
+        for _ in range(3):
+            one_step()
+    step = one_step if fused else split_step
 
     for i in range(max(args.warmup, 3)):
         if not small:
@@ -374,9 +392,10 @@ def run_ours(args, layer, rank, world, local_rank):
         mx.sync_status(stream)
         t_step = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / K, world)
 
-        # Per-kernel durations for the roofline: the same steps with an event
-        # between the two kernels (which also keeps the GEMM from starting early,
-        # so this is its stand-alone duration).
+        # Per-kernel durations for the roofline: the split form's two kernels
+        # with an event between them (which also keeps the GEMM from starting
+        # early, so this is its stand-alone duration), and the split step as
+        # the timed region runs it.
         Kk = min(K, 500)
         ek = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(Kk)]
         torch.cuda.synchronize()
@@ -393,6 +412,44 @@ def run_ours(args, layer, rank, world, local_rank):
         t_gemm = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ek) / Kk, world)
         t_quant = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ek) / Kk, world)
         gemm_timed = f"{Kk} launches with an event before and after each, L2 flushed before each"
+        other = None
+        if one_ok and not fused:
+            eo = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Kk)]
+            torch.cuda.synchronize()
+            for i in range(Kk):
+                flush.fill_(i & 0xFF)
+                eo[i][0].record(stream)
+                one_step()
+                eo[i][1].record(stream)
+            torch.cuda.synchronize()
+            barrier(world)
+            mx.sync_status(stream)
+            t_one = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in eo) / Kk, world)
+            other = {"one_launch_step": {
+                "ms": t_one, "tops": layer.ops() / (t_one * 1e-3) / 1e12,
+                "timed": f"{Kk} launches of the GEMM that quantizes X itself (mixllm_linear_one_launch), "
+                         "L2 flushed before each"}}
+        if fused:
+            # the fused step is one kernel: the timed steps are its launches
+            t_split_gemm = t_gemm
+            es = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Kk)]
+            torch.cuda.synchronize()
+            for i in range(Kk):
+                flush.fill_(i & 0xFF)
+                es[i][0].record(stream)
+                split_step()
+                es[i][1].record(stream)
+            torch.cuda.synchronize()
+            barrier(world)
+            mx.sync_status(stream)
+            t_split = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in es) / Kk, world)
+            other = {"split_step": {"step_ms": t_split, "step_tops": layer.ops() / (t_split * 1e-3) / 1e12,
+                     "gemm_ms": t_split_gemm, "quantize_act_ms": t_quant,
+                     "timed": f"{Kk} split steps (quantize_act, then the GEMM as its programmatic dependent), "
+                              "L2 flushed before each; the two kernels apart as in quantize_act_kernel"}}
+            t_gemm = t_step
+            gemm_timed = (f"the timed steps: {K} launches of the GEMM that quantizes X itself, an event "
+                          "before and after each, L2 flushed before each")
 
     # end to end through the public API: pinned host X in, host Y out
     Xh = torch.from_numpy(X).pin_memory()
@@ -449,10 +506,13 @@ def run_ours(args, layer, rank, world, local_rank):
             stream.wait_event(x_ready[b])
             if i >= nslot:
                 stream.wait_event(y_free[b])
-            mx.quantize_act_into(Xds[b], A_q, s_a, stream)
-            if small:
+            if fused:
+                mx.linear_into(Xds[b], wsets[i % len(wsets)], Yds[b], ws_lin, stream, one_launch=True)
+            elif small:
+                mx.quantize_act_into(Xds[b], A_q, s_a, stream)
                 mx.gemm_w4w8a8_small_m_into(A_q, s_a, wsets[i % len(wsets)], Yds[b], ws, stream)
             else:
+                mx.quantize_act_into(Xds[b], A_q, s_a, stream)
                 (mx.gemm_w4w8a8_plain_i2f_into if args.i2f == "plain" else mx.gemm_w4w8a8_into)(
                     A_q, s_a, wsets[i % len(wsets)], Yds[b], stream)
             x_free[b].record(stream)
@@ -525,27 +585,35 @@ def run_ours(args, layer, rank, world, local_rank):
             "columns, N(0,0.02) W, random 8-bit channel set)",
             "config": dict(config_of(layer, world, len(copies) if small else 0),
                            **({"i2f": "plain int->float convert (ablation)"} if args.i2f == "plain" and not small else {})),
-            "gemm_kernel": {"path": mx.small_m_kernel(layer.M, layer.K, p.N4, p.N8) if small else "tiled",
+            "gemm_kernel": {"path": mx.small_m_kernel(layer.M, layer.K, p.N4, p.N8) if small else
+                            ("tiled, quantizing X itself" if fused else "tiled"),
                             "ms": t_gemm, "tops": gemm_tops,
                             "frac_of_int8_peak": gemm_tops / int8_peak,
                             "frac_of_nominal_4500": gemm_tops / 4500.0,
                             "timed": gemm_timed},
             "quantize_act_kernel": {"ms": t_quant,
-                                    "gbs": (layer.M * layer.K * 3 + layer.M * layer.G * 4) / (t_quant * 1e-3) / 1e9},
+                                    "gbs": (layer.M * layer.K * 3 + layer.M * layer.G * 4) / (t_quant * 1e-3) / 1e9,
+                                    **({"note": "stand-alone quantizer of the split form, not in the fused step"}
+                                       if fused else {})},
+            **(other or {}),
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": {"value": ops * world / (t_e2e * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": layer.M * layer.K * 2, "d2h_bytes_per_step": layer.M * layer.N * 2,
                     "ms_per_step": t_e2e,
-                    "timed": f"{Ke} steps pipelined: X in on one copy stream, quantize + GEMM, Y out on "
+                    "timed": f"{Ke} steps pipelined: X in on one copy stream, "
+                             f"{'the fused GEMM' if fused else 'quantize + GEMM'}, Y out on "
                              f"another, two slots; weights cycled over {len(wsets)} copies",
                     "serial": {"value": ops * world / (t_e2e_serial * 1e-3) / 1e12, "ms_per_step": t_e2e_serial,
                                "timed": "copy in, compute, copy out on one stream, L2 flushed before each step"}},
-            "gpu_launches": 2 * K,
-            "step": "quantize_act then the fused GEMM, launched as its programmatic dependent (its "
-                    "prologue overlaps the quantizer's tail; it reads A_q and s_a only after the quantizer ends)"
-                    + ("; M <= 8 runs the GEMV, 9 <= M <= 64 the few-token tensor-core kernel (both split-K)"
-                       if small else ""),
+            "gpu_launches": K if fused else 2 * K,
+            "step": ("one launch of the fused GEMM that quantizes X itself: every CTA quantizes an even "
+                     "share of the (token, group) pairs into the workspace, then loads A_q and s_a once "
+                     "all shares are counted in (mixllm_linear)") if fused else
+                    ("quantize_act then the fused GEMM, launched as its programmatic dependent (its "
+                     "prologue overlaps the quantizer's tail; it reads A_q and s_a only after the quantizer ends)"
+                     + ("; M <= 8 runs the GEMV, 9 <= M <= 64 the few-token tensor-core kernel (both split-K)"
+                        if small else "")),
             "clocks": clocks.summary(),
         }
     return line

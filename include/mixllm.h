@@ -311,6 +311,64 @@ MIXLLM_API mixllm_status mixllm_linear_small_m(const void *X_f16, int64_t M, int
                                                size_t workspace_bytes, void *stream);
 
 /*
+ * The whole layer from fp16 activations for any number of tokens: the
+ * activation quantization and the fused W4.4A8 GEMM of the MLSys 2026 talk
+ * notes on MixLLM (notes.yuuk.io, §設計判断の概要 for the quantizers,
+ * §二段階逆量子化による int8 Tensor Core 活用 for the two-step GEMM).  The
+ * codes, scales and Y are bit-identical to mixllm_quantize_act followed by
+ * mixllm_gemm_w4w8a8 (M > 64) or mixllm_gemm_w4w8a8_small_m (M <= 64).
+ * For M <= 64 this is mixllm_linear_small_m.  For M > 64 the quantizer
+ * writes A_q and s_a into the workspace and the tiled GEMM runs as its
+ * programmatic dependent (its prologue and weight copies overlap the
+ * quantizer): two launches.
+ *   X_f16      device fp16 [M, K] row-major, 16-byte aligned.
+ *   workspace  device, at least mixllm_linear_workspace_bytes() bytes,
+ *              256-byte aligned, owned by the caller.  For M > 64 it holds
+ *              A_q [M, K] int8, then s_a [M, K/128] fp32, then two uint32
+ *              counters (each part 256-byte aligned).  It must be zero-filled
+ *              before its first use; every call returns the counters to zero
+ *              (A_q and s_a are scratch, left holding this call's codes), so
+ *              it stays ready.  Two calls that run at the same time must not
+ *              share one.  After MIXLLM_ERR_TIMEOUT zero it again.
+ *   workspace_bytes  its size.
+ * Other arguments: as mixllm_gemm_w4w8a8.  Asynchronous on `stream`.
+ * Errors: MIXLLM_ERR_INVALID_ARG for bad sizes, pointers or alignment, or a
+ * workspace that is too small; MIXLLM_ERR_TIMEOUT (reported by
+ * mixllm_sync_status) if a device-side wait gave up.
+ */
+MIXLLM_API mixllm_status mixllm_linear_workspace_bytes(int64_t M, int64_t K, int64_t N4, int64_t N8, size_t *bytes);
+MIXLLM_API mixllm_status mixllm_linear(const void *X_f16, int64_t M, int64_t K, const uint8_t *W4, const uint8_t *z4,
+                                       const void *s_w4_f16, const int32_t *idx4, int64_t N4, const int8_t *W8,
+                                       const void *s_w8_f16, const int32_t *idx8, int64_t N8, void *Y_f16,
+                                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * mixllm_linear for M > 64 as ONE launch: the tiled GEMM quantizes X itself
+ * (the pages' two steps with no A_q pass between kernels: MLSys 2026 talk
+ * notes on MixLLM, §二段階逆量子化による int8 Tensor Core 活用; the
+ * awesome-system-papers summary, 核心方法).  Every CTA first quantizes an even
+ * share of the (token, group) pairs into the workspace, with all of its
+ * threads and the quantizer's own arithmetic, and adds its count to a
+ * counter there; each CTA loads A_q and s_a only once the count is
+ * complete, and the last CTA to finish returns the counters to zero.
+ * Same result, bit for bit, as mixllm_linear.  The quantization then runs
+ * at one CTA per SM on the GEMM's critical path, which on B200 costs more
+ * than the separate quantizer whose tail the GEMM's prologue overlaps; the
+ * entry point is kept to measure that choice.
+ * Arguments, workspace and errors: as mixllm_linear, plus
+ * MIXLLM_ERR_INVALID_ARG for 1 <= M <= 64 and MIXLLM_ERR_UNSUPPORTED when
+ * K / 128 is not a multiple of 4 or M * K / 128 reaches 2^31.  All of the
+ * grid's CTAs must be resident at once (one per SM, at most one per SM of
+ * the device); a device-side wait that gives up is reported by
+ * mixllm_sync_status as MIXLLM_ERR_TIMEOUT.
+ */
+MIXLLM_API mixllm_status mixllm_linear_one_launch(const void *X_f16, int64_t M, int64_t K, const uint8_t *W4,
+                                                  const uint8_t *z4, const void *s_w4_f16, const int32_t *idx4,
+                                                  int64_t N4, const int8_t *W8, const void *s_w8_f16,
+                                                  const int32_t *idx8, int64_t N8, void *Y_f16, void *workspace,
+                                                  size_t workspace_bytes, void *stream);
+
+/*
  * mixllm_gemm_w4w8a8_small_m without a workspace argument and without any
  * allocation: the split partial sums and tile counters live in a fixed 8 MiB
  * scratch array in the library's static device memory (one per device,

@@ -20,8 +20,10 @@ from ._lib import (  # noqa: F401
     gemm_w4w8a8_small_m_noalloc_into,
     gemm_w4w8a8_small_m_into,
     linear,
+    linear_into,
     linear_small_m_into,
     linear_small_m_workspace,
+    linear_workspace,
     load,
     pack_weights,
     pack_weights_host,

@@ -43,6 +43,11 @@ SIGNATURES = {
     "mixllm_linear_small_m_workspace_bytes": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(ctypes.c_size_t)]),
     "mixllm_linear_small_m": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64,
                                              _vp, _vp, ctypes.c_size_t, _vp]),
+    "mixllm_linear_workspace_bytes": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.POINTER(ctypes.c_size_t)]),
+    "mixllm_linear": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64,
+                                     _vp, _vp, ctypes.c_size_t, _vp]),
+    "mixllm_linear_one_launch": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64,
+                                                _vp, _vp, ctypes.c_size_t, _vp]),
     "mixllm_select_top_t_workspace_bytes": (ctypes.c_int, [_i64, ctypes.POINTER(ctypes.c_size_t)]),
     "mixllm_select_top_t": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, ctypes.c_size_t, _vp]),
     "mixllm_gemm_w4w8a8_small_m": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64,
@@ -300,6 +305,31 @@ def linear_small_m_into(X, p: PackedLinear, Y, workspace: torch.Tensor, stream=N
                                         workspace.numel(), _stream(stream)), "mixllm_linear_small_m")
 
 
+def linear_workspace(M: int, p: PackedLinear, device) -> torch.Tensor:
+    """A zero-filled workspace for mixllm_linear (every call leaves its
+    counters at zero, so it can be reused by calls that do not overlap)."""
+    out = ctypes.c_size_t(0)
+    _check(load().mixllm_linear_workspace_bytes(M, p.K, p.N4, p.N8, ctypes.byref(out)),
+           "mixllm_linear_workspace_bytes")
+    return torch.zeros(max(256, out.value), dtype=torch.uint8, device=device)
+
+
+def linear_into(X, p: PackedLinear, Y, workspace: torch.Tensor, stream=None, one_launch: bool = False):
+    """The layer from fp16 X for any M, quantization included (mixllm_linear);
+    one_launch (M > 64): the tiled GEMM quantizes X itself
+    (mixllm_linear_one_launch), same result."""
+    _need_cuda(X, Y, workspace)
+    M, K = X.shape
+    _require(K == p.K and tuple(Y.shape) == (M, p.N) and Y.dtype == torch.float16 and Y.is_contiguous(),
+             "Y must be a contiguous fp16 [M, N] and X must have the layer's K")
+    _require(X.dtype == torch.float16 and X.is_contiguous() and workspace.is_contiguous(),
+             "X must be a contiguous fp16 [M, K] and the workspace contiguous")
+    fn = "mixllm_linear_one_launch" if one_launch else "mixllm_linear"
+    _check(getattr(load(), fn)(_ptr(X), M, K, _ptr(p.W4), _ptr(p.z4), _ptr(p.s_w4), _ptr(p.idx4), p.N4,
+                               _ptr(p.W8), _ptr(p.s_w8), _ptr(p.idx8), p.N8, _ptr(Y), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(stream)), fn)
+
+
 SMALL_M_KERNELS = ("tensor-core split-K", "GEMV split-K", "GEMV persistent")
 
 
@@ -371,12 +401,16 @@ def small_m_debug_partials(A_q, s_a, p: PackedLinear, kind: str, stream=None):
 
 
 def linear(X: torch.Tensor, p: PackedLinear, stream=None, workspace: torch.Tensor = None) -> torch.Tensor:
-    """The whole layer: quantize X then run the fused GEMM (the few-token
-    variant for M <= 64, with `workspace` or a fresh zero-filled one)."""
-    A_q, s_a = quantize_act(X, stream)
-    if 0 < A_q.shape[0] <= SMALL_M_MAX:
-        return gemm_w4w8a8_small_m(A_q, s_a, p, workspace, stream)
-    return gemm_w4w8a8(A_q, s_a, p, stream)
+    """The whole layer from fp16 X (mixllm_linear), with `workspace` or a
+    fresh zero-filled one."""
+    M = X.shape[0]
+    Y = torch.empty((M, p.N), dtype=torch.float16, device=X.device)
+    if M == 0:
+        return Y
+    if workspace is None:
+        workspace = linear_workspace(M, p, X.device)
+    linear_into(X, p, Y, workspace, stream)
+    return Y
 
 
 def sync_status(stream=None):

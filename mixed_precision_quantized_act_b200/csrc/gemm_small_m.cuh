@@ -934,6 +934,30 @@ cudaError_t launch_linear_small_m(const GemmArgs &a, void *ws, size_t ws_bytes, 
   return launch_gemm_small_m(q, ws, p.bytes(), stream, msg);
 }
 
+// Tiled layer workspace: A_q [M, K], s_a [M, G] fp32, then the two counters
+// of the fused quantization (each part 256-byte aligned).
+size_t linear_workspace_bytes(int64_t M, int64_t N4, int64_t N8, int64_t K) {
+  if (M <= kSmallMMaxM) return linear_small_m_workspace_bytes(M, N4, N8, K);
+  return round256(static_cast<size_t>(M * K)) + round256(static_cast<size_t>(M * (K / 128)) * 4) + 256;
+}
+
+cudaError_t launch_linear(const GemmArgs &a, void *ws, size_t ws_bytes, bool one_launch, cudaStream_t stream,
+                          const char **msg) {
+  if (a.M <= kSmallMMaxM) return launch_linear_small_m(a, ws, ws_bytes, stream, msg);
+  if (ws_bytes < linear_workspace_bytes(a.M, a.N4, a.N8, a.K) || !ws) {
+    *msg = "workspace too small for this shape";
+    return cudaErrorInvalidValue;
+  }
+  unsigned char *base = static_cast<unsigned char *>(ws);
+  const size_t aq_bytes = round256(static_cast<size_t>(a.M * a.K));
+  const size_t sa_bytes = round256(static_cast<size_t>(a.M * (a.K / 128)) * 4);
+  GemmArgs q = a;
+  q.A_q = reinterpret_cast<int8_t *>(base);
+  q.s_a = reinterpret_cast<float *>(base + aq_bytes);
+  q.qcnt = reinterpret_cast<uint32_t *>(base + aq_bytes + sa_bytes);
+  return launch_linear_tiled(q, one_launch, stream, msg);
+}
+
 bool small_m_kernel_allowed(int64_t M, int64_t N4, int64_t N8, int64_t K, int kind) {
   if (M < 1 || M > kSmallMMaxM || kind < 0 || kind > 2) return false;
   if (kind == 0) return true;

@@ -73,6 +73,7 @@
 
 #include "launch.h"
 #include "ptx_sm100.cuh"
+#include "quant.cuh"  // quant_act_8x16: the fused form quantizes with the quantizer's own arithmetic
 
 namespace mixllm {
 
@@ -249,7 +250,7 @@ struct GroupCursor {
   }
 };
 
-template <int BN, bool kDebugP, bool kCvtI2F>
+template <int BN, bool kDebugP, bool kCvtI2F, bool kFuseQ>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_w4w8a8_kernel(const __grid_constant__ CUtensorMap tmA4, const __grid_constant__ CUtensorMap tmA8,
                        const uint8_t *__restrict__ W4, const __grid_constant__ CUtensorMap tmW8,
@@ -258,7 +259,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const float *__restrict__ s_a, const __half *__restrict__ s_w4,
                        const int32_t *__restrict__ idx4, const __half *__restrict__ s_w8,
                        const int32_t *__restrict__ idx8, int M, int K, int N4, int N8, int N4p, int N8p, int mt,
-                       int T4, int T8, int c4, int c8, __half *__restrict__ Y, int32_t *__restrict__ P) {
+                       int T4, int T8, int c4, int c8, __half *__restrict__ Y, int32_t *__restrict__ P,
+                       const __half *__restrict__ X, int8_t *__restrict__ Aq_w, float *__restrict__ sa_w,
+                       uint32_t *__restrict__ qcnt) {
   using C = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -400,9 +403,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     pdl_wait();
-    for (int ci = 0; ci < S && ci < nchunks; ++ci) {
-      load_chunk(pk, ci, false, true);
-      pk.next(sched, G, CH, nch, mt, BN);
+    if constexpr (!kFuseQ) {
+      for (int ci = 0; ci < S && ci < nchunks; ++ci) {
+        load_chunk(pk, ci, false, true);
+        pk.next(sched, G, CH, nch, mt, BN);
+      }
     }
   }
   if (warp == 1) {
@@ -414,11 +419,81 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  if constexpr (kFuseQ) {
+    // The fused form quantizes the layer's activations first, with every
+    // thread of the CTA (no role has anything else to do until the A_q tiles
+    // exist; only the first stages' weight copies are in flight).  The M*G
+    // (token, group) pairs are split evenly over the grid in token-major
+    // order; a half-warp takes one pair with quant_act_8x16 -- the
+    // stand-alone quantizer's arithmetic, so A_q and s_a are bit-identical
+    // to it -- with kQB pairs' loads in flight per half-warp.  The CTA then
+    // adds its pair count to qcnt[0] (release); every CTA's producer and
+    // scale warp wait for the full count (acquire) before their first A_q or
+    // s_a load.
+    pdl_wait();  // X may be the previous kernel's output
+    const int npairs = M * G;
+    const int p0 = static_cast<int>(static_cast<int64_t>(npairs) * blockIdx.x / gridDim.x);
+    const int p1 = static_cast<int>(static_cast<int64_t>(npairs) * (blockIdx.x + 1) / gridDim.x);
+    const int hw = static_cast<int>(threadIdx.x) >> 4, lane16 = threadIdx.x & 15;
+    const unsigned qmask = 0xFFFFu << (threadIdx.x & 16);
+    constexpr int kHW = kThreads / 16, kQB = 4;
+    for (int pb = p0 + hw; pb < p1; pb += kHW * kQB) {
+      uint4 raw[kQB];
+#pragma unroll
+      for (int j = 0; j < kQB; ++j) {
+        const int p = pb + j * kHW;
+        if (p < p1) {
+          const int m = p / G, g = p - m * G;
+          raw[j] = __ldg(reinterpret_cast<const uint4 *>(X + static_cast<int64_t>(m) * K + g * kKG + lane16 * 8));
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kQB; ++j) {
+        const int p = pb + j * kHW;
+        if (p < p1) {
+          const int m = p / G, g = p - m * G;
+          uint32_t packed[2];
+          const float sq = quant_act_8x16(raw[j], qmask, packed);
+          *reinterpret_cast<uint2 *>(Aq_w + static_cast<int64_t>(m) * K + g * kKG + lane16 * 8) =
+              make_uint2(packed[0], packed[1]);
+          if (lane16 == 0) sa_w[p] = sq;  // s_a[m, g] is element m*G + g = p
+        }
+      }
+    }
+    fence_proxy_async_global();  // the codes are read by other CTAs' TMA
+    __syncthreads();
+    // the first epilogue thread publishes, and later counts the CTA done:
+    // one thread, so the publication is ordered before that count
+    if (threadIdx.x == 128 && p1 > p0) {
+      __threadfence();
+      red_release_gpu_u32(qcnt, static_cast<uint32_t>(p1 - p0));
+    }
+  }
+
   if (warp < 4) {
     regs_dec<kRegsCtl>();
     if (warp == 0) {
       // ---------------------------------------------------------- producer
-      if (lane == 0) drain_ring(produce(pk, S < nchunks ? S : nchunks));
+      if (lane == 0) {
+        const int first = S < nchunks ? S : nchunks;
+        if constexpr (kFuseQ) {
+          // the A_q tiles exist once every CTA has quantized its share
+          if (first == 0) {
+            // no tiles: nothing to load, nothing to wait for
+          } else if (wait_count_gpu(qcnt, static_cast<uint32_t>(M * G), abort_flag)) {
+            fence_proxy_async_global();
+            for (int ci = 0; ci < first; ++ci) {
+              load_chunk(pk, ci, false, true);
+              pk.next(sched, G, CH, nch, mt, BN);
+            }
+            drain_ring(produce(pk, first));
+          } else {
+            drain_ring(first);  // bounded: the token boxes of these stages were never issued
+          }
+        } else {
+          drain_ring(produce(pk, first));
+        }
+      }
     } else if (warp == 1 || warp == 3) {
       // ---------------------------------------------------------- MMA issuers
       // Two threads issue alternate groups (warp 1 the even ones, warp 3 the
@@ -526,16 +601,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(sc_raw(st) + C::kScSwBytes, &tmSa, &scfull[st], k.g0, k.m0);
         };
         ChunkCursor sk;  // next raw chunk to load (lane 0)
+        int q_ok = 1;    // fused form: s_a exists (lane 0 waited for it)
         if (lane == 0) {
           prefetch_tmap(&tmSa);
           prefetch_tmap(tmSw);
           pdl_wait();
+          if constexpr (kFuseQ) {
+            if (nsc > 0) {
+              q_ok = wait_count_gpu(qcnt, static_cast<uint32_t>(M * G), abort_flag) ? 1 : 0;
+              if (q_ok) fence_proxy_async_global();
+            }
+          }
           sk.start(sched, G, C::kScG, mt, BN);
-          for (int c = 0; c < C::kScStages && c < nsc; ++c) {
+          for (int c = 0; q_ok && c < C::kScStages && c < nsc; ++c) {
             load_sc(sk, c);
             sk.next(sched, G, C::kScG, nscc, mt, BN);
           }
         }
+        q_ok = __shfl_sync(0xFFFFFFFFu, q_ok, 0);
         __syncwarp();
         int c = 0;
         for (; c < nsc; ++c) {
@@ -560,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         // let the raw copies still in flight land before the CTA can exit
-        if (lane == 0) {
+        if (lane == 0 && q_ok) {
           const int issued = nsc < c + C::kScStages ? nsc : c + C::kScStages;
           for (int cc = (issued > C::kScStages ? issued - C::kScStages : 0); cc < issued; ++cc)
             (void)mbar_wait_drain(&scfull[cc % C::kScStages], (cc / C::kScStages) & 1, 1ll << 26);
@@ -586,8 +669,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           cp_async_commit();
         };
         pdl_wait();
-        for (int gi = 0; gi < C::kStgDist; ++gi) issue(gi);
-        for (int gi = 0; gi < total; ++gi) {
+        // fused form: every lane acquires the published s_a itself
+        const bool q_ok = !kFuseQ || total == 0 || wait_count_gpu(qcnt, static_cast<uint32_t>(M * G), abort_flag);
+        for (int gi = 0; q_ok && gi < C::kStgDist; ++gi) issue(gi);
+        for (int gi = 0; q_ok && gi < total; ++gi) {
           const int i = gi % C::kStgSlots;
           cp_async_wait<C::kStgDist - 1>();
           __syncwarp();
@@ -702,7 +787,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0)
       for (int a = 0; a < C::kAccBufs; ++a) mbar_arrive(&accempty[a]);
     pdl_wait();  // before the idx reads below
-
     float2 acc[CPT / 2];
 #pragma unroll
     for (int j = 0; j < CPT / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
@@ -831,6 +915,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tmem_ld_wait();
     tmem_st_wait();
+    if constexpr (kFuseQ) {
+      // This CTA's producer and scale warp are past their waits on qcnt[0]
+      // (its last tile drained: their loads came after those waits; a CTA
+      // without tiles does not wait), and this thread published the CTA's
+      // pairs before, so the CTA counts itself done, and the last one
+      // returns both counters to zero for the next call.
+      if (threadIdx.x == 128 && atom_add_acq_rel_gpu_u32(qcnt + 1, 1u) == gridDim.x - 1) {
+        qcnt[0] = 0u;
+        qcnt[1] = 0u;
+      }
+    }
   }
 
   tc_fence_before();
@@ -1003,7 +1098,7 @@ static void split_ctas(int64_t T4, int64_t T8, int sms, int *c4, int *c8) {
   *c8 = static_cast<int>((sms - a) < T8 ? (sms - a) : T8);
 }
 
-template <int BN, bool kDebugP, bool kCvtI2F>
+template <int BN, bool kDebugP, bool kCvtI2F, bool kFuseQ = false>
 static cudaError_t launch_gemm_bn(const GemmArgs &a, cudaStream_t stream, const char **msg) {
   using C = GemmCfg<BN>;
   auto enc = get_encode_fn();
@@ -1056,7 +1151,7 @@ static cudaError_t launch_gemm_bn(const GemmArgs &a, cudaStream_t stream, const 
   }
   int c4 = 0, c8 = 0;
   split_ctas(T4, T8, device_sm_count(), &c4, &c8);
-  auto kern = gemm_w4w8a8_kernel<BN, kDebugP, kCvtI2F>;
+  auto kern = gemm_w4w8a8_kernel<BN, kDebugP, kCvtI2F, kFuseQ>;
   int dev = 0;
   cudaGetDevice(&dev);
   static std::atomic<unsigned long long> configured{0};  // one bit per device ordinal
@@ -1086,7 +1181,9 @@ static cudaError_t launch_gemm_bn(const GemmArgs &a, cudaStream_t stream, const 
       static_cast<const __half *>(a.s_w8), a.idx8, static_cast<int>(a.M), static_cast<int>(a.K),
       static_cast<int>(a.N4), static_cast<int>(a.N8), static_cast<int>(padded_channels(a.N4)),
       static_cast<int>(padded_channels(a.N8)), static_cast<int>(mt), static_cast<int>(T4), static_cast<int>(T8), c4,
-      c8, static_cast<__half *>(a.Y), a.P);
+      c8, static_cast<__half *>(a.Y), a.P, static_cast<const __half *>(kFuseQ ? a.X : nullptr),
+      kFuseQ ? const_cast<int8_t *>(a.A_q) : nullptr, kFuseQ ? const_cast<float *>(a.s_a) : nullptr,
+      kFuseQ ? a.qcnt : nullptr);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) *msg = "launch of the fused GEMM failed";
   return e;
@@ -1099,6 +1196,36 @@ cudaError_t launch_gemm_w4w8a8(const GemmArgs &a, cudaStream_t stream, const cha
   }
   if (a.P) return launch_gemm_bn<128, true, false>(a, stream, msg);
   return launch_gemm_bn<128, false, false>(a, stream, msg);
+}
+
+// The layer from fp16 X: a.X is the input; a.A_q, a.s_a and a.qcnt point
+// into the caller's workspace (A_q [M, K], s_a [M, G] 16-byte aligned, two
+// zeroed counters).  Two launches: the stand-alone quantizer into the
+// workspace, then the GEMM as its programmatic dependent.  one_launch: the
+// GEMM quantizes X itself (the scales must take the TMA path, G % 4 == 0,
+// and M*G must fit 32 bits).
+bool linear_tiled_fuses(int64_t M, int64_t K) {
+  const int64_t G = K / kKG;
+  return G % GemmCfg<128>::kScG == 0 && M * G <= 0x7FFFFFFF;
+}
+
+cudaError_t launch_linear_tiled(const GemmArgs &a, bool one_launch, cudaStream_t stream, const char **msg) {
+  if (one_launch) {
+    if (!linear_tiled_fuses(a.M, a.K) || (reinterpret_cast<uintptr_t>(a.s_a) & 15u) != 0) {
+      *msg = "the one-launch form takes K / 128 a multiple of 4 and M * K / 128 below 2^31";
+      return cudaErrorNotSupported;
+    }
+    return launch_gemm_bn<128, false, false, true>(a, stream, msg);
+  }
+  cudaError_t e = launch_quantize_act(a.X, a.M, a.K, const_cast<int8_t *>(a.A_q), const_cast<float *>(a.s_a), stream);
+  if (e != cudaSuccess) {
+    *msg = "launch of the activation quantizer failed";
+    return e;
+  }
+  GemmArgs q = a;
+  q.X = nullptr;
+  q.qcnt = nullptr;
+  return launch_gemm_bn<128, false, false>(q, stream, msg);
 }
 
 }  // namespace mixllm

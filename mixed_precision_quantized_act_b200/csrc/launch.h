@@ -35,11 +35,25 @@ struct GemmArgs {
   int32_t *P;  // debug partials [M, N, G] or null
   const void *X = nullptr;  // fp16 [M, K] activations: the fused few-token path quantizes them itself
   bool cvt_i2f = false;     // tiled GEMM only: plain int -> float convert instead of the bias trick (measurement)
+  uint32_t *qcnt = nullptr; // fused tiled layer: two counters in the workspace (pairs quantized, CTAs done)
 };
 
 // Returns a CUDA error, or cudaErrorNotSupported when the tensor-map encoder
 // is unavailable.  *msg receives a static description on failure.
 cudaError_t launch_gemm_w4w8a8(const GemmArgs &a, cudaStream_t stream, const char **msg);
+
+// The tiled layer from fp16 X (M > 64) into a.A_q / a.s_a (workspace): the
+// quantizer, then the GEMM; or (one_launch) the GEMM quantizing the
+// activations itself and publishing them through a.qcnt (two counters, zero
+// before the call and again after it; cudaErrorNotSupported for shapes that
+// form does not take).
+bool linear_tiled_fuses(int64_t M, int64_t K);
+cudaError_t launch_linear_tiled(const GemmArgs &a, bool one_launch, cudaStream_t stream, const char **msg);
+// Any M: the few-token layer (launch_linear_small_m) for M <= 64, else the
+// tiled one, each with its workspace layout (linear_workspace_bytes()).
+size_t linear_workspace_bytes(int64_t M, int64_t N4, int64_t N8, int64_t K);
+cudaError_t launch_linear(const GemmArgs &a, void *ws, size_t ws_bytes, bool one_launch, cudaStream_t stream,
+                          const char **msg);
 
 // Few-token variant (M <= 64): split-K over the groups with a workspace of
 // small_m_workspace_bytes() bytes: fp32 partial sums, then one int32 counter

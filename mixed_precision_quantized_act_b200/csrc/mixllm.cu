@@ -408,6 +408,67 @@ mixllm_status mixllm_linear_small_m(const void *X_f16, int64_t M, int64_t K, con
   return ok();
 }
 
+mixllm_status mixllm_linear_workspace_bytes(int64_t M, int64_t K, int64_t N4, int64_t N8, size_t *bytes) {
+  mixllm_status st = check_k(K, MIXLLM_GROUP);
+  if (st != MIXLLM_OK) return st;
+  if (!bytes) return fail(MIXLLM_ERR_INVALID_ARG, "null bytes");
+  if (M < 0) return fail(MIXLLM_ERR_INVALID_ARG, "M < 0");
+  if (N4 < 0 || N8 < 0 || N4 + N8 > 0x7FFFFFF0) return fail(MIXLLM_ERR_INVALID_ARG, "bad N4 / N8");
+  *bytes = M == 0 ? 0 : mixllm::linear_workspace_bytes(M, N4, N8, K);
+  return ok();
+}
+
+static mixllm_status linear_entry(const void *X_f16, int64_t M, int64_t K, const uint8_t *W4, const uint8_t *z4,
+                                  const void *s_w4_f16, const int32_t *idx4, int64_t N4, const int8_t *W8,
+                                  const void *s_w8_f16, const int32_t *idx8, int64_t N8, void *Y_f16,
+                                  void *workspace, size_t workspace_bytes, void *stream, bool one_launch) {
+  if (one_launch && M > 0 && M <= 64)
+    return fail(MIXLLM_ERR_INVALID_ARG, "the one-launch tiled form takes M > 64 (M = %lld)", static_cast<long long>(M));
+  if (M > 0 && M <= 64)
+    return mixllm_linear_small_m(X_f16, M, K, W4, z4, s_w4_f16, idx4, N4, W8, s_w8_f16, idx8, N8, Y_f16, workspace,
+                                 workspace_bytes, stream);
+  if (M > 0 && N4 + N8 > 0) {
+    if (!X_f16 || !Y_f16) return fail(MIXLLM_ERR_INVALID_ARG, "null X or Y");
+    if (!aligned(X_f16, 16)) return fail(MIXLLM_ERR_INVALID_ARG, "X must be 16-byte aligned");
+  }
+  bool empty = false;
+  // the weight and size checks of the GEMM (X stands in for A_q / s_a, whose checks it passes)
+  mixllm_status st = check_gemm(static_cast<const int8_t *>(X_f16), static_cast<const float *>(X_f16), M, K, W4, z4,
+                                s_w4_f16, idx4, N4, W8, s_w8_f16, idx8, N8, Y_f16, nullptr, &empty);
+  if (st != MIXLLM_OK) return st;
+  if (empty) return ok();
+  const size_t need = mixllm::linear_workspace_bytes(M, N4, N8, K);
+  if (workspace_bytes < need)
+    return fail(MIXLLM_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu this shape needs",
+                workspace_bytes, need);
+  if (!workspace || !aligned(workspace, 256))
+    return fail(MIXLLM_ERR_INVALID_ARG, "workspace must be a 256-byte aligned device buffer");
+  mixllm::GemmArgs a{nullptr, nullptr, M, K, W4, z4, s_w4_f16, idx4, N4, W8, s_w8_f16, idx8, N8, Y_f16, nullptr};
+  a.X = X_f16;
+  const char *msg = "";
+  cudaError_t e =
+      mixllm::launch_linear(a, workspace, workspace_bytes, one_launch, static_cast<cudaStream_t>(stream), &msg);
+  if (e == cudaErrorNotSupported) return fail(MIXLLM_ERR_UNSUPPORTED, "%s", msg);
+  if (e != cudaSuccess) return fail(MIXLLM_ERR_CUDA, "%s: %s", msg, cudaGetErrorString(e));
+  return ok();
+}
+
+mixllm_status mixllm_linear(const void *X_f16, int64_t M, int64_t K, const uint8_t *W4, const uint8_t *z4,
+                            const void *s_w4_f16, const int32_t *idx4, int64_t N4, const int8_t *W8,
+                            const void *s_w8_f16, const int32_t *idx8, int64_t N8, void *Y_f16, void *workspace,
+                            size_t workspace_bytes, void *stream) {
+  return linear_entry(X_f16, M, K, W4, z4, s_w4_f16, idx4, N4, W8, s_w8_f16, idx8, N8, Y_f16, workspace,
+                      workspace_bytes, stream, false);
+}
+
+mixllm_status mixllm_linear_one_launch(const void *X_f16, int64_t M, int64_t K, const uint8_t *W4, const uint8_t *z4,
+                                       const void *s_w4_f16, const int32_t *idx4, int64_t N4, const int8_t *W8,
+                                       const void *s_w8_f16, const int32_t *idx8, int64_t N8, void *Y_f16,
+                                       void *workspace, size_t workspace_bytes, void *stream) {
+  return linear_entry(X_f16, M, K, W4, z4, s_w4_f16, idx4, N4, W8, s_w8_f16, idx8, N8, Y_f16, workspace,
+                      workspace_bytes, stream, true);
+}
+
 mixllm_status mixllm_channel_salience(const float *W, int64_t N, int64_t K, const float *G, int64_t D, float *S,
                                       void *stream) {
   mixllm_status st = check_k(K, MIXLLM_GROUP);

@@ -235,6 +235,51 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Orders this thread's generic-proxy accesses of global memory with its
+// async-proxy (TMA) accesses: after plain stores that another CTA will read
+// with TMA, and before a TMA load of data another CTA wrote with plain stores.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ----------------------------------------------------------------- counters in global memory
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu_u32(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Atomic add at GPU scope with release semantics (no return value).
+__device__ __forceinline__ void red_release_gpu_u32(uint32_t *p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu_u32(uint32_t *p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// Waits (one thread) until the counter at p reaches `target`, with acquire
+// semantics.  Bounded like mbar_wait: gives up after `limit` SM clock cycles
+// (recording a timeout and setting *abort) or at once when *abort is set.
+__device__ __forceinline__ bool wait_count_gpu(const uint32_t *p, uint32_t target, volatile int *abort,
+                                               long long limit = (1ll << 32)) {
+  if (ld_acquire_gpu_u32(p) >= target) return true;
+  const long long t0 = clock64();
+  while (true) {
+    __nanosleep(100);
+    if (ld_acquire_gpu_u32(p) >= target) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > limit) {
+      *abort = 1;
+      record_status(kStatusTimeout);
+      return false;
+    }
+  }
+}
+
 // ----------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {

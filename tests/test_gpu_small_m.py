@@ -135,7 +135,7 @@ def test_small_m_wide_and_long_layers(dev, layer):
 def test_small_m_linear_dispatch_and_validation(dev):
     layer = _layer("sm_m5_ragged", 5, 300, 384, 37)
     X, W, is8, A_q, s_a, p, ws, Y = _run(dev, layer, 14)
-    Y_lin = mx.linear(torch.from_numpy(X).to(dev), p, workspace=ws)
+    Y_lin = mx.linear(torch.from_numpy(X).to(dev), p, workspace=mx.linear_workspace(layer.M, p, dev))
     mx.sync_status()
     assert torch.equal(Y.view(torch.int16), Y_lin.view(torch.int16))
     need = mx.small_m_workspace_bytes(layer.M, layer.K, p.N4, p.N8)
