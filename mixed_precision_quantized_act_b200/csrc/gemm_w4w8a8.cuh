@@ -8,7 +8,9 @@
 //     acc += float(P_g) * s_w[n,g] * s_a[m,g]      fp32
 //   then Y[m, idx[n]] = fp16(acc).
 //
-// How it runs on B200.  A tile is 128 output channels x 128 tokens.  The
+// How it runs on B200.  A tile is 128 output channels x 128 tokens (x 64
+// tokens, with four accumulators instead of two, when the layer has so few
+// tiles that even 64-token ones leave SMs idle).  The
 // weights are the MMA's A operand (the tile's channels are the TMEM lanes of
 // the accumulator) and the activations its B operand (the tokens are the
 // accumulator's columns).  The grid is persistent: CTA c of a channel set
@@ -77,7 +79,9 @@
 
 namespace mixllm {
 
-constexpr int kBM = 128;          // tile tokens = accumulator columns
+// Tile tokens = accumulator columns: 128, or 64 when even 64-token tiles
+// leave SMs idle (see gemm_tile_m).
+constexpr int kBM = 128;
 constexpr int kKG = 128;          // K per group = K per pipeline stage
 // Epilogue warps: 16 (32 token columns each, 24 warps in all) or, with
 // MIXLLM_EPI_WARPS=8, 8 (64 columns each, 16 warps, twice the registers).
@@ -100,10 +104,11 @@ constexpr int kRegsEpi = kEpiWarps == 16 ? 96 : 184;
 static_assert(128 * (kRegsCtl + kRegsXform) + kEpiThreads * kRegsEpi <= kThreads * kRegsLaunch, "register split");
 static_assert(kThreads * kRegsLaunch <= 65536, "register file");
 
-template <int BN>
+template <int BN, int BM = kBM>
 struct GemmCfg {
   static_assert(BN == 128, "the warp roles below are laid out for BN = 128");
-  static constexpr int kABytes = kBM * kKG;        // 16 KB A_q tile of one group
+  static_assert(BM == 128 || BM == 64, "token tile");
+  static constexpr int kABytes = BM * kKG;         // 16 (8) KB A_q tile of one group
   static constexpr int kW8Bytes = BN * kKG;        // 16 KB int8 weight tile of one group
   static constexpr int kW4Bytes = BN * kKG / 2;    //  8 KB packed uint4 weight tile of one group
   static constexpr int kZBytes = BN / 2;           // zero points of one group, two per byte
@@ -117,8 +122,8 @@ struct GemmCfg {
   // bound a group at that time.
   static constexpr int kC4 = 4, kC8 = 3;  // groups per chunk: 4-bit, 8-bit tiles
   static constexpr int kStages = 2;
-  static constexpr int kStage4 = kC4 * (kABytes + kW4Bytes);  // 96 KiB
-  static constexpr int kStage8 = kC8 * (kABytes + kW8Bytes);  // 96 KiB
+  static constexpr int kStage4 = kC4 * (kABytes + kW4Bytes);  // 96 KiB (64 KiB at BM = 64)
+  static constexpr int kStage8 = kC8 * (kABytes + kW8Bytes);  // 96 KiB (72 KiB at BM = 64)
   static constexpr int kRingBytes = kStages * (kStage4 > kStage8 ? kStage4 : kStage8);
   static constexpr int kTBufs = 8;   // unpacked 4-bit tiles in TMEM, 32 columns each
   // Two threads issue the MMAs of alternate groups.  A barrier waited by one
@@ -131,30 +136,31 @@ struct GemmCfg {
   // ring behind as long as kDone covers every ring released through it.
   static constexpr int kDone = 8;
   static_assert(kDone >= kStages * kC4 && kDone >= kStages * kC8 && kDone >= kTBufs, "done ring");
-  static constexpr int kAccBufs = 2;
+  // TMEM accumulators: two of 128 columns, or four of 64 (the same columns)
+  static constexpr int kAccBufs = BM == 128 ? 2 : 4;
   // The scale table: a slot holds kTabG consecutive groups, so the epilogue
   // waits for it, and releases it, once per kTabG groups.
   static constexpr int kTabG = 4, kTabSlots = 2;
-  // tensor memory: kAccBufs int32 accumulators of kBM (token) columns, then
+  // tensor memory: kAccBufs int32 accumulators of BM (token) columns, then
   // the unpacked weight tiles, 128 bytes of K per lane = 32 columns each
-  static constexpr int kTmemABase = kAccBufs * kBM;
+  static constexpr int kTmemABase = kAccBufs * BM;
   static constexpr int kTmemABufCols = kKG / 4;
   static constexpr int kTmemCols = 512;
   static_assert(kTmemABase + kTBufs * kTmemABufCols <= kTmemCols, "tensor memory");
-  static constexpr int kColsPerThread = BN * kBM / kEpiThreads;  // token columns per epilogue thread
+  static constexpr int kColsPerThread = BN * BM / kEpiThreads;  // token columns per epilogue thread
   static_assert(kColsPerThread % 32 == 0, "the preset fills 32 columns at a time, the drain loads 16");
   static constexpr int kTabWBytes = BN * 16;                      // {s_w, s_w, cb, cb} per channel
-  static constexpr int kTabBytes = kTabWBytes + kBM * 4;          // + s_a of the tile's tokens (one group)
+  static constexpr int kTabBytes = kTabWBytes + BM * 4;           // + s_a of the tile's tokens (one group)
   static constexpr int kTabSlotBytes = kTabG * kTabBytes;
   // Raw scales.  Vector path (G % 4 == 0, s_a 16-byte aligned): per chunk of
-  // kScG groups one 2-D box of s_w [kScG][BN] fp16 and one of s_a [kBM][kScG]
+  // kScG groups one 2-D box of s_w [kScG][BN] fp16 and one of s_a [BM][kScG]
   // fp32, into kScStages stages.  Fallback: a staging ring of kStgSlots
   // single groups filled with cp.async, kStgDist groups ahead.
   static constexpr int kScG = 4, kScStages = 3;
-  static constexpr int kScSwBytes = kScG * BN * 2, kScBytes = kScSwBytes + kBM * kScG * 4;
+  static constexpr int kScSwBytes = kScG * BN * 2, kScBytes = kScSwBytes + BM * kScG * 4;
   static constexpr int kStgSlots = 12;                            // raw scale staging ring
   static constexpr int kStgDist = 10;                             // groups prefetched ahead
-  static constexpr int kStgBytes = BN * 2 + kBM * 4;              // raw fp16 s_w + fp32 s_a
+  static constexpr int kStgBytes = BN * 2 + BM * 4;               // raw fp16 s_w + fp32 s_a
   static constexpr int kStgArea = kScStages * kScBytes > kStgSlots * kStgBytes ? kScStages * kScBytes
                                                                                 : kStgSlots * kStgBytes;
   // shared-memory layout (offsets from a 1024-byte aligned base)
@@ -203,7 +209,8 @@ struct TileSched {
 // role advances its cursors once per group or chunk).  Chunk: up to CH
 // consecutive groups of one tile, starting at group g0 of the tile and at
 // running group index gi0.
-struct ChunkCursor {
+template <int BM>
+struct ChunkCursorT {
   int tl, c, g0, ng, gi0, m0, n0;
   __device__ __forceinline__ void start(const TileSched &sc, int G, int CH, int mt, int BN) {
     tl = c = g0 = gi0 = 0;
@@ -213,7 +220,7 @@ struct ChunkCursor {
   __device__ __forceinline__ void tile(const TileSched &sc, int mt, int BN) {
     if (tl < sc.count) {
       const int t = sc.tile(tl);
-      m0 = (t % mt) * kBM;
+      m0 = (t % mt) * BM;
       n0 = (t / mt) * BN;
     }
   }
@@ -250,7 +257,7 @@ struct GroupCursor {
   }
 };
 
-template <int BN, bool kDebugP, bool kCvtI2F, bool kFuseQ>
+template <int BN, int BM, bool kDebugP, bool kCvtI2F, bool kFuseQ>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_w4w8a8_kernel(const __grid_constant__ CUtensorMap tmA4, const __grid_constant__ CUtensorMap tmA8,
                        const uint8_t *__restrict__ W4, const __grid_constant__ CUtensorMap tmW8,
@@ -262,7 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                        int T4, int T8, int c4, int c8, __half *__restrict__ Y, int32_t *__restrict__ P,
                        const __half *__restrict__ X, int8_t *__restrict__ Aq_w, float *__restrict__ sa_w,
                        uint32_t *__restrict__ qcnt) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, BM>;
+  using ChunkCursor = ChunkCursorT<BM>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
@@ -294,6 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nch = (G + CH - 1) / CH;       // chunks per tile (the last may hold fewer groups)
   const int nchunks = sched.count * nch;   // chunks this CTA loads
   const int a_bytes = CH * C::kABytes;
+  const int w8_bytes = CH * C::kW8Bytes;  // an 8-bit chunk's weight tiles (the A_q box's size only when BM = BN)
   const int stage_bytes = is4 ? C::kStage4 : C::kStage8;
   // checked builds: the shared-memory window every access must stay in
   const uint32_t smem_lo = smem_u32(smem), smem_hi = smem_lo + static_cast<uint32_t>(C::kSmemBytes);
@@ -337,12 +346,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tokens) tma_load_3d(stage_a(s), tmA, &full[s], 0, k.m0, k.g0);
     } else {
       if (!(chk_smem(smem_u32(stage_a(s)), a_bytes, smem_lo, smem_hi) &&
-            chk_smem(smem_u32(stage_w(s)), a_bytes, smem_lo, smem_hi))) {
+            chk_smem(smem_u32(stage_w(s)), w8_bytes, smem_lo, smem_hi))) {
         if (weights) mbar_arrive_expect_tx(&full[s], 0u);
         return;
       }
       if (weights) {
-        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(2 * a_bytes));
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(a_bytes + w8_bytes));
         tma_load_3d(stage_w(s), &tmW8, &full[s], 0, k.n0, k.g0);
       }
       if (tokens) tma_load_3d(stage_a(s), tmA, &full[s], 0, k.m0, k.g0);
@@ -500,10 +509,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // odd ones): one thread pays for every tcgen05.mma and commit it issues
       // and leaves the tensor pipe idle between groups, two keep it busy.
       // The weights are the MMA's A operand (BN channels = the TMEM lanes of
-      // the accumulator), the activations its B operand (kBM token columns):
+      // the accumulator), the activations its B operand (BM token columns):
       // on 4-bit tiles A comes from the unpacked buffer in tensor memory.
       if (lane == 0) {
-        constexpr uint32_t idesc = idesc_i8(BN, kBM);
+        constexpr uint32_t idesc = idesc_i8(BN, BM);
         const int who = warp == 1 ? 0 : 1;
         GroupCursor gc;
         gc.start();
@@ -517,8 +526,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&accempty[a], (gi / C::kAccBufs) & 1, abort_flag)) break;
           tc_fence_after();
           const uint32_t x_addr = smem_u32(stage_a(st) + j * C::kABytes);
-          const uint32_t d = tmem_base + static_cast<uint32_t>(a * kBM);
-          bool in_range = chk_tmem(d, tmem_base, C::kTmemCols, kBM, 128) && chk_smem(x_addr, C::kABytes, smem_lo, smem_hi);
+          const uint32_t d = tmem_base + static_cast<uint32_t>(a * BM);
+          bool in_range = chk_tmem(d, tmem_base, C::kTmemCols, BM, 128) && chk_smem(x_addr, C::kABytes, smem_lo, smem_hi);
           if (is4)
             in_range = in_range && chk_tmem(tmem_base + static_cast<uint32_t>(C::kTmemABase + b * C::kTmemABufCols),
                                             tmem_base, C::kTmemCols, C::kTmemABufCols, 128);
@@ -565,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // raw_sw: the tile's BN fp16 s_w of this group; sa_src[t * sa_stride]: s_a of token t
         if (!(chk_smem(smem_u32(table_w(gi)), C::kTabBytes, smem_lo, smem_hi) &&
               chk_smem(smem_u32(raw_sw), BN * 2, smem_lo, smem_hi) &&
-              chk_smem(smem_u32(sa_src), static_cast<uint32_t>(((kBM - 1) * sa_stride + 1) * 4), smem_lo, smem_hi)))
+              chk_smem(smem_u32(sa_src), static_cast<uint32_t>(((BM - 1) * sa_stride + 1) * 4), smem_lo, smem_hi)))
           return;  // checked build: the entry is left as it was
         const uint2 raw = *reinterpret_cast<const uint2 *>(raw_sw + 8 * lane);
         const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&raw.x));
@@ -579,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         float *tsa = table_sa(gi);
 #pragma unroll
-        for (int j = 0; j < kBM / 32; ++j) tsa[lane + 32 * j] = sa_src[(lane + 32 * j) * sa_stride];
+        for (int j = 0; j < BM / 32; ++j) tsa[lane + 32 * j] = sa_src[(lane + 32 * j) * sa_stride];
       };
       if (vec_scales) {
         // Vector path: per chunk of kScG groups of a tile, one 2-D box of s_w
@@ -660,7 +669,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int i = gi % C::kStgSlots;
             cp_async_8(stg_sw(i) + 8 * lane, s_w + static_cast<int64_t>(g) * Np + n0 + 4 * lane);
 #pragma unroll
-            for (int j = 0; j < kBM / 32; ++j) {
+            for (int j = 0; j < BM / 32; ++j) {
               const int row = lane + 32 * j;
               const bool in = m0 + row < M;
               cp_async_4(stg_sa(i) + row, s_a + (in ? static_cast<int64_t>(m0 + row) * G + g : 0), in ? 4u : 0u);
@@ -768,7 +777,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int CPT = C::kColsPerThread;
     const int e = warp - 4;                 // 0 .. kEpiWarps - 1
     const int quad = warp & 3;              // TMEM lane quadrant of this warp (= its SM sub-partition)
-    const int part = e >> 2;                // which CPT-column part of the 128 tokens
+    const int part = e >> 2;                // which CPT-column part of the tile's BM tokens
     const int ch = quad * 32 + lane;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + part * CPT;
 
@@ -780,7 +789,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int a = 0; a < C::kAccBufs; ++a)
 #pragma unroll
       for (int c = 0; c < CPT; c += 32)
-        if (chk_tmem(lane_base + a * kBM + c, tmem_base, C::kTmemCols, 32)) tmem_st_32x32b_x32_fill(lane_base + a * kBM + c, kPreset);
+        if (chk_tmem(lane_base + a * BM + c, tmem_base, C::kTmemCols, 32)) tmem_st_32x32b_x32_fill(lane_base + a * BM + c, kPreset);
     tmem_st_wait();
     tc_fence_before();
     __syncwarp();
@@ -800,12 +809,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     int gi = 0;  // running group index
     for (int tl = 0; live && tl < sched.count; ++tl) {
       const int t = sched.tile(tl);
-      const int m0 = (t % mt) * kBM;
+      const int m0 = (t % mt) * BM;
       const int n0 = (t / mt) * BN;
       const int nout = n0 + ch < Nset ? __ldg(idx + n0 + ch) : -1;  // output column of this thread's channel
       for (int g = 0; g < G; ++g, ++gi) {
         const int a = gi % C::kAccBufs, tslot = (gi / C::kTabG) % C::kTabSlots;
-        const uint32_t col = lane_base + static_cast<uint32_t>(a * kBM);
+        const uint32_t col = lane_base + static_cast<uint32_t>(a * BM);
         if (!warp_wait_u32(a_done + 8 * (gi % C::kDone), (gi / C::kDone) & 1, abort_flag)) {
           live = false;
           break;
@@ -1098,9 +1107,9 @@ static void split_ctas(int64_t T4, int64_t T8, int sms, int *c4, int *c8) {
   *c8 = static_cast<int>((sms - a) < T8 ? (sms - a) : T8);
 }
 
-template <int BN, bool kDebugP, bool kCvtI2F, bool kFuseQ = false>
-static cudaError_t launch_gemm_bn(const GemmArgs &a, cudaStream_t stream, const char **msg) {
-  using C = GemmCfg<BN>;
+template <int BN, int BM, bool kDebugP, bool kCvtI2F, bool kFuseQ = false>
+static cudaError_t launch_gemm_bm(const GemmArgs &a, cudaStream_t stream, const char **msg) {
+  using C = GemmCfg<BN, BM>;
   auto enc = get_encode_fn();
   if (!enc) {
     *msg = "cuTensorMapEncodeTiled is not available from the driver";
@@ -1113,8 +1122,8 @@ static cudaError_t launch_gemm_bn(const GemmArgs &a, cudaStream_t stream, const 
   memset(&tmZ, 0, sizeof(tmZ));
   // A_q in chunks of groups (one box per chunk and set), W8 likewise, the
   // zero points of a 4-bit chunk as one 2-D box
-  if ((a.N4 > 0 && !encode_groups_3d(enc, &tmA4, a.A_q, a.K, a.M, kBM, C::kC4)) ||
-      (a.N8 > 0 && !encode_groups_3d(enc, &tmA8, a.A_q, a.K, a.M, kBM, C::kC8))) {
+  if ((a.N4 > 0 && !encode_groups_3d(enc, &tmA4, a.A_q, a.K, a.M, BM, C::kC4)) ||
+      (a.N8 > 0 && !encode_groups_3d(enc, &tmA8, a.A_q, a.K, a.M, BM, C::kC8))) {
     *msg = "tensor map encoding of A_q failed";
     return cudaErrorInvalidValue;
   }
@@ -1135,14 +1144,14 @@ static cudaError_t launch_gemm_bn(const GemmArgs &a, cudaStream_t stream, const 
   const int64_t G = a.K / kKG;
   int vec = (G % C::kScG == 0 && (reinterpret_cast<uintptr_t>(a.s_a) & 15u) == 0) ? 1 : 0;
   if (vec) {
-    const bool ok = encode_2d(enc, &tmSa, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.s_a, G, a.M, G * 4, C::kScG, kBM) &&
+    const bool ok = encode_2d(enc, &tmSa, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.s_a, G, a.M, G * 4, C::kScG, BM) &&
                     (a.N4 == 0 || encode_2d(enc, &tmSw4, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.s_w4, padded_channels(a.N4),
                                             G, padded_channels(a.N4) * 2, BN, C::kScG)) &&
                     (a.N8 == 0 || encode_2d(enc, &tmSw8, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.s_w8, padded_channels(a.N8),
                                             G, padded_channels(a.N8) * 2, BN, C::kScG));
     if (!ok) vec = 0;
   }
-  const int64_t mt = (a.M + kBM - 1) / kBM;
+  const int64_t mt = (a.M + BM - 1) / BM;
   const int64_t T4 = mt * ((a.N4 + BN - 1) / BN);
   const int64_t T8 = mt * ((a.N8 + BN - 1) / BN);
   if (T4 + T8 > 0x7FFFFFFF || (T4 + T8) * (a.K / kKG) > 0x7FFFFFFF) {
@@ -1151,7 +1160,7 @@ static cudaError_t launch_gemm_bn(const GemmArgs &a, cudaStream_t stream, const 
   }
   int c4 = 0, c8 = 0;
   split_ctas(T4, T8, device_sm_count(), &c4, &c8);
-  auto kern = gemm_w4w8a8_kernel<BN, kDebugP, kCvtI2F, kFuseQ>;
+  auto kern = gemm_w4w8a8_kernel<BN, BM, kDebugP, kCvtI2F, kFuseQ>;
   int dev = 0;
   cudaGetDevice(&dev);
   static std::atomic<unsigned long long> configured{0};  // one bit per device ordinal
@@ -1187,6 +1196,30 @@ static cudaError_t launch_gemm_bn(const GemmArgs &a, cudaStream_t stream, const 
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) *msg = "launch of the fused GEMM failed";
   return e;
+}
+
+// The token tile: 64 when even the 64-token tiles fit one wave (at most one
+// per SM), else 128.  A group of a 128 x 64 tile costs nearly as much time
+// as one of a 128 x 128 tile (the per-group chain of barriers, MMA issue and
+// TMEM drain dominates; measured on B200: ~0.65 against ~0.69 us), so
+// halving the tile pays only where it fills SMs that would otherwise idle
+// (M = 256 at N = 4096: 66 tiles of 128 tokens, 32.5 -> 27.2 us) and costs
+// up to a third elsewhere.  MIXLLM_TILE_M (a build macro: 64 or 128) fixes
+// it instead.
+#ifndef MIXLLM_TILE_M
+#define MIXLLM_TILE_M 0
+#endif
+int gemm_tile_m(int64_t M, int64_t N4, int64_t N8) {
+  if (MIXLLM_TILE_M == 64 || MIXLLM_TILE_M == 128) return MIXLLM_TILE_M;
+  const int64_t mt = (M + kBM - 1) / kBM;
+  const int64_t tiles = mt * ((N4 + 127) / 128 + (N8 + 127) / 128);
+  return 2 * tiles <= static_cast<int64_t>(device_sm_count()) ? 64 : 128;
+}
+
+template <int BN, bool kDebugP, bool kCvtI2F, bool kFuseQ = false>
+static cudaError_t launch_gemm_bn(const GemmArgs &a, cudaStream_t stream, const char **msg) {
+  if (gemm_tile_m(a.M, a.N4, a.N8) == 64) return launch_gemm_bm<BN, 64, kDebugP, kCvtI2F, kFuseQ>(a, stream, msg);
+  return launch_gemm_bm<BN, 128, kDebugP, kCvtI2F, kFuseQ>(a, stream, msg);
 }
 
 cudaError_t launch_gemm_w4w8a8(const GemmArgs &a, cudaStream_t stream, const char **msg) {

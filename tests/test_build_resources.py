@@ -16,7 +16,10 @@ MAIN = os.path.join(ROOT, "mixed_precision_quantized_act_b200", "csrc", "mixllm.
 # spill loads in bytes allowed per kernel (mangled-name prefix -> budget); the
 # tiled GEMM and the few-token tensor-core kernel are the hot paths
 BUDGETS = [
-    ("_ZN6mixllm18gemm_w4w8a8_kernelILi128ELb0E", 0),
+    ("_ZN6mixllm18gemm_w4w8a8_kernelILi128ELi128ELb0ELb0ELb0E", 0),  # 128-token tiles
+    ("_ZN6mixllm18gemm_w4w8a8_kernelILi128ELi64ELb0ELb0ELb0E", 0),   # 64-token tiles
+    ("_ZN6mixllm18gemm_w4w8a8_kernelILi128ELi128ELb0ELb0ELb1E", 0),  # quantizing X itself
+    ("_ZN6mixllm18gemm_w4w8a8_kernelILi128ELi64ELb0ELb0ELb1E", 8),
     ("_ZN6mixllm19gemm_small_m_kernelILi16E", 0),
     ("_ZN6mixllm19gemm_small_m_kernelILi32E", 0),
     ("_ZN6mixllm19gemm_small_m_kernelILi64E", 32),

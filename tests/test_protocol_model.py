@@ -51,8 +51,12 @@ def kernel_constants():
     m = re.search(r"constexpr int kTabG = (\d+), kTabSlots = (\d+);", text)
     assert m, "kTabG / kTabSlots"
     c["kTabG"], c["kTabSlots"] = int(m.group(1)), int(m.group(2))
-    for k in ("kStages", "kTBufs", "kDone", "kAccBufs", "kXformWarps"):
+    for k in ("kStages", "kTBufs", "kDone", "kXformWarps"):
         c[k] = num(r"constexpr int %s = (\d+);" % k, k)
+    # accumulators: one count for 128-token tiles, another for 64-token ones
+    m = re.search(r"constexpr int kAccBufs = BM == 128 \? (\d+) : (\d+);", text)
+    assert m, "kAccBufs"
+    c["kAccBufs"], c["kAccBufs64"] = int(m.group(1)), int(m.group(2))
     c["kEpiWarps"] = num(r"#define MIXLLM_EPI_WARPS (\d+)", "MIXLLM_EPI_WARPS")
     return c
 
@@ -273,10 +277,13 @@ class Model:
               "not every group drained")
 
 
+@pytest.mark.parametrize("bm", [128, 64], ids=["tile128", "tile64"])
 @pytest.mark.parametrize("is4", [True, False], ids=["4bit", "8bit"])
 @pytest.mark.parametrize("G,tiles", [(1, 3), (2, 2), (3, 2), (5, 3), (7, 1), (32, 1), (32, 2), (9, 4)])
-def test_kernel_protocol_holds_under_random_interleavings(G, tiles, is4):
+def test_kernel_protocol_holds_under_random_interleavings(G, tiles, is4, bm):
     c = kernel_constants()
+    if bm == 64:
+        c = dict(c, kAccBufs=c["kAccBufs64"])
     for seed in range(30 if G * tiles < 32 else 8):
         Model(G, tiles, is4, c, random.Random(seed * 1000 + G * 10 + tiles)).run()
 
