@@ -276,6 +276,7 @@ def run_ours(args, layer, rank, world, local_rank):
 
     # few tokens (decode): the split-K path with its workspace; otherwise the tiled kernel
     small = layer.M <= mx.SMALL_M_MAX
+    other = None  # the tiled line's timing of the other M > 64 form
     copies = [p]
     if small:
         ws = mx.small_m_workspace(layer.M, p, dev)
@@ -412,7 +413,6 @@ def run_ours(args, layer, rank, world, local_rank):
         t_gemm = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ek) / Kk, world)
         t_quant = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ek) / Kk, world)
         gemm_timed = f"{Kk} launches with an event before and after each, L2 flushed before each"
-        other = None
         if one_ok and not fused:
             eo = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Kk)]
             torch.cuda.synchronize()
