@@ -176,7 +176,9 @@ MIXLLM_API mixllm_status mixllm_pack_weights_host(const float *W, int64_t N, int
  *              list every column exactly once (not checked here).
  * The weights' packed rows are padded by the caller-provided layout only in
  * the scale and zero arrays; nothing is read outside the buffers sized by
- * mixllm_packed_sizes.  Asynchronous on `stream`.
+ * mixllm_packed_sizes.  The launch picks its token tile (128, or 64 when the
+ * layer's tiles would leave SMs idle); Y's bits do not depend on it.
+ * Asynchronous on `stream`.
  */
 MIXLLM_API mixllm_status mixllm_gemm_w4w8a8(const int8_t *A_q, const float *s_a, int64_t M, int64_t K,
                                  const uint8_t *W4, const uint8_t *z4, const void *s_w4_f16,
