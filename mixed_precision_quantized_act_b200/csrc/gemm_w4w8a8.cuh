@@ -20,24 +20,27 @@
 // groups are loaded and multiplied while the epilogue still drains the last
 // tile.  Both channel sets share the launch: the first CTAs take the 4-bit
 // tiles, the others the 8-bit ones (the rings are laid out per set).
-// 24 warps, warp-specialized, registers rebalanced with setmaxnreg toward the
+// 16 warps (the default build: 8 epilogue warps; MIXLLM_EPI_WARPS=16 builds
+// 24 with 16 epilogue warps of half the columns, and the unpack warps move
+// up by 8), warp-specialized, registers rebalanced with setmaxnreg toward the
 // epilogue:
-//   warp 0      TMA producer: the A_q tile [128 x 128] (128-byte swizzle) of
+//   warp 0      TMA producer: the A_q tile [BM x 128] (128-byte swizzle) of
 //               every group -- with the int8 weight tile on 8-bit tiles --
 //               into a ring of stages; on 4-bit tiles the packed uint4 weight
 //               tile (one contiguous 8 KiB block per tile and group) and the
 //               group's zero points into a ring of their own.
 //   warps 1, 3  one thread each issues the MMAs of alternate groups: 4 x
 //               tcgen05.mma.kind::i8 (K = 32 each) into one of two int32
-//               accumulators in tensor memory (TMEM), then one commit to the
+//               accumulators in tensor memory (TMEM; four of 64 columns with
+//               64-token tiles), then one commit to the
 //               group's `done` barrier, which frees the A_q stage and the
 //               unpacked weight buffer and hands the accumulator over.
 //   warp 2      stages per group the channel scales ({s_w, s_w, -1.5*2^23*s_w,
 //               same} per channel, fp32) and the token scales s_a of the tile
 //               in a small ring the epilogue reads.
-//   warps 4-19  epilogue, four warps per TMEM lane quadrant (so four per SM
-//               sub-partition: while one waits on a TMEM load the others keep
-//               the FMA pipe busy), 32 token columns each: tcgen05.ld of the
+//   warps 4-11  epilogue, two warps per TMEM lane quadrant (so two per SM
+//               sub-partition: while one waits on a TMEM load the other keeps
+//               the FMA pipe busy), BM/2 token columns each: tcgen05.ld of the
 //               group's int32 partials, which the accumulator holds biased by
 //               0x4b400000 (TMEM is preset to the bias and refilled with it
 //               after every drain), so their bits read as float are
@@ -47,9 +50,9 @@
 //               rounding, since 1.5*2^23*s_w is exact for an fp16-valued s_w;
 //               then acc = fma(u, s_a, acc); both as f32x2 FMAs.  The running
 //               sums stay in registers; after the tile's last group each
-//               thread writes its 32 fp16 outputs straight to Y[m, idx[n]]
+//               thread writes its BM/2 fp16 outputs straight to Y[m, idx[n]]
 //               (a warp store covers 32 channels of one token row).
-//   warps 20-23 4-bit set only: unpack the nibbles and subtract the zero
+//   warps 12-15 4-bit set only: unpack the nibbles and subtract the zero
 //               point in SWAR form (four bytes per 32-bit op, no borrow
 //               between bytes) -- the B200 counterpart of the pages' vsub4
 //               pre-dequantization (§ソフトウェアパイプライン) -- and store the
