@@ -222,3 +222,42 @@ int main(void) {
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, (r.returncode, r.stderr)
     assert int(r.stdout) == _lib.packed_sizes(4096, 4096, 410)[0]
+
+
+def test_linear_workspace_plan_and_host_checks(L):
+    """Workspace of mixllm_linear / mixllm_linear_one_launch: for M > 64, A_q
+    [M, K] int8, s_a [M, K/128] fp32 and two uint32 counters, each part
+    rounded up to 256 bytes; for M <= 64 the few-token layer's own workspace.
+    The host rejects the one-launch form for 1 <= M <= 64 and null buffers
+    before touching a device; empty problems succeed without one."""
+    def ws(fn, M, K, N4, N8):
+        out = ctypes.c_size_t(0)
+        st = getattr(L, fn)(M, K, N4, N8, ctypes.byref(out))
+        return st, out.value
+
+    r256 = lambda b: (b + 255) // 256 * 256  # noqa: E731
+    for M in (65, 200, 512, 1024):
+        for K in (384, 512, 4096, 14336):
+            assert ws("mixllm_linear_workspace_bytes", M, K, 3686, 410) == (
+                _lib.OK, r256(M * K) + r256(M * (K // 128) * 4) + 256)
+    for M in (1, 2, 9, 64):
+        assert ws("mixllm_linear_workspace_bytes", M, 4096, 3686, 410) == \
+            ws("mixllm_linear_small_m_workspace_bytes", M, 4096, 3686, 410)
+    assert ws("mixllm_linear_workspace_bytes", 0, 4096, 3686, 410) == (_lib.OK, 0)
+    assert ws("mixllm_linear_workspace_bytes", 512, 100, 3686, 410)[0] == _lib.ERR_UNSUPPORTED
+    assert ws("mixllm_linear_workspace_bytes", -1, 4096, 3686, 410)[0] == _lib.ERR_INVALID_ARG
+
+    null = None
+    # (X, M, K, W4, z4, s_w4, idx4, N4, W8, s_w8, idx8, N8, Y, workspace, bytes, stream)
+    args = [null, 16, 4096, null, null, null, null, 100, null, null, null, 10, null, null, 0, null]
+    assert L.mixllm_linear_one_launch(*args) == _lib.ERR_INVALID_ARG
+    assert b"M > 64" in L.mixllm_last_error()
+    a = list(args); a[1] = 512
+    assert L.mixllm_linear(*a) == _lib.ERR_INVALID_ARG           # null X and Y
+    assert L.mixllm_linear_one_launch(*a) == _lib.ERR_INVALID_ARG
+    a = list(args); a[1] = 512; a[0] = ctypes.c_void_p(0x1008); a[12] = ctypes.c_void_p(0x3000)
+    assert L.mixllm_linear(*a) == _lib.ERR_INVALID_ARG           # X not 16-byte aligned
+    assert b"16-byte" in L.mixllm_last_error()
+    a = list(args); a[1] = 0
+    assert L.mixllm_linear(*a) == _lib.OK                        # empty: no device needed
+    assert L.mixllm_linear_one_launch(*a) == _lib.OK
